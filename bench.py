@@ -1,0 +1,550 @@
+"""Benchmark of the MoE permutation path: layout -> dispatch -> combine.
+
+One step = ep_layout + ep_dispatch + ep_combine over one synthetic batch of
+the workload "8k": T=8192 tokens, hidden 7168, top-8 of 256 experts over 8
+virtual ranks, uniform distinct routing with Dirichlet(1) weights, BF16
+dispatch and BF16 combine.  The combine input y (the expert outputs) is made
+once before timing by a stand-in expert op y = bf16(c[e] x) on the device;
+the expert op is user code, not part of the path, and is not timed.
+
+value = (dispatch bytes + combine bytes) / step time, with
+  dispatch bytes = T*2H read + T*k*rowB written (rowB = 2H, or H + 4H/128 for FP8)
+  combine bytes  = T*k*2H read + T*2H written
+summed over all ranks (each rank runs an independent replica: the path does
+not shard across GPUs here, so N GPUs run N replicas and no data crosses
+between them).  Timing: CUDA events on the launching stream around each
+step, L2 flushed (a 2x L2 write) between steps outside the events, barrier +
+synchronize around the timed region, max over ranks.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(the plain C reference) instead, on a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine GB/s & % of HBM peak; 8192x7168, top-8 of 256 experts"
+UNIT = "GB/s"
+MAIN_WORKLOAD = "8k"
+SECONDARY = ("skewed", "dsv3", "decode")
+WORKLOAD_TEXT = {
+    "8k": "8K batch: T=8192 H=7168 E=256 R=8 top-8 uniform distinct, Dirichlet(1) weights, "
+          "BF16 dispatch + BF16 combine, 128-row expert padding",
+    "skewed": "skewed: T=8192 H=7168 E=256 R=32 top-8 Zipf(1.2), FP8 e4m3 1x128 dispatch + "
+              "BF16 combine",
+    "dsv3": "DeepSeek-V3 shape: T=4096 H=7168 E=256 R=8 group-limited top-8, FP8 dispatch",
+    "decode": "decode: T=128 H=7168 E=256 R=16 group-limited top-8, FP8 dispatch",
+}
+LAUNCHES_PER_STEP = 5  # layout: count, scan, assign; dispatch; combine
+
+
+def algo_bytes(T, H, k, fmt):
+    row = 2 * H if fmt == "bf16" else H + 4 * (H // 128)
+    disp = T * 2 * H + T * k * row
+    comb = T * k * 2 * H + T * 2 * H
+    return disp, comb
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, read+write)"
+    return 6650.0, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("ep_dispatch.cu", "ep_combine.cu", "ep_layout.cu", "ep_internal.cuh"):
+        with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if it
+    was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    e = d.get("kernels", {}).get(kernel)
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during timing."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.proc = None
+        self.path = None
+        try:
+            import tempfile
+
+            fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                   "-lms", "50"]
+            if bus_id:
+                cmd += ["-i", bus_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        import datetime
+
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:9]))
+            except Exception:
+                continue
+        os.unlink(self.path)
+        inwin = [r for r in rows if t0 - 0.06 <= r[0] <= t1 + 0.06]
+        window = "timed"
+        if len(inwin) < 3:
+            inwin, window = rows, "whole run (timed region shorter than the sampling period)"
+        if not inwin:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inwin:
+            for n, v in zip(names, r[3][1:]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[1] for r in inwin),
+                "sm_max_mhz": max(r[2] for r in inwin), "reasons": sorted(reasons),
+                "samples": len(inwin), "window": window}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def gpu_setup(name, seed, dev):
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from workloads import make_workload
+
+    w = make_workload(name, seed)
+    h = ep.ep_handle_create(w.T, w.k, w.E, w.R, w.block_m, device=dev)
+    x = torch.from_numpy(w.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.from_numpy(w.topk_idx).to(dev)
+    wt = torch.from_numpy(w.topk_weights).to(dev)
+    cap = ep.ep_recv_rows_upper_bound(w.T, w.k, w.E, w.block_m)
+    if w.fmt == "bf16":
+        recv = torch.empty((cap, w.H), dtype=torch.bfloat16, device=dev)
+        scales = None
+    else:
+        recv = torch.empty((cap, w.H), dtype=torch.float8_e4m3fn, device=dev)
+        scales = torch.empty((cap, w.H // 128), dtype=torch.float32, device=dev)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+    # one untimed pass to produce y with the stand-in expert op
+    ep.ep_layout(h, idx)
+    ep.ep_dispatch(h, x, w.fmt, recv_x=recv, recv_scales=scales)
+    P = int(ep.ep_handle_view(h, "total_recv_rows").item())
+    rows = torch.arange(P, device=dev)
+    off = ep.ep_handle_view(h, "expert_off")
+    e = torch.searchsorted(off[1:].contiguous(), rows, right=True)
+    c = torch.from_numpy(w.expert_c).to(dev)[e].unsqueeze(1)
+    y = torch.empty((cap, w.H), dtype=torch.bfloat16, device=dev)
+    if scales is None:
+        y[:P] = (recv[:P].float() * c).to(torch.bfloat16)
+    else:
+        y[:P] = (recv[:P].float() * scales[:P].repeat_interleave(128, 1) * c).to(torch.bfloat16)
+    ep.ep_handle_check(h)
+    return dict(w=w, h=h, x=x, idx=idx, wt=wt, recv=recv, scales=scales, out=out, y=y, P=P)
+
+
+def gpu_step(s, ev=None):
+    import combine_ep_layout_08_b200 as ep
+
+    h, w = s["h"], s["w"]
+    if ev is not None:
+        ev[0].record()
+    ep.ep_layout(h, s["idx"])
+    if ev is not None:
+        ev[1].record()
+    ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+    if ev is not None:
+        ev[2].record()
+    ep.ep_combine(h, s["y"], s["wt"], out=s["out"])
+    if ev is not None:
+        ev[3].record()
+
+
+def time_gpu(s, steps, warmup, flush, barrier):
+    """Per-step event timing; returns dict of per-kernel and per-step ms lists."""
+    import torch
+
+    for _ in range(warmup):
+        flush()
+        gpu_step(s)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.time()
+    for i in range(steps):
+        flush()
+        gpu_step(s, evs[i])
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    lay = [e[0].elapsed_time(e[1]) for e in evs]
+    dis = [e[1].elapsed_time(e[2]) for e in evs]
+    com = [e[2].elapsed_time(e[3]) for e in evs]
+    tot = [e[0].elapsed_time(e[3]) for e in evs]
+    return dict(layout=lay, dispatch=dis, combine=com, step=tot, wall=(t0, t1))
+
+
+def time_gpu_e2e(s, steps, warmup):
+    """Same step through the public API with host buffers: pinned H2D of x,
+    topk_idx and weights, the three calls, D2H of out -- all inside the events."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+
+    w = s["w"]
+    dev = s["x"].device
+    hx = s["x"].cpu().pin_memory()
+    hidx = s["idx"].cpu().pin_memory()
+    hwt = s["wt"].cpu().pin_memory()
+    hout = torch.empty(s["out"].shape, dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(s["x"])
+    didx = torch.empty_like(s["idx"])
+    dwt = torch.empty_like(s["wt"])
+    h = s["h"]
+
+    def one():
+        dx.copy_(hx, non_blocking=True)
+        didx.copy_(hidx, non_blocking=True)
+        dwt.copy_(hwt, non_blocking=True)
+        ep.ep_layout(h, didx)
+        ep.ep_dispatch(h, dx, w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+        ep.ep_combine(h, s["y"], dwt, out=s["out"])
+        hout.copy_(s["out"], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    h2d = hx.numel() * 2 + hidx.numel() * 8 + hwt.numel() * 4
+    d2h = hout.numel() * 2
+    return statistics.mean(ts), h2d, d2h
+
+
+def graph_latency_us(s, reps=200):
+    """Decode-style latency: one CUDA graph holding layout+dispatch+combine."""
+    import torch
+
+    st = torch.cuda.Stream(device=s["x"].device)
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        gpu_step(s)
+    torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gpu_step(s)
+    for _ in range(20):
+        g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    b.synchronize()
+    us = a.elapsed_time(b) * 1000.0 / reps
+    del g
+    return us
+
+
+# ----------------------------------------------------------------- CPU arm
+
+def cpu_oracle_step(w, tokens, y_full=None):
+    """One oracle step (layout + dispatch + combine) on the first `tokens`
+    tokens; y for combine is made by the oracle's stand-in expert (untimed)."""
+    import oracle
+
+    idx = np.ascontiguousarray(w.topk_idx[:tokens])
+    xb = np.ascontiguousarray(w.x_bits[:tokens])
+    wt = np.ascontiguousarray(w.topk_weights[:tokens])
+    lay0 = oracle.layout(idx, w.E, w.R, w.block_m)
+    if w.fmt == "bf16":
+        r0 = oracle.dispatch_bf16(xb, lay0.dst_row, lay0.total_rows)
+        y = oracle.expert_scale_bf16(r0, lay0, w.expert_c)
+    else:
+        q0, s0 = oracle.dispatch_fp8(xb, lay0.dst_row, lay0.total_rows)
+        y = oracle.expert_scale_fp8(q0, s0, lay0, w.expert_c)
+    t0 = time.perf_counter()
+    lay = oracle.layout(idx, w.E, w.R, w.block_m)
+    if w.fmt == "bf16":
+        oracle.dispatch_bf16(xb, lay.dst_row, lay.total_rows)
+    else:
+        oracle.dispatch_fp8(xb, lay.dst_row, lay.total_rows)
+    oracle.combine(y, wt, lay.dst_row)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """The oracle as it stands, single-threaded, on a bounded token sample."""
+    import oracle
+
+    oracle.build()
+    probe = min(w.T, 64)
+    t = cpu_oracle_step(w, probe)
+    per_tok = t / probe
+    tokens = int(max(probe, min(w.T, budget_s / 2.0 / max(per_tok, 1e-9))))
+    reps = max(1, int(budget_s / max(per_tok * tokens, 1e-9)))
+    reps = min(reps, 5)
+    times = [cpu_oracle_step(w, tokens) for _ in range(reps)]
+    d, c = algo_bytes(tokens, w.H, w.k, w.fmt)
+    gbs = (d + c) / statistics.mean(times) / 1e9
+    return {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "first %d of %d tokens of the same workload, %d repetitions, "
+                      "single-threaded C oracle (gcc -O2), layout+dispatch+combine" % (
+                          tokens, w.T, reps)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    from workloads import make_workload
+
+    import oracle
+
+    oracle.build()
+    w = make_workload(MAIN_WORKLOAD, 0)
+    probe = 64
+    per_tok = cpu_oracle_step(w, probe) / probe
+    budget = 90.0
+    tokens = int(max(8, min(w.T, budget / max(1, args.steps + args.warmup) / per_tok)))
+    for _ in range(args.warmup):
+        cpu_oracle_step(w, tokens)
+    ts = [cpu_oracle_step(w, tokens) for _ in range(args.steps)]
+    d, c = algo_bytes(tokens, w.H, w.k, w.fmt)
+    ms = statistics.mean(ts) * 1e3
+    val = (d + c) / (ms / 1e3) / 1e9
+    line = {"metric": METRIC, "value": round(val, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens_per_step": tokens},
+            "cpu_baseline": {"value": round(val, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "first %d of %d tokens per step" % (tokens, w.T)},
+            "e2e": {"value": round(val, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- main
+
+def aggregate_max(value: float, group=None) -> float:
+    """Max over ranks (a scalar all-reduce; no data-path collective)."""
+    import torch
+    import torch.distributed as dist
+
+    if group is None and not (dist.is_available() and dist.is_initialized()):
+        return value
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from combine_ep_layout_08_b200 import _build
+
+    if rank == 0:
+        _build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    barrier()
+    props = torch.cuda.get_device_properties(dev)
+    flush_buf = torch.empty(2 * int(props.L2_cache_size), dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    peak, peak_src = load_peaks()
+    s = gpu_setup(MAIN_WORKLOAD, args.seed + rank, dev)
+    w = s["w"]
+    bus = None
+    try:
+        bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    except Exception:
+        bus = None
+    sampler = ClockSampler(bus) if rank == 0 else None
+    tm = time_gpu(s, args.steps, args.warmup, flush, barrier)
+    clocks = sampler.stop(*tm["wall"]) if sampler else None
+
+    d_bytes, c_bytes = algo_bytes(w.T, w.H, w.k, w.fmt)
+    step_ms = aggregate_max(statistics.mean(tm["step"]))
+    lay_ms = aggregate_max(statistics.mean(tm["layout"]))
+    dis_ms = aggregate_max(statistics.mean(tm["dispatch"]))
+    com_ms = aggregate_max(statistics.mean(tm["combine"]))
+    value = world * (d_bytes + c_bytes) / (step_ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_gpu_e2e(s, max(3, min(args.steps, 50)), 3)
+        e_ms = aggregate_max(e_ms)
+        e2e = {"value": round(world * (d_bytes + c_bytes) / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms, 4)}
+
+    secondary = {}
+    if not args.no_secondary:
+        del s
+        torch.cuda.empty_cache()
+        for name in SECONDARY:
+            s2 = gpu_setup(name, args.seed + rank, dev)
+            w2 = s2["w"]
+            n = max(3, min(args.steps, 100))
+            t2 = time_gpu(s2, n, min(args.warmup, 10), flush, barrier)
+            db, cb = algo_bytes(w2.T, w2.H, w2.k, w2.fmt)
+            ent = {"workload": WORKLOAD_TEXT[name],
+                   "step_us": round(statistics.mean(t2["step"]) * 1e3, 2),
+                   "layout_us": round(statistics.mean(t2["layout"]) * 1e3, 2),
+                   "dispatch_us": round(statistics.mean(t2["dispatch"]) * 1e3, 2),
+                   "combine_us": round(statistics.mean(t2["combine"]) * 1e3, 2),
+                   "dispatch_GBps": round(db / (statistics.mean(t2["dispatch"]) / 1e3) / 1e9, 1),
+                   "combine_GBps": round(cb / (statistics.mean(t2["combine"]) / 1e3) / 1e9, 1),
+                   "value_GBps": round((db + cb) / (statistics.mean(t2["step"]) / 1e3) / 1e9, 1)}
+            if name == "decode":
+                ent["graph_step_us"] = round(graph_latency_us(s2), 2)
+            secondary[name] = ent
+            del s2
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    dom = "dispatch" if dis_ms >= com_ms else "combine"
+    dom_ms = max(dis_ms, com_ms)
+    dom_bytes = d_bytes if dom == "dispatch" else c_bytes
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    kname = "dispatch_bf16_kernel" if dom == "dispatch" else "combine_kernel"
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kname),
+                "kernel": kname, "peak_source": peak_src}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens": w.T, "hidden": w.H,
+                       "experts": w.E, "virtual_ranks": w.R, "topk": w.k, "fmt": w.fmt,
+                       "parallelism": "replicas" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (write of 2x L2), outside the events",
+                       "bytes_per_step": d_bytes + c_bytes},
+            "pct_of_measured_hbm": round(value / world / peak, 4),
+            "pct_of_hbm_spec_8TBps": round(value / world / 8000.0, 4),
+            "kernels": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(dis_ms * 1e3, 2),
+                        "combine_us": round(com_ms * 1e3, 2),
+                        "dispatch_GBps": round(d_bytes / (dis_ms / 1e3) / 1e9, 1),
+                        "combine_GBps": round(c_bytes / (com_ms / 1e3) / 1e9, 1),
+                        "dispatch_p50_p95_p99_us": [round(np.percentile(tm["dispatch"], q) * 1e3, 2)
+                                                    for q in (50, 95, 99)],
+                        "combine_p50_p95_p99_us": [round(np.percentile(tm["combine"], q) * 1e3, 2)
+                                                   for q in (50, 95, 99)]},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

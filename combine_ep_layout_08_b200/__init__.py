@@ -1,0 +1,302 @@
+"""B200-native MoE expert-parallel permutation engine (dispatch layout,
+dispatch, combine) -- Python binding.
+
+This module only marshals arguments: every step runs in the CUDA kernels of
+``libep.so`` behind the C ABI of ``include/ep.h``; PyTorch supplies device
+memory and the current stream.  The function names are the C names.  There
+is no CPU fallback: if the library is missing, every call raises.
+
+Typical use::
+
+    h = ep_handle_create(max_tokens=8192, num_topk=8, num_experts=256, num_ranks=8)
+    ep_layout(h, topk_idx)                         # int64 [T, k] on the GPU
+    recv_x, recv_scales = ep_dispatch(h, x, fmt="fp8")
+    y = expert(recv_x, recv_scales)                # user code, receive layout
+    out = ep_combine(h, y, topk_weights)           # bf16 [T, H]
+    ep_handle_check(h)                             # raises on a device-side error
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
+    "ep_layout", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
+    "ep_handle_check", "ep_strerror", "library_path", "load_library",
+    "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
+    "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
+]
+
+EP_OK = 0
+EP_ERR_INVALID_ARG = 1
+EP_ERR_ALIGNMENT = 2
+EP_ERR_WORKSPACE_TOO_SMALL = 3
+EP_ERR_CAPACITY = 4
+EP_ERR_BAD_INDEX = 5
+EP_ERR_CUDA = 6
+EP_ERR_STATE = 7
+EP_ERR_NO_MEMORY = 8
+
+EP_FMT_BF16 = 0
+EP_FMT_FP8_E4M3_1X128 = 1
+_FMTS = {"bf16": EP_FMT_BF16, "fp8": EP_FMT_FP8_E4M3_1X128}
+
+VIEWS = {
+    "num_tokens_per_expert": (0, torch.int32),
+    "num_tokens_per_rank": (1, torch.int32),
+    "num_rows_per_rank": (2, torch.int32),
+    "expert_off": (3, torch.int32),
+    "rank_off": (4, torch.int32),
+    "is_token_in_rank": (5, torch.uint8),
+    "dst_row": (6, torch.int32),
+    "recv_src": (7, torch.int32),
+    "total_recv_rows": (8, torch.int32),
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libep.so")
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libep.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                "libep.so is missing at %s; build it with "
+                "`python -m combine_ep_layout_08_b200._build` (nvcc, sm_100a). "
+                "There is no CPU fallback." % _LIB_PATH)
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        sigs = {
+            "ep_workspace_bytes": ([I, I, I, I, I], SZ),
+            "ep_recv_rows_upper_bound": ([I, I, I, I], I64),
+            "ep_handle_create": ([P, SZ, I, I, I, I, I, ctypes.POINTER(P)], I),
+            "ep_handle_destroy": ([P], None),
+            "ep_layout": ([P, P, I, P], I),
+            "ep_handle_view": ([P, I, ctypes.POINTER(I64)], P),
+            "ep_handle_read_counts": ([P, P, P, P, P, P], I),
+            "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
+            "ep_combine": ([P, P, I64, P, I, P, P], I),
+            "ep_handle_check": ([P, P], I),
+            "ep_strerror": ([I], ctypes.c_char_p),
+            "ep_last_error_message": ([], ctypes.c_char_p),
+        }
+        for name, (args, res) in sigs.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+class EPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = load_library()
+        msg = lib.ep_strerror(status).decode()
+        if status == EP_ERR_CUDA:
+            msg += " -- " + lib.ep_last_error_message().decode()
+        super().__init__("%s: %s" % (where, msg))
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != EP_OK:
+        raise EPError(status, where)
+
+
+def ep_strerror(status: int) -> str:
+    return load_library().ep_strerror(status).decode()
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _on(h: "EPHandle"):
+    """Make the handle's device current for the duration of a library call."""
+    return torch.cuda.device(h.device)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() > 0 else 0)
+
+
+def ep_workspace_bytes(max_tokens: int, num_topk: int, num_experts: int, num_ranks: int,
+                       block_m: int = 128) -> int:
+    return int(load_library().ep_workspace_bytes(max_tokens, num_topk, num_experts, num_ranks,
+                                                 block_m))
+
+
+def ep_recv_rows_upper_bound(T: int, num_topk: int, num_experts: int, block_m: int = 128) -> int:
+    return int(load_library().ep_recv_rows_upper_bound(T, num_topk, num_experts, block_m))
+
+
+class EPHandle:
+    """Owns the device workspace (a torch uint8 tensor) and the C handle."""
+
+    def __init__(self, max_tokens: int, num_topk: int, num_experts: int, num_ranks: int,
+                 block_m: int = 128, device=None):
+        lib = load_library()
+        device = torch.device("cuda") if device is None else torch.device(device)
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.device = device
+        self.max_tokens, self.k, self.E, self.R, self.block_m = (
+            max_tokens, num_topk, num_experts, num_ranks, block_m)
+        nbytes = ep_workspace_bytes(max_tokens, num_topk, num_experts, num_ranks, block_m)
+        if nbytes == 0:
+            raise EPError(EP_ERR_INVALID_ARG, "ep_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        _check(lib.ep_handle_create(_ptr(self.workspace), nbytes, max_tokens, num_topk,
+                                    num_experts, num_ranks, block_m, ctypes.byref(h)),
+               "ep_handle_create")
+        self._h = h
+        self.T = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            load_library().ep_handle_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ep_handle_create(max_tokens: int, num_topk: int, num_experts: int, num_ranks: int,
+                     block_m: int = 128, device=None) -> EPHandle:
+    return EPHandle(max_tokens, num_topk, num_experts, num_ranks, block_m, device)
+
+
+def ep_layout(h: EPHandle, topk_idx: torch.Tensor) -> None:
+    """get_dispatch_layout of int64 [T, k] top-k indices (-1 = unused slot)."""
+    if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or topk_idx.shape[1] != h.k:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout: topk_idx must be int64 [T, %d]" % h.k)
+    if not topk_idx.is_cuda or not topk_idx.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout: topk_idx must be a contiguous CUDA tensor")
+    T = topk_idx.shape[0]
+    with _on(h):
+        _check(load_library().ep_layout(h.handle, _ptr(topk_idx), T, _stream(h.device)),
+               "ep_layout")
+    h.T = T
+
+
+def ep_handle_view(h: EPHandle, what: str) -> torch.Tensor:
+    """A tensor view of one layout array inside the workspace (no copy)."""
+    code, dtype = VIEWS[what]
+    n = ctypes.c_int64()
+    p = load_library().ep_handle_view(h.handle, code, ctypes.byref(n))
+    if not p:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_handle_view(%s)" % what)
+    off = p - h.workspace.data_ptr()
+    nbytes = n.value * torch.empty((), dtype=dtype).element_size()
+    v = h.workspace[off: off + nbytes].view(dtype)
+    T = h.T or 0
+    if what == "is_token_in_rank":
+        v = v.view(T, h.R)
+    elif what == "dst_row":
+        v = v.view(T, h.k)
+    return v
+
+
+def ep_handle_read_counts(h: EPHandle) -> dict:
+    """Counts of the last layout, copied to the host (synchronises the stream)."""
+    import numpy as np
+
+    a = np.zeros(h.E, np.int32)
+    b = np.zeros(h.R, np.int32)
+    c = np.zeros(h.R, np.int32)
+    d = np.zeros(1, np.int32)
+    with _on(h):
+        _check(load_library().ep_handle_read_counts(
+            h.handle, a.ctypes.data_as(ctypes.c_void_p), b.ctypes.data_as(ctypes.c_void_p),
+            c.ctypes.data_as(ctypes.c_void_p), d.ctypes.data_as(ctypes.c_void_p),
+            _stream(h.device)), "ep_handle_read_counts")
+    return dict(num_tokens_per_expert=a, num_tokens_per_rank=b, num_rows_per_rank=c,
+                total_recv_rows=int(d[0]))
+
+
+def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
+                recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
+                capacity_rows: Optional[int] = None):
+    """Scatter bf16 x [T, H] into the receive layout.  Returns (recv_x, recv_scales);
+    recv_scales is None for BF16.  Buffers not given are allocated with
+    capacity_rows rows (default: the no-sync upper bound)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != h.T or not x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: x must be contiguous bf16 [T, H]")
+    T, H = x.shape
+    f = _FMTS[fmt]
+    if recv_x is None:
+        cap = capacity_rows if capacity_rows is not None else \
+            ep_recv_rows_upper_bound(T, h.k, h.E, h.block_m)
+        dt = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
+        recv_x = torch.empty((cap, H), dtype=dt, device=x.device)
+    cap = recv_x.shape[0]
+    if f == EP_FMT_FP8_E4M3_1X128 and recv_scales is None:
+        recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+    want = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
+    if recv_x.dtype != want or recv_x.shape[1] != H or not recv_x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_x must be contiguous %s [*, %d]"
+                      % (want, H))
+    if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128:
+        if (recv_scales.dtype != torch.float32 or recv_scales.shape[0] < cap
+                or recv_scales.shape[1] != H // 128 or not recv_scales.is_contiguous()):
+            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_scales must be f32 [cap, H/128]")
+    with _on(h):
+        _check(load_library().ep_dispatch(h.handle, _ptr(x), H, f, _ptr(recv_x),
+                                          _ptr(recv_scales) if f else ctypes.c_void_p(0), cap,
+                                          _stream(h.device)), "ep_dispatch")
+    return recv_x, (recv_scales if f == EP_FMT_FP8_E4M3_1X128 else None)
+
+
+def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Weighted gather-reduce of bf16 y [rows, H] (receive layout) into bf16 [T, H]."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_combine")
+    if y.dtype != torch.bfloat16 or y.dim() != 2 or not y.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: y must be contiguous bf16 [rows, H]")
+    if (topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (h.T, h.k)
+            or not topk_weights.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: topk_weights must be f32 [T, k]")
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty((h.T, H), dtype=torch.bfloat16, device=y.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (h.T, H) or not out.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: out must be contiguous bf16 [T, H]")
+    with _on(h):
+        _check(load_library().ep_combine(h.handle, _ptr(y), y.shape[0], _ptr(topk_weights), H,
+                                         _ptr(out), _stream(h.device)), "ep_combine")
+    return out
+
+
+def ep_handle_check(h: EPHandle, raise_on_error: bool = True) -> int:
+    """Synchronise, read and clear the sticky device error word."""
+    with _on(h):
+        st = load_library().ep_handle_check(h.handle, _stream(h.device))
+    if raise_on_error:
+        _check(st, "ep_handle_check")
+    return st

@@ -1,0 +1,378 @@
+// ep_api.cu -- the C ABI declared in include/ep.h: argument checks, the
+// workspace carve, the handle, and the kernel launches.  No device memory is
+// allocated here; the handle is one small host allocation.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+ep_status_t cuda_fail(cudaError_t e, const char* where)
+{
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return EP_ERR_CUDA;
+}
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+Handle* as_handle(ep_handle_t h)
+{
+    Handle* p = reinterpret_cast<Handle*>(h);
+    return (p && p->magic == kHandleMagic) ? p : nullptr;
+}
+
+bool valid_shape(int max_tokens, int k, int E, int R, int block_m)
+{
+    if (max_tokens < 0 || k < 1 || k > EP_MAX_TOPK || E < 1 || E > EP_MAX_EXPERTS || R < 1 ||
+        R > E || E % R != 0 || block_m < 1 || block_m > EP_MAX_BLOCK_M)
+        return false;
+    // every row and entry index must fit in int32
+    const int64_t entries = (int64_t)max_tokens * k;
+    if (entries > INT32_MAX)
+        return false;
+    if (recv_rows_bound(max_tokens, k, E, block_m) > INT32_MAX)
+        return false;
+    if ((int64_t)max_tokens * R > INT64_C(1) << 40)
+        return false;
+    return true;
+}
+
+}  // namespace
+
+int64_t recv_rows_bound(int64_t T, int64_t k, int64_t E, int64_t block_m)
+{
+    const int64_t n = T * k;
+    const int64_t m = n < E ? n : E;
+    const int64_t b = n + m * (block_m - 1);
+    return b / block_m * block_m;
+}
+
+bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c)
+{
+    if (!valid_shape(max_tokens, k, E, R, block_m))
+        return false;
+    const int64_t nchunks = ((int64_t)max_tokens + kChunkTokens - 1) / kChunkTokens;
+    const int64_t rows = recv_rows_bound(max_tokens, k, E, block_m);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + (bytes ? bytes : 1));
+        return at;
+    };
+    c->chunk_counts = take(sizeof(int32_t) * (size_t)nchunks * E);
+    c->chunk_rank = take(sizeof(int32_t) * (size_t)nchunks * R);
+    c->cnt = take(sizeof(int32_t) * (size_t)E);
+    c->expert_off = take(sizeof(int32_t) * (size_t)(E + 1));
+    c->rank_off = take(sizeof(int32_t) * (size_t)(R + 1));
+    c->tokens_per_rank = take(sizeof(int32_t) * (size_t)R);
+    c->rows_per_rank = take(sizeof(int32_t) * (size_t)R);
+    c->total_rows = take(sizeof(int32_t));
+    c->err = take(sizeof(int32_t));
+    c->is_token_in_rank = take((size_t)max_tokens * R);
+    c->dst_row = take(sizeof(int32_t) * (size_t)max_tokens * k);
+    c->recv_src = take(sizeof(int32_t) * (size_t)rows);
+    c->total = off;
+    return true;
+}
+
+cudaError_t persistent_grid(const void* kernel, int block_threads, size_t dyn_smem,
+                            int max_per_sm, int* grid)
+{
+    // Cache per (kernel, device); a handful of kernels and devices at most.
+    struct Entry {
+        const void* kernel;
+        int device, grid;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+
+    int dev = 0;
+    cudaError_t rc = cudaGetDevice(&dev);
+    if (rc != cudaSuccess)
+        return rc;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].kernel == kernel && cache[i].device == dev) {
+                *grid = cache[i].grid;
+                return cudaSuccess;
+            }
+    }
+    int sms = 0, per_sm = 0;
+    if ((rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return rc;
+    if ((rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, block_threads,
+                                                            dyn_smem)) != cudaSuccess)
+        return rc;
+    if (per_sm < 1)
+        per_sm = 1;
+    if (per_sm > max_per_sm)
+        per_sm = max_per_sm;
+    *grid = sms * per_sm;
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64)
+        cache[used++] = Entry{kernel, dev, *grid};
+    return cudaSuccess;
+}
+
+}  // namespace ep
+
+using ep::Handle;
+
+extern "C" {
+
+size_t ep_workspace_bytes(int max_tokens, int num_topk, int num_experts, int num_ranks,
+                          int block_m)
+{
+    ep::Carve c;
+    if (!ep::carve_workspace(max_tokens, num_topk, num_experts, num_ranks, block_m, &c))
+        return 0;
+    return c.total;
+}
+
+int64_t ep_recv_rows_upper_bound(int T, int num_topk, int num_experts, int block_m)
+{
+    if (T < 0 || num_topk < 1 || num_experts < 1 || block_m < 1)
+        return -1;
+    return ep::recv_rows_bound(T, num_topk, num_experts, block_m);
+}
+
+ep_status_t ep_handle_create(void* workspace, size_t workspace_bytes, int max_tokens,
+                             int num_topk, int num_experts, int num_ranks, int block_m,
+                             ep_handle_t* out)
+{
+    if (!out)
+        return EP_ERR_INVALID_ARG;
+    *out = nullptr;
+    ep::Carve c;
+    if (!ep::carve_workspace(max_tokens, num_topk, num_experts, num_ranks, block_m, &c))
+        return EP_ERR_INVALID_ARG;
+    if (!workspace)
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(workspace, ep::kAlign))
+        return EP_ERR_ALIGNMENT;
+    if (workspace_bytes < c.total)
+        return EP_ERR_WORKSPACE_TOO_SMALL;
+    Handle* h = static_cast<Handle*>(calloc(1, sizeof(Handle)));
+    if (!h)
+        return EP_ERR_NO_MEMORY;
+    char* base = static_cast<char*>(workspace);
+    h->magic = ep::kHandleMagic;
+    h->max_tokens = max_tokens;
+    h->k = num_topk;
+    h->E = num_experts;
+    h->R = num_ranks;
+    h->block_m = block_m;
+    h->max_rows = ep::recv_rows_bound(max_tokens, num_topk, num_experts, block_m);
+    h->max_chunks = ((int64_t)max_tokens + ep::kChunkTokens - 1) / ep::kChunkTokens;
+    h->chunk_counts = reinterpret_cast<int32_t*>(base + c.chunk_counts);
+    h->chunk_rank = reinterpret_cast<int32_t*>(base + c.chunk_rank);
+    h->cnt = reinterpret_cast<int32_t*>(base + c.cnt);
+    h->expert_off = reinterpret_cast<int32_t*>(base + c.expert_off);
+    h->rank_off = reinterpret_cast<int32_t*>(base + c.rank_off);
+    h->tokens_per_rank = reinterpret_cast<int32_t*>(base + c.tokens_per_rank);
+    h->rows_per_rank = reinterpret_cast<int32_t*>(base + c.rows_per_rank);
+    h->total_rows = reinterpret_cast<int32_t*>(base + c.total_rows);
+    h->err = reinterpret_cast<int32_t*>(base + c.err);
+    h->is_token_in_rank = reinterpret_cast<uint8_t*>(base + c.is_token_in_rank);
+    h->dst_row = reinterpret_cast<int32_t*>(base + c.dst_row);
+    h->recv_src = reinterpret_cast<int32_t*>(base + c.recv_src);
+    h->T = -1;
+    h->has_layout = 0;
+    h->err_cleared = 0;
+    *out = reinterpret_cast<ep_handle_t>(h);
+    return EP_OK;
+}
+
+void ep_handle_destroy(ep_handle_t hh)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h)
+        return;
+    h->magic = 0;
+    free(h);
+}
+
+ep_status_t ep_layout(ep_handle_t hh, const int64_t* topk_idx, int T, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || T < 0 || T > h->max_tokens || (T > 0 && !topk_idx))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(topk_idx, 8))
+        return EP_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!h->err_cleared) {
+        // The workspace starts with unknown contents: zero the error word once.
+        cudaError_t rc = cudaMemsetAsync(h->err, 0, sizeof(int32_t), s);
+        if (rc != cudaSuccess)
+            return ep::cuda_fail(rc, "ep_layout (clear error word)");
+        h->err_cleared = 1;
+    }
+    cudaError_t rc = ep::launch_layout(*h, topk_idx, T, s);
+    if (rc != cudaSuccess) {
+        h->has_layout = 0;
+        return ep::cuda_fail(rc, "ep_layout");
+    }
+    h->T = T;
+    h->has_layout = 1;
+    return EP_OK;
+}
+
+const void* ep_handle_view(ep_handle_t hh, ep_view_t what, int64_t* count)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h)
+        return nullptr;
+    const int64_t T = h->has_layout ? h->T : 0;
+    const void* p = nullptr;
+    int64_t n = 0;
+    switch (what) {
+    case EP_VIEW_NUM_TOKENS_PER_EXPERT: p = h->cnt; n = h->E; break;
+    case EP_VIEW_NUM_TOKENS_PER_RANK: p = h->tokens_per_rank; n = h->R; break;
+    case EP_VIEW_NUM_ROWS_PER_RANK: p = h->rows_per_rank; n = h->R; break;
+    case EP_VIEW_EXPERT_OFFSET: p = h->expert_off; n = h->E + 1; break;
+    case EP_VIEW_RANK_OFFSET: p = h->rank_off; n = h->R + 1; break;
+    case EP_VIEW_IS_TOKEN_IN_RANK: p = h->is_token_in_rank; n = T * h->R; break;
+    case EP_VIEW_DST_ROW: p = h->dst_row; n = T * h->k; break;
+    case EP_VIEW_RECV_SRC: p = h->recv_src; n = h->max_rows; break;
+    case EP_VIEW_TOTAL_RECV_ROWS: p = h->total_rows; n = 1; break;
+    default: return nullptr;
+    }
+    if (count)
+        *count = n;
+    return p;
+}
+
+ep_status_t ep_handle_read_counts(ep_handle_t hh, int32_t* num_tokens_per_expert,
+                                  int32_t* num_tokens_per_rank, int32_t* num_rows_per_rank,
+                                  int32_t* total_recv_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = cudaSuccess;
+    if (num_tokens_per_expert && rc == cudaSuccess)
+        rc = cudaMemcpyAsync(num_tokens_per_expert, h->cnt, sizeof(int32_t) * h->E,
+                             cudaMemcpyDeviceToHost, s);
+    if (num_tokens_per_rank && rc == cudaSuccess)
+        rc = cudaMemcpyAsync(num_tokens_per_rank, h->tokens_per_rank, sizeof(int32_t) * h->R,
+                             cudaMemcpyDeviceToHost, s);
+    if (num_rows_per_rank && rc == cudaSuccess)
+        rc = cudaMemcpyAsync(num_rows_per_rank, h->rows_per_rank, sizeof(int32_t) * h->R,
+                             cudaMemcpyDeviceToHost, s);
+    if (total_recv_rows && rc == cudaSuccess)
+        rc = cudaMemcpyAsync(total_recv_rows, h->total_rows, sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, s);
+    if (rc == cudaSuccess)
+        rc = cudaStreamSynchronize(s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_handle_read_counts");
+}
+
+ep_status_t ep_dispatch(ep_handle_t hh, const void* x, int H, ep_fmt_t fmt, void* recv_x,
+                        float* recv_scales, int64_t recv_capacity_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || recv_capacity_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (fmt != EP_FMT_BF16 && fmt != EP_FMT_FP8_E4M3_1X128)
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_BF16 && H % 8 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_FP8_E4M3_1X128 && H % 128 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (h->T > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_FP8_E4M3_1X128 && h->T > 0 && recv_capacity_rows > 0 && !recv_scales)
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(x, 16) || !ep::aligned(recv_x, 16) || !ep::aligned(recv_scales, 16))
+        return EP_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = (fmt == EP_FMT_BF16)
+                         ? ep::launch_dispatch_bf16(*h, x, H, recv_x, recv_capacity_rows, s)
+                         : ep::launch_dispatch_fp8(*h, x, H, recv_x, recv_scales,
+                                                   recv_capacity_rows, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch");
+}
+
+ep_status_t ep_combine(ep_handle_t hh, const void* y, int64_t y_rows, const float* topk_weights,
+                       int H, void* out, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (h->T > 0 && (!out || !topk_weights || (!y && y_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(y, 16) || !ep::aligned(out, 16) || !ep::aligned(topk_weights, 4))
+        return EP_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = ep::launch_combine(*h, y, y_rows, topk_weights, H, out, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine");
+}
+
+ep_status_t ep_handle_check(ep_handle_t hh, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h)
+        return EP_ERR_INVALID_ARG;
+    if (!h->err_cleared)
+        return EP_OK;  // nothing has run on this handle yet
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t word = 0;
+    cudaError_t rc = cudaMemcpyAsync(&word, h->err, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (rc == cudaSuccess)
+        rc = cudaStreamSynchronize(s);
+    if (rc == cudaSuccess)
+        rc = cudaMemsetAsync(h->err, 0, sizeof(int32_t), s);
+    if (rc == cudaSuccess)
+        rc = cudaStreamSynchronize(s);
+    if (rc != cudaSuccess)
+        return ep::cuda_fail(rc, "ep_handle_check");
+    if (word & ep::kErrBadIndex)
+        return EP_ERR_BAD_INDEX;
+    if (word & (ep::kErrDispatchCap | ep::kErrCombineCap))
+        return EP_ERR_CAPACITY;
+    return EP_OK;
+}
+
+const char* ep_strerror(ep_status_t status)
+{
+    switch (status) {
+    case EP_OK: return "EP_OK";
+    case EP_ERR_INVALID_ARG: return "EP_ERR_INVALID_ARG: invalid argument";
+    case EP_ERR_ALIGNMENT: return "EP_ERR_ALIGNMENT: pointer misaligned";
+    case EP_ERR_WORKSPACE_TOO_SMALL: return "EP_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+    case EP_ERR_CAPACITY: return "EP_ERR_CAPACITY: receive row beyond buffer capacity";
+    case EP_ERR_BAD_INDEX: return "EP_ERR_BAD_INDEX: top-k index outside [-1, E)";
+    case EP_ERR_CUDA: return "EP_ERR_CUDA: CUDA runtime error";
+    case EP_ERR_STATE: return "EP_ERR_STATE: no layout on this handle";
+    case EP_ERR_NO_MEMORY: return "EP_ERR_NO_MEMORY: host allocation failed";
+    }
+    return "unknown ep_status_t";
+}
+
+const char* ep_last_error_message(void) { return ep::g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,166 @@
+// ep_combine.cu -- combine on sm_100a: gather of the k expert outputs of each
+// token and weighted reduction back into token order.
+//
+// Combine takes the expert outputs and routing weights and returns results
+// in the original token order ("DeepEP是什麼？MoE Dispatch、Combine、
+// All-to-all與V2架構", stage table of section "MoE為什麼需要All-to-all",
+// row Combine: reverse all-to-all plus reduction); it moves the same
+// batch x top_k x hidden x sizeof(dtype) bytes as dispatch ("DeepEP 编址服务
+// 深度对抗分析", section 五.2).  Reduction semantics (stated in ep.h): fp32
+// accumulator, one fused multiply-add per used slot in slot order
+// j = 0..k-1, round-to-nearest-even to bf16 at the end.
+//
+// HBM-bound: k row reads (k x 2H bytes) and one row write per token.  Work
+// unit: one warp x (token, 32 x U 16-byte vectors of the row).  When every
+// slot of the token is used and in range (the common case), all k x U loads
+// of a lane are issued before the first multiply-add; the chain itself is
+// still evaluated in slot order.
+#include <cuda_bf16.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kThreads = 256;
+constexpr int kU = 2;  // 16-byte vectors per lane per unit
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4& v)
+{
+    acc[0] = __fmaf_rn(w, bf16_lo(v.x), acc[0]);
+    acc[1] = __fmaf_rn(w, bf16_hi(v.x), acc[1]);
+    acc[2] = __fmaf_rn(w, bf16_lo(v.y), acc[2]);
+    acc[3] = __fmaf_rn(w, bf16_hi(v.y), acc[3]);
+    acc[4] = __fmaf_rn(w, bf16_lo(v.z), acc[4]);
+    acc[5] = __fmaf_rn(w, bf16_hi(v.z), acc[5]);
+    acc[6] = __fmaf_rn(w, bf16_lo(v.w), acc[6]);
+    acc[7] = __fmaf_rn(w, bf16_hi(v.w), acc[7]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return a | (b << 16);
+}
+
+template <int KMAX>
+__device__ __forceinline__ void combine_unit_all_valid(const uint4* __restrict__ y, int64_t vpr,
+                                                       int k, int d, float w, int64_t v0,
+                                                       float (&acc)[kU][8])
+{
+    // Issue every load first (k <= KMAX), then reduce in slot order.
+    uint4 v[KMAX][kU];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+            const int dj = __shfl_sync(kFull, d, j);
+            const uint4* row = y + (int64_t)dj * vpr;
+#pragma unroll
+            for (int i = 0; i < kU; ++i)
+                if (v0 + 32 * i < vpr)
+                    v[j][i] = __ldcs(row + v0 + 32 * i);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+            const float wj = __shfl_sync(kFull, w, j);
+#pragma unroll
+            for (int i = 0; i < kU; ++i)
+                if (v0 + 32 * i < vpr)
+                    fma8(acc[i], wj, v[j][i]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restrict__ weights,
+               int T, int k, int64_t vpr, const int32_t* __restrict__ dst_row,
+               uint4* __restrict__ out, int32_t* err)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t wg = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+    const int64_t unit_vec = 32 * kU;
+    const int64_t upr = (vpr + unit_vec - 1) / unit_vec;
+    const int64_t units = (int64_t)T * upr;
+
+    for (int64_t u = wg; u < units; u += nw) {
+        const int64_t t = u / upr;
+        const int64_t v0 = (u - t * upr) * unit_vec + lane;
+        int d = -1;
+        float w = 0.0f;
+        if (lane < k) {
+            d = __ldg(dst_row + t * k + lane);
+            w = __ldg(weights + t * k + lane);
+        }
+        if (d >= y_rows) {
+            atomicOr(err, kErrCombineCap);
+            d = -1;
+        }
+        const bool all_valid = __all_sync(kFull, lane >= k || d >= 0);
+
+        float acc[kU][8];
+#pragma unroll
+        for (int i = 0; i < kU; ++i)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
+
+        if (all_valid && k <= 8) {
+            combine_unit_all_valid<8>(y, vpr, k, d, w, v0, acc);
+        } else {
+            for (int j = 0; j < k; ++j) {
+                const int dj = __shfl_sync(kFull, d, j);
+                const float wj = __shfl_sync(kFull, w, j);
+                if (dj < 0)
+                    continue;
+                const uint4* row = y + (int64_t)dj * vpr;
+                uint4 v[kU];
+#pragma unroll
+                for (int i = 0; i < kU; ++i)
+                    if (v0 + 32 * i < vpr)
+                        v[i] = __ldcs(row + v0 + 32 * i);
+#pragma unroll
+                for (int i = 0; i < kU; ++i)
+                    if (v0 + 32 * i < vpr)
+                        fma8(acc[i], wj, v[i]);
+            }
+        }
+
+        uint4* o = out + t * vpr;
+#pragma unroll
+        for (int i = 0; i < kU; ++i)
+            if (v0 + 32 * i < vpr) {
+                uint4 r;
+                r.x = pack_bf16x2(acc[i][0], acc[i][1]);
+                r.y = pack_bf16x2(acc[i][2], acc[i][3]);
+                r.z = pack_bf16x2(acc[i][4], acc[i][5]);
+                r.w = pack_bf16x2(acc[i][6], acc[i][7]);
+                o[v0 + 32 * i] = r;
+            }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
+                           int H, void* out, cudaStream_t s)
+{
+    if (h.T == 0)
+        return cudaSuccess;
+    int grid = 0;
+    cudaError_t rc = persistent_grid((const void*)combine_kernel, kThreads, 0, 8, &grid);
+    if (rc != cudaSuccess)
+        return rc;
+    combine_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(y), y_rows, w, h.T, h.k,
+                                             (int64_t)H / 8, h.dst_row,
+                                             static_cast<uint4*>(out), h.err);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

@@ -1,0 +1,74 @@
+// ep_internal.cuh -- shared definitions of the CUDA library (not installed).
+//
+// The handle, the workspace carve, the sticky error bits and the launchers
+// each kernel file exports to the C-ABI layer (ep_api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+namespace ep {
+
+constexpr uint32_t kHandleMagic = 0x45504c38u;  // "EPL8"
+
+// Sticky device error bits (one int32 in the workspace).
+constexpr int kErrBadIndex = 1;      // top-k index outside [-1, E)
+constexpr int kErrDispatchCap = 2;   // dispatch row >= recv capacity
+constexpr int kErrCombineCap = 4;    // combine row >= y rows
+
+// The layout works on chunks of kChunkTokens consecutive tokens, one warp
+// per chunk: the (token, slot) entries of a chunk are contiguous in topk_idx.
+constexpr int kChunkTokens = 32;
+
+struct Handle {
+    uint32_t magic;
+    int max_tokens, k, E, R, block_m;
+    int64_t max_rows;  // capacity of recv_src: the padded-row bound at max_tokens
+    int64_t max_chunks;
+    // device pointers into the caller's workspace
+    int32_t* chunk_counts;   // [max_chunks][E]  per-chunk expert counts, then prefixes
+    int32_t* chunk_rank;     // [max_chunks][R]  per-chunk token-per-rank counts
+    int32_t* cnt;            // [E]
+    int32_t* expert_off;     // [E+1]
+    int32_t* rank_off;       // [R+1]
+    int32_t* tokens_per_rank;// [R]
+    int32_t* rows_per_rank;  // [R]
+    int32_t* total_rows;     // [1]
+    int32_t* err;            // [1]
+    uint8_t* is_token_in_rank;  // [max_tokens][R]
+    int32_t* dst_row;        // [max_tokens][k]
+    int32_t* recv_src;       // [max_rows]
+    // state of the last layout
+    int T;
+    int has_layout;
+    int err_cleared;  // the sticky error word has been zeroed once on the device
+};
+
+// Workspace carve: offsets of each array, 256-byte aligned.  Returns the
+// total size, or 0 if the sizes overflow.
+struct Carve {
+    size_t chunk_counts, chunk_rank, cnt, expert_off, rank_off, tokens_per_rank,
+        rows_per_rank, total_rows, err, is_token_in_rank, dst_row, recv_src, total;
+};
+
+int64_t recv_rows_bound(int64_t T, int64_t k, int64_t E, int64_t block_m);
+bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c);
+
+// Launchers (each returns the cudaError_t of its launches).
+cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s);
+cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,
+                                 int64_t cap_rows, cudaStream_t s);
+cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
+                                float* recv_scales, int64_t cap_rows, cudaStream_t s);
+cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
+                           int H, void* out, cudaStream_t s);
+
+// Persistent-grid size: min(resident blocks per SM from the occupancy API,
+// max_per_sm) x the SM count of the current device, cached per kernel and
+// device.
+cudaError_t persistent_grid(const void* kernel, int block_threads, size_t dyn_smem,
+                            int max_per_sm, int* grid);
+
+}  // namespace ep

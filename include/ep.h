@@ -1,0 +1,193 @@
+/*
+ * ep.h -- C ABI of the single-GPU MoE expert-parallel permutation engine.
+ *
+ * The engine runs the three data-parallel steps that surround the expert
+ * GEMM of a Mixture-of-Experts layer, with the expert-parallel ranks modelled
+ * as R virtual partitions of one GPU's memory:
+ *
+ *   ep_layout    routing metadata: per-expert and per-rank counts, padded
+ *                expert-major offsets, is_token_in_rank, and the receive row
+ *                of every (token, top-k slot);
+ *   ep_dispatch  scatter of each token's hidden row into the expert-major
+ *                receive buffer, as BF16 or as FP8 e4m3 with one fp32 scale
+ *                per 128 channels;
+ *   ep_combine   gather of the k expert outputs of each token, reduced with
+ *                the routing weights in fp32, back into token order.
+ *
+ * Source of the operations.  "DeepEP是什麼？MoE Dispatch、Combine、
+ * All-to-all與V2架構" (yololab.net), stage table of the section
+ * "MoE為什麼需要All-to-all": dispatch takes tokens, top-k indices and weights
+ * and yields hidden states arranged by expert; combine takes the expert
+ * outputs and routing weights and yields results in the original token order.
+ * The same page's ElasticBuffer section has the buffer own the "dispatch
+ * layout" and be sized from max tokens, top-k, hidden and EP degree; the
+ * DeepEP v2 release notes (donniechu.com, "Có gì mới trong v2") pair the
+ * buffer with an EPHandle that carries dispatch state into combine.  Here the
+ * caller owns every buffer, and the opaque ep_handle_t carries the layout.
+ *
+ * Layout rules (the pages name a "GEMM layout" without defining it; this is
+ * the reading taken): expert e belongs to rank floor(e / (E/R)); one flat
+ * receive buffer holds experts in index order; expert e's block starts at
+ * expert_off[e] and is padded up to a multiple of block_m rows; inside a
+ * block, rows are in (source token, slot) order; rank r's receive buffer is
+ * rows [rank_off[r], rank_off[r+1]).  Pad rows are never written.
+ *
+ * Conventions.  All tensors are dense row-major.  "device" pointers must be
+ * addresses of the current CUDA device's global memory; "host" pointers are
+ * ordinary CPU memory.  Every call that takes a stream enqueues its work on
+ * that stream (a cudaStream_t passed as void*, NULL = legacy default stream)
+ * and returns without waiting, except the ones documented as synchronising.
+ * The library never allocates device memory; the handle itself is a small
+ * host allocation made by ep_handle_create.
+ *
+ * Errors.  Argument problems that the host can see are returned at once and
+ * nothing is enqueued.  Problems only the GPU can see (an index outside
+ * [-1, E), a receive row beyond the capacity given) set bits in a sticky
+ * device error word inside the workspace; the offending rows are skipped,
+ * nothing out of bounds is touched, and ep_handle_check reports them.  No
+ * kernel traps and no kernel waits on another.
+ *
+ * Thread safety: calls on one handle must not run concurrently from several
+ * host threads; distinct handles are independent.
+ */
+#ifndef EP_H_
+#define EP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ep_handle_s* ep_handle_t;
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1,          /* bad size, null pointer, unsupported shape */
+    EP_ERR_ALIGNMENT = 2,            /* a pointer misses its required alignment */
+    EP_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes < ep_workspace_bytes(...) */
+    EP_ERR_CAPACITY = 4,             /* a receive row did not fit the buffer given */
+    EP_ERR_BAD_INDEX = 5,            /* a top-k index outside [-1, E) */
+    EP_ERR_CUDA = 6,                 /* a CUDA runtime call failed; see ep_last_error_message */
+    EP_ERR_STATE = 7,                /* e.g. dispatch/combine before any ep_layout */
+    EP_ERR_NO_MEMORY = 8             /* host malloc of the handle failed */
+} ep_status_t;
+
+typedef enum {
+    EP_FMT_BF16 = 0,            /* receive rows are the bf16 input rows */
+    EP_FMT_FP8_E4M3_1X128 = 1   /* e4m3 rows + one fp32 scale per 128 channels */
+} ep_fmt_t;
+
+/* Views of the layout held in the workspace (see ep_handle_view). */
+typedef enum {
+    EP_VIEW_NUM_TOKENS_PER_EXPERT = 0, /* int32 [E]     slots routed to each expert */
+    EP_VIEW_NUM_TOKENS_PER_RANK = 1,   /* int32 [R]     tokens with >= 1 slot on rank r */
+    EP_VIEW_NUM_ROWS_PER_RANK = 2,     /* int32 [R]     non-pad receive rows of rank r */
+    EP_VIEW_EXPERT_OFFSET = 3,         /* int32 [E+1]   padded block starts; [E] = P */
+    EP_VIEW_RANK_OFFSET = 4,           /* int32 [R+1]   rank r owns rows [off[r], off[r+1]) */
+    EP_VIEW_IS_TOKEN_IN_RANK = 5,      /* uint8 [T][R]  1 if token t sends to rank r */
+    EP_VIEW_DST_ROW = 6,               /* int32 [T][k]  receive row of slot (t,j), -1 unused */
+    EP_VIEW_RECV_SRC = 7,              /* int32 [P]     source token of each row, -1 on pad */
+    EP_VIEW_TOTAL_RECV_ROWS = 8        /* int32 [1]     P, the padded receive rows */
+} ep_view_t;
+
+/* Limits of this build. */
+#define EP_MAX_TOPK 32
+#define EP_MAX_EXPERTS 8192
+#define EP_MAX_BLOCK_M 4096
+
+/* Bytes of device workspace a handle needs for up to max_tokens tokens
+ * (host; pure arithmetic).  Returns 0 if the arguments are invalid:
+ * max_tokens >= 0, 1 <= num_topk <= EP_MAX_TOPK,
+ * 1 <= num_experts <= EP_MAX_EXPERTS, 1 <= num_ranks, num_experts % num_ranks
+ * == 0, 1 <= block_m <= EP_MAX_BLOCK_M, and every row count below 2^31. */
+size_t ep_workspace_bytes(int max_tokens, int num_topk, int num_experts, int num_ranks,
+                          int block_m);
+
+/* Upper bound on the padded receive rows P for T tokens (host, no sync):
+ * T*k + min(E, T*k)*(block_m - 1), rounded down to a multiple of block_m.
+ * Sizing recv buffers with it lets a whole step run without reading P back,
+ * e.g. inside a CUDA graph.  Returns -1 for invalid arguments. */
+int64_t ep_recv_rows_upper_bound(int T, int num_topk, int num_experts, int block_m);
+
+/* Create a handle over a caller-owned device workspace (host; makes no CUDA
+ * call).  workspace: device pointer, 256-byte aligned, at least
+ * ep_workspace_bytes(...) bytes, owned by the caller and kept alive, and not
+ * used for anything else, until ep_handle_destroy.  On success *out receives
+ * the handle; on failure *out is set to NULL. */
+ep_status_t ep_handle_create(void* workspace, size_t workspace_bytes, int max_tokens,
+                             int num_topk, int num_experts, int num_ranks, int block_m,
+                             ep_handle_t* out);
+
+/* Free the host-side handle (not the workspace).  NULL is ignored.  Work
+ * already enqueued that uses the workspace is unaffected. */
+void ep_handle_destroy(ep_handle_t h);
+
+/* Dispatch layout (get_dispatch_layout).  topk_idx: device int64 [T][k],
+ * 8-byte aligned (may be NULL when T == 0); each value is an expert in
+ * [0, E) or -1 for an unused slot.  0 <= T <= max_tokens.  Fills every view
+ * of ep_view_t.  The layout stays valid, and is what ep_dispatch and
+ * ep_combine use, until the next ep_layout on this handle.  An index outside
+ * [-1, E) sets EP_ERR_BAD_INDEX in the sticky error word and is treated as -1. */
+ep_status_t ep_layout(ep_handle_t h, const int64_t* topk_idx, int T, void* stream);
+
+/* Device pointer of a layout view inside the workspace (host; no CUDA call);
+ * *count (if not NULL) receives its number of elements for the last layout
+ * (P for EP_VIEW_RECV_SRC is only known on the device, so its count is the
+ * capacity reserved for max_tokens).  Returns NULL for an unknown view. */
+const void* ep_handle_view(ep_handle_t h, ep_view_t what, int64_t* count);
+
+/* Copy the counts of the last layout to host memory and wait for the stream
+ * (SYNCHRONISING).  Any output pointer may be NULL.  num_tokens_per_expert:
+ * int32 [E]; num_tokens_per_rank: int32 [R]; num_rows_per_rank: int32 [R];
+ * total_recv_rows: int32 [1] (P). */
+ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
+                                  int32_t* num_tokens_per_rank, int32_t* num_rows_per_rank,
+                                  int32_t* total_recv_rows, void* stream);
+
+/* Dispatch the T tokens of the last layout.
+ * x: device bf16 [T][H], 16-byte aligned.
+ * EP_FMT_BF16: H % 8 == 0; recv_x: device bf16 [recv_capacity_rows][H],
+ *   16-byte aligned; recv_scales ignored.  recv_x[dst_row[t][j]] = x[t].
+ * EP_FMT_FP8_E4M3_1X128: H % 128 == 0; recv_x: device e4m3 bytes
+ *   [recv_capacity_rows][H], 16-byte aligned; recv_scales: device fp32
+ *   [recv_capacity_rows][H/128], 16-byte aligned.  For every token and every
+ *   block b of 128 channels: amax = max |x|, s = amax / 448 (fp32 division),
+ *   q = e4m3(x / s) (fp32 division, round to nearest even, saturate to
+ *   +-448); amax == 0 gives s = 0 and q = 0.  Written to every dst row.
+ *   This is the reading taken of the FP8 section of the yololab page, which
+ *   asks to confirm scale granularity and format without fixing them.
+ * Only the rows listed in dst_row are written; pad rows keep their contents.
+ * A row >= recv_capacity_rows is skipped and sets EP_ERR_CAPACITY. */
+ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void* recv_x,
+                        float* recv_scales, int64_t recv_capacity_rows, void* stream);
+
+/* Combine into token order for the T tokens of the last layout.
+ * y: device bf16 [y_rows][H] in the receive layout, 16-byte aligned, H % 8 == 0.
+ * topk_weights: device fp32 [T][k], 4-byte aligned.
+ * out: device bf16 [T][H], 16-byte aligned, must not overlap y.
+ * out[t][h] = bf16_rn(acc), acc = 0 then, for j = 0..k-1 over the used
+ * slots, acc = fma(w[t][j], y[dst_row[t][j]][h], acc) in fp32.  Weights are
+ * used as given (no renormalisation); unused slots (-1) are skipped.
+ * A row >= y_rows is skipped and sets EP_ERR_CAPACITY. */
+ep_status_t ep_combine(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
+                       int H, void* out, void* stream);
+
+/* Wait for the stream (SYNCHRONISING), read and clear the sticky device
+ * error word.  Returns EP_ERR_BAD_INDEX, EP_ERR_CAPACITY (bad index wins if
+ * both are set) or EP_OK. */
+ep_status_t ep_handle_check(ep_handle_t h, void* stream);
+
+/* Human-readable name of a status. */
+const char* ep_strerror(ep_status_t status);
+
+/* Text of the last CUDA error seen by this host thread inside the library
+ * ("" if none). */
+const char* ep_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_H_ */

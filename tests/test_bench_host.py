@@ -1,0 +1,67 @@
+"""Host logic of bench.py on the CPU: the algorithmic byte model, and the
+max-over-ranks reduction used for multi-GPU timing (world_size 2, gloo)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_algorithmic_bytes_match_the_stated_model():
+    # dispatch = T*2H read + T*k*rowB written; combine = T*k*2H read + T*2H written
+    assert bench.algo_bytes(8192, 7168, 8, "bf16") == (1056964608, 1056964608)
+    assert bench.algo_bytes(8192, 7168, 8, "fp8") == (601882624, 1056964608)
+    assert bench.algo_bytes(4096, 7168, 8, "fp8") == (300941312, 528482304)
+    assert bench.algo_bytes(128, 7168, 8, "fp8") == (9404416, 16515072)
+    assert bench.algo_bytes(128, 256, 2, "bf16") == (196608, 196608)
+    # the pages' per-stage volume: batch x top_k x hidden x sizeof(dtype)
+    T, H, k = 8192, 7168, 8
+    d, c = bench.algo_bytes(T, H, k, "bf16")
+    assert d - T * 2 * H == T * k * H * 2 == c - T * 2 * H
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local = [3.5, 7.25][rank]
+        got = bench.aggregate_max(local)
+        q.put((rank, got))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res == {0: 7.25, 1: 7.25}
+
+
+def test_aggregate_max_single_process_is_identity():
+    assert bench.aggregate_max(1.5) == 1.5
+
+
+def test_kernel_hash_is_stable():
+    assert bench.kernel_source_hash() == bench.kernel_source_hash()
+    assert len(bench.kernel_source_hash()) == 16
