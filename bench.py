@@ -67,12 +67,18 @@ def load_peaks():
     return 6650.0, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
-def kernel_source_hash():
-    h = hashlib.sha256()
-    for name in ("ep_dispatch.cu", "ep_combine.cu", "ep_layout.cu", "ep_internal.cuh"):
-        with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
+KERNEL_FILES = {
+    "dispatch_bf16_kernel": "ep_dispatch.cu",
+    "dispatch_fp8_kernel": "ep_dispatch.cu",
+    "combine_kernel": "ep_combine.cu",
+}
+
+
+def kernel_source_hash(kernel: str = "dispatch_bf16_kernel"):
+    """Hash of the source file that holds a kernel (first 16 hex digits)."""
+    name = KERNEL_FILES.get(kernel, "ep_dispatch.cu")
+    with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
@@ -83,10 +89,10 @@ def ncu_traffic(kernel: str):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     e = d.get("kernels", {}).get(kernel)
-    return None if e is None else e.get("dram_bytes_per_launch")
+    if e is None or e.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return e.get("dram_bytes_per_launch")
 
 
 # ----------------------------------------------------------------- clocks
