@@ -179,6 +179,51 @@ ep_status_t ep_combine(ep_handle_t h, const void* y, int64_t y_rows, const float
  * both are set) or EP_OK. */
 ep_status_t ep_handle_check(ep_handle_t h, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Dispatch layout without any caller-provided workspace.
+ *
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory: code running while a CUDA graph is being
+ * captured, processes whose device memory is owned up front by a framework
+ * allocator or a pre-reserved pool that forbids more cudaMalloc calls, and
+ * plug-ins that are handed only input and output pointers.
+ *
+ * It computes exactly what ep_layout computes, into caller-provided output
+ * arrays, with the same kernels.  Its only scratch (4 bytes x ceil(T/32) x
+ * (E + R) counters) lives in a fixed array of EP_STATIC_SCRATCH_BYTES inside
+ * this library, which every GPU that loads the library keeps until the
+ * process exits.  Nothing is allocated: no cudaMalloc, no cudaFree, no
+ * allocating library call.
+ *
+ *   - Larger requests (4 * ceil(T/32) * (E + R) > EP_STATIC_SCRATCH_BYTES)
+ *     return EP_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array per device and it keeps the last
+ *     call's contents (nothing in it needs to start at zero).  Calls that
+ *     overlap on the GPU -- on different streams without ordering, or from
+ *     several host threads -- race on it and must be serialised by the caller.
+ *
+ * Outputs (device): num_tokens_per_expert int32 [E], num_tokens_per_rank
+ * int32 [R], num_rows_per_rank int32 [R], expert_off int32 [E+1], rank_off
+ * int32 [R+1], total_recv_rows int32 [1], is_token_in_rank uint8 [T][R],
+ * dst_row int32 [T][k], recv_src int32 [recv_src_capacity] with
+ * recv_src_capacity >= ep_recv_rows_upper_bound(T, k, E, block_m)
+ * (else EP_ERR_CAPACITY), error_word int32 [1]: zeroed by this call, then
+ * EP_ERR_BAD_INDEX's bit (1) is set if an index is outside [-1, E).
+ * topk_idx: device int64 [T][k], 8-byte aligned.  Shape rules as for
+ * ep_workspace_bytes. */
+#define EP_STATIC_SCRATCH_BYTES (4u << 20)
+ep_status_t ep_layout_static_scratch(const int64_t* topk_idx, int T, int num_topk,
+                                     int num_experts, int num_ranks, int block_m,
+                                     int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
+                                     int32_t* num_rows_per_rank, int32_t* expert_off,
+                                     int32_t* rank_off, int32_t* total_recv_rows,
+                                     uint8_t* is_token_in_rank, int32_t* dst_row,
+                                     int32_t* recv_src, int64_t recv_src_capacity,
+                                     int32_t* error_word, void* stream);
+
 /* Human-readable name of a status. */
 const char* ep_strerror(ep_status_t status);
 
