@@ -68,13 +68,13 @@ def load_peaks():
 
 
 KERNEL_FILES = {
-    "dispatch_bf16_kernel": "ep_dispatch.cu",
-    "dispatch_fp8_kernel": "ep_dispatch.cu",
+    "dispatch_bf16_v32_kernel": "ep_dispatch.cu",
+    "dispatch_fp8_v32_kernel": "ep_dispatch.cu",
     "combine_kernel": "ep_combine.cu",
 }
 
 
-def kernel_source_hash(kernel: str = "dispatch_bf16_kernel"):
+def kernel_source_hash(kernel: str = "dispatch_bf16_v32_kernel"):
     """Hash of the source file that holds a kernel (first 16 hex digits)."""
     name = KERNEL_FILES.get(kernel, "ep_dispatch.cu")
     with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name), "rb") as f:
@@ -513,7 +513,7 @@ def main():
     dom_ms = max(dis_ms, com_ms)
     dom_bytes = d_bytes if dom == "dispatch" else c_bytes
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    kname = "dispatch_bf16_kernel" if dom == "dispatch" else "combine_kernel"
+    kname = "dispatch_bf16_v32_kernel" if dom == "dispatch" else "combine_kernel"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kname),
                 "kernel": kname, "peak_source": peak_src}

@@ -83,6 +83,8 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
                int T, int k, int64_t vpr, const int32_t* __restrict__ dst_row,
                uint4* __restrict__ out, int32_t* err)
 {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t wg = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
@@ -157,10 +159,8 @@ cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const
     cudaError_t rc = persistent_grid((const void*)combine_kernel, kThreads, 0, 8, &grid);
     if (rc != cudaSuccess)
         return rc;
-    combine_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(y), y_rows, w, h.T, h.k,
-                                             (int64_t)H / 8, h.dst_row,
-                                             static_cast<uint4*>(out), h.err);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, grid, kThreads, 0, s, static_cast<const uint4*>(y), y_rows, w,
+                      h.T, h.k, (int64_t)H / 8, h.dst_row, static_cast<uint4*>(out), h.err);
 }
 
 }  // namespace ep

@@ -56,6 +56,32 @@ struct Carve {
 int64_t recv_rows_bound(int64_t T, int64_t k, int64_t E, int64_t block_m);
 bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c);
 
+// Programmatic dependent launch (sm_90+): every kernel of the library is
+// launched with programmatic stream serialization allowed, starts with
+// pdl_wait() -- it returns once the preceding kernel in the stream has
+// completed and its memory is visible -- and then pdl_trigger(), which lets
+// the next kernel's CTAs be scheduled while this one drains.  Nothing is
+// read or written before pdl_wait(), so a kernel may follow any other work.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Launchers (each returns the cudaError_t of its launches).
 cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s);
 cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,

@@ -9,18 +9,27 @@
 // layout itself is stated in ep.h.
 //
 // Positions must be deterministic (order inside an expert block is by source
-// token, then slot), so they are never taken from atomics.  Three launches:
-//   K1 count   one warp per chunk of 32 tokens: shared-memory histogram of
-//              the chunk's experts, is_token_in_rank bytes, per-chunk count
-//              of tokens per rank;
+// token, then slot), so they are never taken from atomics: integer
+// shared-memory atomics only build histograms, whose sums do not depend on
+// order.  Entries are grouped in chunks of 32 tokens, one warp per chunk.
+//
+// Large batches, three launches:
+//   K1 count   per chunk: shared-memory histogram of the chunk's experts,
+//              is_token_in_rank bytes, per-chunk count of tokens per rank;
 //   K2 scan    per expert, exclusive prefix of the chunk counts over chunks
 //              (in place), per-expert totals and per-rank token totals;
 //   K3 assign  every CTA scans the padded expert sizes into expert_off; each
 //              warp replays its chunk in order, ranking equal experts inside
 //              each group of 32 entries with __match_any_sync, to give
 //              dst_row and recv_src; pad rows of recv_src are set to -1.
-// Integer shared-memory atomics are used only for counts, whose sums do not
-// depend on order.
+// Small batches (at most 32 chunks) run the same three phases inside one CTA
+// (layout_small_kernel), with the chunk counts in shared memory.
+//
+// The work is latency-bound (at 8K tokens the layout reads 0.5 MB), so each
+// kernel issues all of its global loads before it uses any of them, and every
+// kernel is launched with programmatic dependent launch: it may start while
+// its predecessor drains, and waits (griddepcontrol.wait) before it touches
+// memory.
 #include <algorithm>
 
 #include "ep_internal.cuh"
@@ -31,6 +40,7 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kScanThreads = 1024;
 constexpr size_t kSmemBudget = 200 * 1024;
+constexpr int kBatch = 8;  // entries per lane loaded before any is used
 
 __device__ __forceinline__ unsigned lanemask_lt()
 {
@@ -41,133 +51,22 @@ __device__ __forceinline__ unsigned lanemask_lt()
 
 __device__ __forceinline__ int32_t pad_up(int32_t c, int32_t b) { return ((c + b - 1) / b) * b; }
 
-// K1.  Shared memory per warp: hist[E], rank_hist[R], entry_rank[32 k].
-__global__ void layout_count_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                    int R, int epr, int64_t nchunks,
-                                    int32_t* __restrict__ chunk_counts,
-                                    int32_t* __restrict__ chunk_rank,
-                                    uint8_t* __restrict__ is_token_in_rank, int32_t* err)
+// An expert in [0, E), or -1 for an unused slot; anything else is flagged.
+__device__ __forceinline__ int to_expert(int64_t v, int E, int& bad)
 {
-    extern __shared__ int32_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int per_warp = E + R + kChunkTokens * k;
-    int32_t* hist = smem + (size_t)warp * per_warp;
-    int32_t* rhist = hist + E;
-    int32_t* erank = rhist + R;
-
-    const int64_t c = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-    if (c >= nchunks)
-        return;  // the whole warp leaves; no block barrier follows
-    const int64_t t0 = c * kChunkTokens;
-    const int ntok = (int)min((int64_t)kChunkTokens, (int64_t)T - t0);
-    const int nent = ntok * k;
-
-    for (int e = lane; e < E; e += 32) hist[e] = 0;
-    for (int r = lane; r < R; r += 32) rhist[r] = 0;
-    __syncwarp();
-
-    const int64_t* src = topk_idx + t0 * k;
-    int bad = 0;
-    for (int f = lane; f < nent; f += 32) {
-        const int64_t v = src[f];
-        int e = -1;
-        if (v >= 0 && v < E)
-            e = (int)v;
-        else if (v != -1)
-            bad = 1;
-        erank[f] = e >= 0 ? e / epr : -1;
-        if (e >= 0)
-            atomicAdd(&hist[e], 1);
-    }
-    if (__any_sync(kFull, bad) && lane == 0)
-        atomicOr(err, kErrBadIndex);
-    __syncwarp();
-
-    // is_token_in_rank bytes of the chunk, p = t * R + r: consecutive lanes
-    // write consecutive bytes.
-    for (int p = lane; p < ntok * R; p += 32) {
-        const int t = p / R, r = p - t * R;
-        int hit = 0;
-        for (int j = 0; j < k; ++j) hit |= (erank[t * k + j] == r);
-        is_token_in_rank[(t0 + t) * R + r] = (uint8_t)hit;
-        if (hit)
-            atomicAdd(&rhist[r], 1);
-    }
-    __syncwarp();
-
-    for (int e = lane; e < E; e += 32) chunk_counts[c * E + e] = hist[e];
-    for (int r = lane; r < R; r += 32) chunk_rank[c * R + r] = rhist[r];
+    if (v >= 0 && v < E)
+        return (int)v;
+    if (v != -1)
+        bad = 1;
+    return -1;
 }
 
-// K2.  Blocks [0, ceil(E/32)) own 32 experts each, the rest 32 ranks each;
-// lane = column, warp w = a contiguous range of chunks.
-__global__ void __launch_bounds__(kScanThreads)
-layout_scan_kernel(int32_t* __restrict__ chunk_counts, const int32_t* __restrict__ chunk_rank,
-                   int E, int R, int64_t nchunks, int32_t* __restrict__ cnt,
-                   int32_t* __restrict__ tokens_per_rank)
+// Block-wide exclusive scan of pad(cnt[e]) into off[0..E] (shared memory).
+// cnt may live in global or shared memory.  Uses wsum[32] as scratch.
+__device__ void scan_padded(const int32_t* cnt, int E, int block_m, int32_t* off, int32_t* wsum)
 {
-    __shared__ int32_t part[32][33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int eblocks = (E + 31) / 32;
-    const bool is_expert = (int)blockIdx.x < eblocks;
-    const int ncol = is_expert ? E : R;
-    const int col = (is_expert ? (int)blockIdx.x : (int)blockIdx.x - eblocks) * 32 + lane;
-    const bool colok = col < ncol;
-    const int32_t* M = is_expert ? chunk_counts : chunk_rank;
-
-    const int64_t rpw = (nchunks + 31) / 32;
-    const int64_t r0 = min(nchunks, (int64_t)warp * rpw);
-    const int64_t r1 = min(nchunks, r0 + rpw);
-
-    int32_t sum = 0;
-    if (colok)
-        for (int64_t r = r0; r < r1; ++r) sum += M[r * ncol + col];
-    part[warp][lane] = sum;
-    __syncthreads();
-
-    int32_t pre = 0, total = 0;
-    for (int w = 0; w < 32; ++w) {
-        const int32_t v = part[w][lane];
-        pre += (w < warp) ? v : 0;
-        total += v;
-    }
-    if (is_expert && colok) {
-        int32_t run = pre;
-        for (int64_t r = r0; r < r1; ++r) {
-            const int32_t v = chunk_counts[r * ncol + col];
-            chunk_counts[r * ncol + col] = run;
-            run += v;
-        }
-    }
-    if (warp == 0 && colok) {
-        if (is_expert)
-            cnt[col] = total;
-        else
-            tokens_per_rank[col] = total;
-    }
-}
-
-// K3.  Shared memory: off[E+1], warp totals[32], then run[E] per warp.
-__global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                     int R, int epr, int block_m, int64_t nchunks,
-                                     const int32_t* __restrict__ chunk_prefix,
-                                     const int32_t* __restrict__ cnt,
-                                     int32_t* __restrict__ expert_off_g,
-                                     int32_t* __restrict__ rank_off_g,
-                                     int32_t* __restrict__ rows_per_rank_g,
-                                     int32_t* __restrict__ total_rows_g,
-                                     int32_t* __restrict__ dst_row,
-                                     int32_t* __restrict__ recv_src)
-{
-    extern __shared__ int32_t smem[];
-    int32_t* off = smem;
-    int32_t* wsum = off + E + 1;
-    int32_t* run_all = wsum + 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
-    const int nthr = blockDim.x;
-
-    // Block-wide exclusive scan of pad(cnt[e]): contiguous segment per thread.
+    const int nwarps = blockDim.x >> 5, nthr = blockDim.x;
     const int seg = (E + nthr - 1) / nthr;
     const int e0 = min(E, (int)threadIdx.x * seg), e1 = min(E, e0 + seg);
     int32_t local = 0;
@@ -201,43 +100,37 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
     if ((int)threadIdx.x == nthr - 1)
         off[E] = run;
     __syncthreads();
+}
 
-    if (blockIdx.x == 0) {
-        for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
-        for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
-        for (int r = threadIdx.x; r < R; r += nthr) {
-            int32_t s = 0;
-            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
-            rows_per_rank_g[r] = s;
-        }
-        if (threadIdx.x == 0)
-            *total_rows_g = off[E];
+// One warp: is_token_in_rank bytes of a chunk from the entries' ranks
+// (erank[t * k + j], -1 for unused), p = t * R + r so that consecutive lanes
+// write consecutive bytes; per-rank token counts go to rhist.
+__device__ __forceinline__ void chunk_rank_bytes(const int32_t* erank, int ntok, int k, int R,
+                                                 int64_t t0, uint8_t* is_token_in_rank,
+                                                 int32_t* rhist)
+{
+    const int lane = threadIdx.x & 31;
+    for (int p = lane; p < ntok * R; p += 32) {
+        const int t = p / R, r = p - t * R;
+        int hit = 0;
+        for (int j = 0; j < k; ++j) hit |= (erank[t * k + j] == r);
+        is_token_in_rank[(t0 + t) * R + r] = (uint8_t)hit;
+        if (hit)
+            atomicAdd(&rhist[r], 1);
     }
+}
 
-    // Pad rows of the experts this CTA owns.
-    for (int e = blockIdx.x; e < E; e += gridDim.x)
-        for (int32_t r = off[e] + cnt[e] + (int32_t)threadIdx.x; r < off[e + 1]; r += nthr)
-            recv_src[r] = -1;
-
-    const int64_t c = (int64_t)blockIdx.x * nwarps + warp;
-    if (c >= nchunks)
-        return;  // no block barrier follows
-    int32_t* runc = run_all + (size_t)warp * E;
-    for (int e = lane; e < E; e += 32) runc[e] = off[e] + chunk_prefix[c * E + e];
-    __syncwarp();
-
-    const int64_t t0 = c * kChunkTokens;
-    const int ntok = (int)min((int64_t)kChunkTokens, (int64_t)T - t0);
-    const int nent = ntok * k;
-    const int64_t* src = topk_idx + t0 * k;
+// One warp: replay a chunk's entries (ents in smem, -1 unused) in order and
+// give each its row.  runc[e] holds the next free row of expert e for this
+// chunk and is advanced here.
+__device__ __forceinline__ void chunk_assign(const int32_t* ents, int nent, int k, int64_t t0,
+                                             int32_t* runc, int32_t* dst_row, int32_t* recv_src)
+{
+    const int lane = threadIdx.x & 31;
     const unsigned lt = lanemask_lt();
     for (int g = 0; g < nent; g += 32) {
         const int f = g + lane;
-        int e = -2;  // lanes past the chunk end
-        if (f < nent) {
-            const int64_t v = src[f];
-            e = (v >= 0 && v < E) ? (int)v : -1;
-        }
+        const int e = f < nent ? ents[f] : -2;  // -2: lanes past the chunk end
         const unsigned peers = __match_any_sync(kFull, e);
         int pos = -1;
         if (e >= 0)
@@ -252,6 +145,302 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
                 recv_src[pos] = (int32_t)(t0 + f / k);
         }
     }
+}
+
+// One warp: load a chunk's entries (all loads of a batch issued first),
+// validate them into ents[] and, if erank is given, their ranks; count them
+// into hist (shared-memory atomics) if hist is given.
+__device__ __forceinline__ int load_chunk(const int64_t* __restrict__ src, int nent, int E,
+                                          int epr, int32_t* ents, int32_t* erank, int32_t* hist)
+{
+    const int lane = threadIdx.x & 31;
+    int bad = 0;
+    for (int base = 0; base < nent; base += 32 * kBatch) {
+        int64_t v[kBatch];
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m) {
+            const int f = base + m * 32 + lane;
+            v[m] = f < nent ? src[f] : -1;
+        }
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m) {
+            const int f = base + m * 32 + lane;
+            if (f < nent) {
+                const int e = to_expert(v[m], E, bad);
+                if (ents)
+                    ents[f] = e;
+                if (erank)
+                    erank[f] = e >= 0 ? e / epr : -1;
+                if (hist && e >= 0)
+                    atomicAdd(&hist[e], 1);
+            }
+        }
+    }
+    return __any_sync(kFull, bad);
+}
+
+// K1.  Shared memory per warp: hist[E], rank_hist[R], entry_rank[32 k].
+__global__ void layout_count_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
+                                    int R, int epr, int64_t nchunks,
+                                    int32_t* __restrict__ chunk_counts,
+                                    int32_t* __restrict__ chunk_rank,
+                                    uint8_t* __restrict__ is_token_in_rank, int32_t* err)
+{
+    extern __shared__ int32_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per_warp = E + R + kChunkTokens * k;
+    int32_t* hist = smem + (size_t)warp * per_warp;
+    int32_t* rhist = hist + E;
+    int32_t* erank = rhist + R;
+
+    const int64_t c = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (c >= nchunks)
+        return;  // the whole warp leaves; no block barrier follows
+    const int64_t t0 = c * kChunkTokens;
+    const int ntok = (int)min((int64_t)kChunkTokens, (int64_t)T - t0);
+    const int nent = ntok * k;
+
+    for (int e = lane; e < E; e += 32) hist[e] = 0;
+    for (int r = lane; r < R; r += 32) rhist[r] = 0;
+    __syncwarp();
+    const int bad = load_chunk(topk_idx + t0 * k, nent, E, epr, nullptr, erank, hist);
+    if (bad && lane == 0)
+        atomicOr(err, kErrBadIndex);
+    __syncwarp();
+    chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) chunk_counts[c * E + e] = hist[e];
+    for (int r = lane; r < R; r += 32) chunk_rank[c * R + r] = rhist[r];
+}
+
+// K2.  Blocks [0, ceil(E/32)) own 32 experts each, the rest 32 ranks each;
+// lane = column, warp w = a contiguous range of chunks.
+__global__ void __launch_bounds__(kScanThreads)
+layout_scan_kernel(int32_t* __restrict__ chunk_counts, const int32_t* __restrict__ chunk_rank,
+                   int E, int R, int64_t nchunks, int32_t* __restrict__ cnt,
+                   int32_t* __restrict__ tokens_per_rank)
+{
+    __shared__ int32_t part[32][33];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int eblocks = (E + 31) / 32;
+    const bool is_expert = (int)blockIdx.x < eblocks;
+    const int ncol = is_expert ? E : R;
+    const int col = (is_expert ? (int)blockIdx.x : (int)blockIdx.x - eblocks) * 32 + lane;
+    const bool colok = col < ncol;
+    const int32_t* M = is_expert ? chunk_counts : chunk_rank;
+
+    const int64_t rpw = (nchunks + 31) / 32;
+    const int64_t r0 = min(nchunks, (int64_t)warp * rpw);
+    const int64_t r1 = min(nchunks, r0 + rpw);
+
+    // all loads of the range first (in registers when it is short)
+    int32_t vals[kBatch];
+    int32_t sum = 0;
+    const bool short_range = (r1 - r0) <= kBatch;
+    if (short_range) {
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m)
+            vals[m] = (colok && r0 + m < r1) ? M[(r0 + m) * ncol + col] : 0;
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m) sum += vals[m];
+    } else if (colok) {
+        for (int64_t r = r0; r < r1; ++r) sum += M[r * ncol + col];
+    }
+    part[warp][lane] = sum;
+    __syncthreads();
+
+    int32_t pre = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+        const int32_t v = part[w][lane];
+        pre += (w < warp) ? v : 0;
+        total += v;
+    }
+    if (is_expert && colok) {
+        int32_t run = pre;
+        if (short_range) {
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m)
+                if (r0 + m < r1) {
+                    chunk_counts[(r0 + m) * ncol + col] = run;
+                    run += vals[m];
+                }
+        } else {
+            for (int64_t r = r0; r < r1; ++r) {
+                const int32_t v = chunk_counts[r * ncol + col];
+                chunk_counts[r * ncol + col] = run;
+                run += v;
+            }
+        }
+    }
+    if (warp == 0 && colok) {
+        if (is_expert)
+            cnt[col] = total;
+        else
+            tokens_per_rank[col] = total;
+    }
+}
+
+// K3.  Shared memory: off[E+1], wsum[32], then per warp run[E] + ents[32 k].
+__global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
+                                     int R, int epr, int block_m, int64_t nchunks,
+                                     const int32_t* __restrict__ chunk_prefix,
+                                     const int32_t* __restrict__ cnt,
+                                     int32_t* __restrict__ expert_off_g,
+                                     int32_t* __restrict__ rank_off_g,
+                                     int32_t* __restrict__ rows_per_rank_g,
+                                     int32_t* __restrict__ total_rows_g,
+                                     int32_t* __restrict__ dst_row,
+                                     int32_t* __restrict__ recv_src)
+{
+    extern __shared__ int32_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    int32_t* off = smem;
+    int32_t* wsum = off + E + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int nthr = blockDim.x;
+    int32_t* runc = wsum + 32 + (size_t)warp * (E + kChunkTokens * k);
+    int32_t* ents = runc + E;
+
+    const int64_t c = (int64_t)blockIdx.x * nwarps + warp;
+    const bool has_chunk = c < nchunks;
+    const int64_t t0 = c * kChunkTokens;
+    const int ntok = has_chunk ? (int)min((int64_t)kChunkTokens, (int64_t)T - t0) : 0;
+    const int nent = ntok * k;
+
+    // Loads that do not depend on each other, issued together: this warp's
+    // row of chunk prefixes (into runc), its entries (into ents) and, in
+    // scan_padded, the expert totals.
+    if (has_chunk) {
+        for (int base = 0; base < E; base += 32 * kBatch) {
+            int32_t v[kBatch];
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m) {
+                const int e = base + m * 32 + lane;
+                v[m] = e < E ? chunk_prefix[c * E + e] : 0;
+            }
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m) {
+                const int e = base + m * 32 + lane;
+                if (e < E)
+                    runc[e] = v[m];
+            }
+        }
+        int ignored = load_chunk(topk_idx + t0 * k, nent, E, epr, ents, nullptr, nullptr);
+        (void)ignored;  // bad indices were flagged by the count pass
+    }
+    scan_padded(cnt, E, block_m, off, wsum);
+
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
+        for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
+        for (int r = threadIdx.x; r < R; r += nthr) {
+            int32_t s = 0;
+            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
+            rows_per_rank_g[r] = s;
+        }
+        if (threadIdx.x == 0)
+            *total_rows_g = off[E];
+    }
+    // Pad rows of the experts this CTA owns.
+    for (int e = blockIdx.x; e < E; e += gridDim.x)
+        for (int32_t r = off[e] + cnt[e] + (int32_t)threadIdx.x; r < off[e + 1]; r += nthr)
+            recv_src[r] = -1;
+
+    if (!has_chunk)
+        return;  // no block barrier follows
+    for (int e = lane; e < E; e += 32) runc[e] += off[e];
+    __syncwarp();
+    chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
+}
+
+// Small batches: the three phases in one CTA; warp w < nchunks owns chunk w,
+// and at least 8 warps share the scans and the pad fill.
+// Shared memory: hist[nc][E] (then per-chunk prefixes, then run), cnt[E],
+// off[E+1], wsum[32], rank_hist[R], per chunk ents[32 k] + erank[32 k],
+// with nc = max(1, nchunks).
+__global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
+                                    int R, int epr, int block_m, int64_t nchunks,
+                                    int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
+                                    int32_t* __restrict__ rank_off_g,
+                                    int32_t* __restrict__ tokens_per_rank_g,
+                                    int32_t* __restrict__ rows_per_rank_g,
+                                    int32_t* __restrict__ total_rows_g,
+                                    uint8_t* __restrict__ is_token_in_rank,
+                                    int32_t* __restrict__ dst_row, int32_t* __restrict__ recv_src,
+                                    int32_t* err)
+{
+    extern __shared__ int32_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5, nthr = blockDim.x;
+    const int nc = (int)max((int64_t)1, nchunks);
+    int32_t* hist_all = smem;                           // [nc][E]
+    int32_t* cnt = hist_all + (size_t)nc * E;           // [E]
+    int32_t* off = cnt + E;                             // [E+1]
+    int32_t* wsum = off + E + 1;                        // [32]
+    int32_t* rhist = wsum + 32;                         // [R]
+    const bool has_chunk = warp < nchunks;
+    int32_t* ents = rhist + R + (size_t)(has_chunk ? warp : 0) * (2 * kChunkTokens * k);
+    int32_t* erank = ents + kChunkTokens * k;
+    int32_t* hist = hist_all + (size_t)(has_chunk ? warp : 0) * E;
+
+    for (int i = threadIdx.x; i < nc * E; i += nthr) hist_all[i] = 0;
+    for (int r = threadIdx.x; r < R; r += nthr) rhist[r] = 0;
+    __syncthreads();
+
+    const int64_t t0 = (int64_t)warp * kChunkTokens;
+    const int ntok = has_chunk ? (int)min((int64_t)kChunkTokens, (int64_t)T - t0) : 0;
+    const int nent = ntok * k;
+    if (has_chunk) {
+        const int bad = load_chunk(topk_idx + t0 * k, nent, E, epr, ents, erank, hist);
+        if (bad && lane == 0)
+            atomicOr(err, kErrBadIndex);
+        __syncwarp();
+        chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
+    }
+    __syncthreads();
+
+    // per-expert prefix over chunks, in place; totals into cnt
+    for (int e = threadIdx.x; e < E; e += nthr) {
+        int32_t run = 0;
+        for (int w = 0; w < nc; ++w) {
+            const int32_t h = hist_all[(size_t)w * E + e];
+            hist_all[(size_t)w * E + e] = run;
+            run += h;
+        }
+        cnt[e] = run;
+    }
+    __syncthreads();
+    scan_padded(cnt, E, block_m, off, wsum);
+
+    for (int e = threadIdx.x; e < E; e += nthr) cnt_g[e] = cnt[e];
+    for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
+    for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
+    for (int r = threadIdx.x; r < R; r += nthr) {
+        int32_t s = 0;
+        for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
+        rows_per_rank_g[r] = s;
+        tokens_per_rank_g[r] = rhist[r];
+    }
+    if (threadIdx.x == 0)
+        *total_rows_g = off[E];
+    // pad rows: one warp per expert, lanes on consecutive rows
+    for (int e = warp; e < E; e += nwarps)
+        for (int32_t r = off[e] + cnt[e] + lane; r < off[e + 1]; r += 32)
+            recv_src[r] = -1;
+
+    if (!has_chunk)
+        return;
+    for (int e = lane; e < E; e += 32) hist[e] += off[e];
+    __syncwarp();
+    chunk_assign(ents, nent, k, t0, hist, dst_row, recv_src);
 }
 
 int warps_for(size_t per_warp_bytes, size_t fixed_bytes)
@@ -270,11 +459,31 @@ cudaError_t set_smem(const void* fn, size_t bytes)
 
 }  // namespace
 
+size_t small_layout_smem(int k, int E, int R, int64_t nchunks)
+{
+    const int64_t nc = std::max<int64_t>(1, nchunks);
+    return sizeof(int32_t) * (size_t)(nc * E + E + E + 1 + 32 + R + nc * 2 * kChunkTokens * k);
+}
+
 cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
     const int64_t nchunks = ((int64_t)T + kChunkTokens - 1) / kChunkTokens;
     cudaError_t rc;
+
+    // one CTA when the batch is small and its counts fit in shared memory
+    if (nchunks <= 32) {
+        const size_t smem = small_layout_smem(k, E, R, nchunks);
+        if (smem <= kSmemBudget) {
+            if ((rc = set_smem((const void*)layout_small_kernel, smem)) != cudaSuccess)
+                return rc;
+            const unsigned nw = (unsigned)std::max<int64_t>(8, nchunks);
+            return launch_pdl(layout_small_kernel, 1, 32 * nw, smem, s, topk_idx, T, k, E, R, epr,
+                              h.block_m, nchunks, h.cnt, h.expert_off, h.rank_off,
+                              h.tokens_per_rank, h.rows_per_rank, h.total_rows,
+                              h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
+        }
+    }
 
     if (nchunks > 0) {
         const size_t per_warp = sizeof(int32_t) * (size_t)(E + R + kChunkTokens * k);
@@ -283,30 +492,27 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
         if ((rc = set_smem((const void*)layout_count_kernel, smem1)) != cudaSuccess)
             return rc;
         const unsigned g1 = (unsigned)((nchunks + w1 - 1) / w1);
-        layout_count_kernel<<<g1, 32 * w1, smem1, s>>>(topk_idx, T, k, E, R, epr, nchunks,
-                                                       h.chunk_counts, h.chunk_rank,
-                                                       h.is_token_in_rank, h.err);
-        if ((rc = cudaGetLastError()) != cudaSuccess)
+        if ((rc = launch_pdl(layout_count_kernel, g1, 32 * w1, smem1, s, topk_idx, T, k, E, R,
+                             epr, nchunks, h.chunk_counts, h.chunk_rank, h.is_token_in_rank,
+                             h.err)) != cudaSuccess)
             return rc;
     }
 
     const unsigned g2 = (unsigned)((E + 31) / 32 + (R + 31) / 32);
-    layout_scan_kernel<<<g2, kScanThreads, 0, s>>>(h.chunk_counts, h.chunk_rank, E, R, nchunks,
-                                                   h.cnt, h.tokens_per_rank);
-    if ((rc = cudaGetLastError()) != cudaSuccess)
+    if ((rc = launch_pdl(layout_scan_kernel, g2, kScanThreads, 0, s, h.chunk_counts,
+                         h.chunk_rank, E, R, nchunks, h.cnt, h.tokens_per_rank)) != cudaSuccess)
         return rc;
 
     const size_t fixed3 = sizeof(int32_t) * (size_t)(E + 1 + 32);
-    const size_t per_warp3 = sizeof(int32_t) * (size_t)E;
+    const size_t per_warp3 = sizeof(int32_t) * (size_t)(E + kChunkTokens * k);
     const int w3 = warps_for(per_warp3, fixed3);
     const size_t smem3 = fixed3 + per_warp3 * w3;
     if ((rc = set_smem((const void*)layout_assign_kernel, smem3)) != cudaSuccess)
         return rc;
     const unsigned g3 = (unsigned)std::max<int64_t>(1, (nchunks + w3 - 1) / w3);
-    layout_assign_kernel<<<g3, 32 * w3, smem3, s>>>(
-        topk_idx, T, k, E, R, epr, h.block_m, nchunks, h.chunk_counts, h.cnt, h.expert_off,
-        h.rank_off, h.rows_per_rank, h.total_rows, h.dst_row, h.recv_src);
-    return cudaGetLastError();
+    return launch_pdl(layout_assign_kernel, g3, 32 * w3, smem3, s, topk_idx, T, k, E, R, epr,
+                      h.block_m, nchunks, h.chunk_counts, h.cnt, h.expert_off, h.rank_off,
+                      h.rows_per_rank, h.total_rows, h.dst_row, h.recv_src);
 }
 
 }  // namespace ep

@@ -63,6 +63,6 @@ def test_aggregate_max_single_process_is_identity():
 
 
 def test_kernel_hash_is_stable():
-    for k in ("dispatch_bf16_kernel", "combine_kernel"):
+    for k in ("dispatch_bf16_v32_kernel", "combine_kernel"):
         assert bench.kernel_source_hash(k) == bench.kernel_source_hash(k)
         assert len(bench.kernel_source_hash(k)) == 16

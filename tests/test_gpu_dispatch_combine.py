@@ -42,7 +42,9 @@ def _check_guards(full, guard_rows=4):
     assert bool((b[-guard_rows:] == SENTINEL).all()), "write above the receive buffer"
 
 
-def dispatch_case(oracle, x_bits, idx, E, R, fmt, B=128):
+def dispatch_case(oracle, x_bits, idx, E, R, fmt, B=128, x_offset=0):
+    """x_offset > 0 places x that many bf16 elements past an aligned base, so a
+    16-byte but not 32-byte aligned x takes the 16-byte kernels."""
     import combine_ep_layout_08_b200 as ep
     from gpu_util import DEV, bits_to_bf16, nonpad_rows
 
@@ -52,7 +54,13 @@ def dispatch_case(oracle, x_bits, idx, E, R, fmt, B=128):
     h = _handle(T, k, E, R, B)
     ep.ep_layout(h, torch.from_numpy(idx).to(DEV))
     P = lay.total_rows
-    x = bits_to_bf16(x_bits)
+    if x_offset:
+        base = torch.empty(T * H + x_offset, dtype=torch.bfloat16, device=DEV)
+        x = base[x_offset:].view(T, H)
+        x.copy_(bits_to_bf16(x_bits))
+        assert x.data_ptr() % 32 != 0 and x.data_ptr() % 16 == 0
+    else:
+        x = bits_to_bf16(x_bits)
     rows = nonpad_rows(lay)
     padr = np.nonzero(lay.recv_src < 0)[0]
     if fmt == "bf16":
@@ -107,6 +115,15 @@ def test_dispatch_fuzz(oracle, T, H, E, R, k, fmt, p_unused):
     x = make_x(T, H, rng)
     idx, _ = random_topk(T, E, k, rng, p_unused=p_unused)
     dispatch_case(oracle, x, idx, E, R, fmt)
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8"])
+def test_dispatch_16byte_kernels_on_unaligned_x(oracle, fmt):
+    rng = np.random.default_rng(11)
+    T, H, E, R, k = 150, 1024, 32, 8, 8
+    x = make_x(T, H, rng)
+    idx, _ = random_topk(T, E, k, rng, p_unused=0.1)
+    dispatch_case(oracle, x, idx, E, R, fmt, x_offset=8)
 
 
 def test_dispatch_fp8_special_values(oracle):

@@ -49,6 +49,9 @@ FUZZ = [
     (64, 8192, 8192, 4, 128, 0.0, True),   # maximum E, R = E
     (4096, 256, 256, 8, 128, 0.5, True),   # many unused slots
     (20000, 256, 8, 8, 128, 0.0, True),    # many chunks
+    (1024, 256, 16, 8, 128, 0.0, True),    # 32 chunks: the one-CTA path's limit
+    (1025, 256, 16, 8, 128, 0.0, True),    # 33 chunks: the three-kernel path
+    (1000, 2048, 8, 8, 128, 0.0, True),    # 32 chunks but counts too big for one CTA
 ]
 
 
@@ -115,6 +118,23 @@ def test_layout_bad_index_sets_error_and_is_skipped(oracle):
     assert_layout_equal(g, oracle.layout(clean, 64, 8))
     # the error word is cleared by the check
     assert ep.ep_handle_check(h, raise_on_error=False) == 0
+
+
+def test_layout_bad_index_large_batch(oracle):
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import assert_layout_equal
+
+    rng = np.random.default_rng(19)
+    idx, _ = random_topk(3000, 256, 8, rng)
+    bad = idx.copy()
+    bad[2999, 7] = 1 << 40
+    bad[1234, 0] = -2
+    g, st, _ = _run(bad, 256, 8)
+    assert st == ep.EP_ERR_BAD_INDEX
+    clean = bad.copy()
+    clean[2999, 7] = -1
+    clean[1234, 0] = -1
+    assert_layout_equal(g, oracle.layout(clean, 256, 8))
 
 
 def test_layout_counts_readback(oracle):
