@@ -27,9 +27,11 @@ import torch
 __all__ = [
     "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
     "ep_layout", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
+    "ep_dispatch_range", "ep_combine_range",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
+    "EP_ERR_TIMEOUT",
 ]
 
 EP_OK = 0
@@ -41,6 +43,7 @@ EP_ERR_BAD_INDEX = 5
 EP_ERR_CUDA = 6
 EP_ERR_STATE = 7
 EP_ERR_NO_MEMORY = 8
+EP_ERR_TIMEOUT = 9
 
 EP_FMT_BF16 = 0
 EP_FMT_FP8_E4M3_1X128 = 1
@@ -56,6 +59,7 @@ VIEWS = {
     "dst_row": (6, torch.int32),
     "recv_src": (7, torch.int32),
     "total_recv_rows": (8, torch.int32),
+    "error_words": (9, torch.int32),
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +95,8 @@ def load_library():
             "ep_handle_read_counts": ([P, P, P, P, P, P], I),
             "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
             "ep_combine": ([P, P, I64, P, I, P, P], I),
+            "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
+            "ep_combine_range": ([P, I, I, P, I64, P, I, P, P], I),
             "ep_handle_check": ([P, P], I),
             "ep_strerror": ([I], ctypes.c_char_p),
             "ep_last_error_message": ([], ctypes.c_char_p),
@@ -291,6 +297,44 @@ def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,
         _check(load_library().ep_combine(h.handle, _ptr(y), y.shape[0], _ptr(topk_weights), H,
                                          _ptr(out), _stream(h.device)), "ep_combine")
     return out
+
+
+def ep_dispatch_range(h: EPHandle, t_begin: int, x_rows: torch.Tensor, fmt: str,
+                      recv_x: torch.Tensor, recv_scales: Optional[torch.Tensor] = None) -> None:
+    """Dispatch tokens [t_begin, t_begin + len(x_rows)) of the last layout into
+    the given receive buffers (x_rows: contiguous bf16 [n, H], the rows of
+    those tokens)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch_range")
+    if x_rows.dtype != torch.bfloat16 or x_rows.dim() != 2 or not x_rows.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: x_rows must be contiguous bf16 [n, H]")
+    f = _FMTS[fmt]
+    n, H = x_rows.shape
+    if recv_x.shape[1] != H or not recv_x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: recv_x must be contiguous [*, H]")
+    with _on(h):
+        _check(load_library().ep_dispatch_range(
+            h.handle, t_begin, n, _ptr(x_rows), H, f, _ptr(recv_x),
+            _ptr(recv_scales) if f else ctypes.c_void_p(0), recv_x.shape[0], _stream(h.device)),
+            "ep_dispatch_range")
+
+
+def ep_combine_range(h: EPHandle, t_begin: int, y: torch.Tensor, topk_weights_rows: torch.Tensor,
+                     out_rows: torch.Tensor) -> None:
+    """Combine tokens [t_begin, t_begin + len(out_rows)) of the last layout
+    (topk_weights_rows: f32 [n, k]; out_rows: bf16 [n, H], contiguous)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_combine_range")
+    n, H = out_rows.shape
+    if (y.dtype != torch.bfloat16 or y.shape[1] != H or not y.is_contiguous()
+            or out_rows.dtype != torch.bfloat16 or not out_rows.is_contiguous()
+            or topk_weights_rows.dtype != torch.float32
+            or tuple(topk_weights_rows.shape) != (n, h.k) or not topk_weights_rows.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_range: bad tensor")
+    with _on(h):
+        _check(load_library().ep_combine_range(
+            h.handle, t_begin, n, _ptr(y), y.shape[0], _ptr(topk_weights_rows), H, _ptr(out_rows),
+            _stream(h.device)), "ep_combine_range")
 
 
 def ep_handle_check(h: EPHandle, raise_on_error: bool = True) -> int:

@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "ep_internal.cuh"
@@ -82,7 +83,7 @@ bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c)
     c->tokens_per_rank = take(sizeof(int32_t) * (size_t)R);
     c->rows_per_rank = take(sizeof(int32_t) * (size_t)R);
     c->total_rows = take(sizeof(int32_t));
-    c->err = take(sizeof(int32_t));
+    c->err = take(3 * sizeof(int32_t));
     c->is_token_in_rank = take((size_t)max_tokens * R);
     c->dst_row = take(sizeof(int32_t) * (size_t)max_tokens * k);
     c->recv_src = take(sizeof(int32_t) * (size_t)rows);
@@ -218,8 +219,9 @@ ep_status_t ep_layout(ep_handle_t hh, const int64_t* topk_idx, int T, void* stre
         return EP_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!h->err_cleared) {
-        // The workspace starts with unknown contents: zero the error word once.
-        cudaError_t rc = cudaMemsetAsync(h->err, 0, sizeof(int32_t), s);
+        // The workspace starts with unknown contents: zero the error word and
+        // the grid barrier's words once.
+        cudaError_t rc = cudaMemsetAsync(h->err, 0, 3 * sizeof(int32_t), s);
         if (rc != cudaSuccess)
             return ep::cuda_fail(rc, "ep_layout (clear error word)");
         h->err_cleared = 1;
@@ -252,6 +254,7 @@ const void* ep_handle_view(ep_handle_t hh, ep_view_t what, int64_t* count)
     case EP_VIEW_DST_ROW: p = h->dst_row; n = T * h->k; break;
     case EP_VIEW_RECV_SRC: p = h->recv_src; n = h->max_rows; break;
     case EP_VIEW_TOTAL_RECV_ROWS: p = h->total_rows; n = 1; break;
+    case EP_VIEW_ERROR_WORDS: p = h->err; n = 3; break;
     default: return nullptr;
     }
     if (count)
@@ -287,49 +290,102 @@ ep_status_t ep_handle_read_counts(ep_handle_t hh, int32_t* num_tokens_per_expert
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_handle_read_counts");
 }
 
-ep_status_t ep_dispatch(ep_handle_t hh, const void* x, int H, ep_fmt_t fmt, void* recv_x,
-                        float* recv_scales, int64_t recv_capacity_rows, void* stream)
+}  // extern "C"
+
+namespace {
+
+// Dispatch / combine of the tokens [t_begin, t_begin + t_count) of the last
+// layout: the kernels see a shallow copy of the handle whose token count and
+// dst_row start at the range.
+ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, int H,
+                          ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                          int64_t recv_capacity_rows, void* stream, const char* what)
 {
-    Handle* h = ep::as_handle(hh);
     if (!h || H <= 0 || recv_capacity_rows < 0)
         return EP_ERR_INVALID_ARG;
     if (!h->has_layout)
         return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
     if (fmt != EP_FMT_BF16 && fmt != EP_FMT_FP8_E4M3_1X128)
         return EP_ERR_INVALID_ARG;
     if (fmt == EP_FMT_BF16 && H % 8 != 0)
         return EP_ERR_INVALID_ARG;
     if (fmt == EP_FMT_FP8_E4M3_1X128 && H % 128 != 0)
         return EP_ERR_INVALID_ARG;
-    if (h->T > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
+    if (t_count > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
         return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_FP8_E4M3_1X128 && h->T > 0 && recv_capacity_rows > 0 && !recv_scales)
+    if (fmt == EP_FMT_FP8_E4M3_1X128 && t_count > 0 && recv_capacity_rows > 0 && !recv_scales)
         return EP_ERR_INVALID_ARG;
     if (!ep::aligned(x, 16) || !ep::aligned(recv_x, 16) || !ep::aligned(recv_scales, 16))
         return EP_ERR_ALIGNMENT;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t rc = (fmt == EP_FMT_BF16)
-                         ? ep::launch_dispatch_bf16(*h, x, H, recv_x, recv_capacity_rows, s)
-                         : ep::launch_dispatch_fp8(*h, x, H, recv_x, recv_scales,
+                         ? ep::launch_dispatch_bf16(sub, x, H, recv_x, recv_capacity_rows, s)
+                         : ep::launch_dispatch_fp8(sub, x, H, recv_x, recv_scales,
                                                    recv_capacity_rows, s);
-    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch");
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
+}
+
+ep_status_t combine_impl(Handle* h, int t_begin, int t_count, const void* y, int64_t y_rows,
+                         const float* topk_weights, int H, void* out, void* stream,
+                         const char* what)
+{
+    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    if (t_count > 0 && (!out || !topk_weights || (!y && y_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(y, 16) || !ep::aligned(out, 16) || !ep::aligned(topk_weights, 4))
+        return EP_ERR_ALIGNMENT;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = ep::launch_combine(sub, y, y_rows, topk_weights, H, out, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+ep_status_t ep_dispatch(ep_handle_t hh, const void* x, int H, ep_fmt_t fmt, void* recv_x,
+                        float* recv_scales, int64_t recv_capacity_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    return dispatch_impl(h, 0, h ? std::max(h->T, 0) : 0, x, H, fmt, recv_x, recv_scales,
+                         recv_capacity_rows, stream, "ep_dispatch");
+}
+
+ep_status_t ep_dispatch_range(ep_handle_t hh, int t_begin, int t_count, const void* x_rows,
+                              int H, ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                              int64_t recv_capacity_rows, void* stream)
+{
+    return dispatch_impl(ep::as_handle(hh), t_begin, t_count, x_rows, H, fmt, recv_x,
+                         recv_scales, recv_capacity_rows, stream, "ep_dispatch_range");
 }
 
 ep_status_t ep_combine(ep_handle_t hh, const void* y, int64_t y_rows, const float* topk_weights,
                        int H, void* out, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
-        return EP_ERR_INVALID_ARG;
-    if (!h->has_layout)
-        return EP_ERR_STATE;
-    if (h->T > 0 && (!out || !topk_weights || (!y && y_rows > 0)))
-        return EP_ERR_INVALID_ARG;
-    if (!ep::aligned(y, 16) || !ep::aligned(out, 16) || !ep::aligned(topk_weights, 4))
-        return EP_ERR_ALIGNMENT;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = ep::launch_combine(*h, y, y_rows, topk_weights, H, out, s);
-    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine");
+    return combine_impl(h, 0, h ? std::max(h->T, 0) : 0, y, y_rows, topk_weights, H, out, stream,
+                        "ep_combine");
+}
+
+ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const void* y,
+                             int64_t y_rows, const float* topk_weights_rows, int H,
+                             void* out_rows, void* stream)
+{
+    return combine_impl(ep::as_handle(hh), t_begin, t_count, y, y_rows, topk_weights_rows, H,
+                        out_rows, stream, "ep_combine_range");
 }
 
 ep_status_t ep_handle_check(ep_handle_t hh, void* stream)
@@ -344,12 +400,16 @@ ep_status_t ep_handle_check(ep_handle_t hh, void* stream)
     cudaError_t rc = cudaMemcpyAsync(&word, h->err, sizeof word, cudaMemcpyDeviceToHost, s);
     if (rc == cudaSuccess)
         rc = cudaStreamSynchronize(s);
+    // Clear the error word; after a barrier time-out also reset the barrier
+    // (its count is left mid-way).
     if (rc == cudaSuccess)
-        rc = cudaMemsetAsync(h->err, 0, sizeof(int32_t), s);
+        rc = cudaMemsetAsync(h->err, 0, ((word & ep::kErrTimeout) ? 3 : 1) * sizeof(int32_t), s);
     if (rc == cudaSuccess)
         rc = cudaStreamSynchronize(s);
     if (rc != cudaSuccess)
         return ep::cuda_fail(rc, "ep_handle_check");
+    if (word & ep::kErrTimeout)
+        return EP_ERR_TIMEOUT;
     if (word & ep::kErrBadIndex)
         return EP_ERR_BAD_INDEX;
     if (word & (ep::kErrDispatchCap | ep::kErrCombineCap))
@@ -369,6 +429,7 @@ const char* ep_strerror(ep_status_t status)
     case EP_ERR_CUDA: return "EP_ERR_CUDA: CUDA runtime error";
     case EP_ERR_STATE: return "EP_ERR_STATE: no layout on this handle";
     case EP_ERR_NO_MEMORY: return "EP_ERR_NO_MEMORY: host allocation failed";
+    case EP_ERR_TIMEOUT: return "EP_ERR_TIMEOUT: a device-side wait gave up; that call's outputs are invalid";
     }
     return "unknown ep_status_t";
 }

@@ -17,6 +17,7 @@ constexpr uint32_t kHandleMagic = 0x45504c38u;  // "EPL8"
 constexpr int kErrBadIndex = 1;      // top-k index outside [-1, E)
 constexpr int kErrDispatchCap = 2;   // dispatch row >= recv capacity
 constexpr int kErrCombineCap = 4;    // combine row >= y rows
+constexpr int kErrTimeout = 8;       // a grid barrier gave up waiting
 
 // The layout works on chunks of kChunkTokens consecutive tokens, one warp
 // per chunk: the (token, slot) entries of a chunk are contiguous in topk_idx.
@@ -36,7 +37,7 @@ struct Handle {
     int32_t* tokens_per_rank;// [R]
     int32_t* rows_per_rank;  // [R]
     int32_t* total_rows;     // [1]
-    int32_t* err;            // [1]
+    int32_t* err;            // [3] sticky error bits, then the grid barrier's count and generation
     uint8_t* is_token_in_rank;  // [max_tokens][R]
     int32_t* dst_row;        // [max_tokens][k]
     int32_t* recv_src;       // [max_rows]
@@ -83,7 +84,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
 }
 
 // Launchers (each returns the cudaError_t of its launches).
-cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s);
+// allow_fused: the single cooperative layout kernel may be used (needs the
+// grid barrier words at h.err[1..2], zero-initialised).
+cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s,
+                          bool allow_fused = true);
 cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,
                                  int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,

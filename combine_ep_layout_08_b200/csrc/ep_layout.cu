@@ -22,6 +22,9 @@
 //              warp replays its chunk in order, ranking equal experts inside
 //              each group of 32 entries with __match_any_sync, to give
 //              dst_row and recv_src; pad rows of recv_src are set to -1.
+// Large batches, one launch (the default): layout_fused_kernel runs the three
+// phases in one cooperative launch, its CTAs separated by two grid barriers;
+// the three kernels remain for launches a cooperative grid cannot serve.
 // Small batches (at most 32 chunks) run the same three phases inside one CTA
 // (layout_small_kernel), with the chunk counts in shared memory.
 //
@@ -103,20 +106,56 @@ __device__ void scan_padded(const int32_t* cnt, int E, int block_m, int32_t* off
 }
 
 // One warp: is_token_in_rank bytes of a chunk from the entries' ranks
-// (erank[t * k + j], -1 for unused), p = t * R + r so that consecutive lanes
-// write consecutive bytes; per-rank token counts go to rhist.
+// (erank[t * k + j], -1 for unused); byte p = t * R + r goes to lane p % 32,
+// so consecutive lanes write consecutive bytes.  Tokens-per-rank counts are
+// added to rhist.  With R <= 32 each token's ranks are first folded into a
+// bitmask held by lane t, the counts come from ballots, and each byte is one
+// shuffle; larger R tests the k entries per byte.
 __device__ __forceinline__ void chunk_rank_bytes(const int32_t* erank, int ntok, int k, int R,
                                                  int64_t t0, uint8_t* is_token_in_rank,
                                                  int32_t* rhist)
 {
     const int lane = threadIdx.x & 31;
-    for (int p = lane; p < ntok * R; p += 32) {
-        const int t = p / R, r = p - t * R;
-        int hit = 0;
-        for (int j = 0; j < k; ++j) hit |= (erank[t * k + j] == r);
-        is_token_in_rank[(t0 + t) * R + r] = (uint8_t)hit;
-        if (hit)
-            atomicAdd(&rhist[r], 1);
+    const int total = ntok * R;
+    const int dt = 32 / R, dr = 32 - (32 / R) * R;  // (t, r) step for p += 32
+    int t = lane / R, r = lane - (lane / R) * R;
+    if (R <= 32) {
+        uint32_t mask = 0;
+        if (lane < ntok)
+            for (int j = 0; j < k; ++j) {
+                const int q = erank[lane * k + j];
+                if (q >= 0)
+                    mask |= 1u << q;
+            }
+        for (int q = 0; q < R; ++q) {
+            const int c = __popc(__ballot_sync(kFull, (mask >> q) & 1u));
+            if (lane == 0 && c)
+                atomicAdd(&rhist[q], c);
+        }
+        for (int p0 = 0; p0 < total; p0 += 32) {
+            const uint32_t m = __shfl_sync(kFull, mask, t & 31);
+            if (p0 + lane < total)
+                is_token_in_rank[(t0 + t) * R + r] = (uint8_t)((m >> r) & 1u);
+            t += dt;
+            r += dr;
+            if (r >= R) {
+                r -= R;
+                ++t;
+            }
+        }
+    } else {
+        for (int p = lane; p < total; p += 32) {
+            int hit = 0;
+            for (int j = 0; j < k; ++j) hit |= (erank[t * k + j] == r);
+            is_token_in_rank[(t0 + t) * R + r] = (uint8_t)hit;
+            if (hit)
+                atomicAdd(&rhist[r], 1);
+            r += 32;
+            while (r >= R) {
+                r -= R;
+                ++t;
+            }
+        }
     }
 }
 
@@ -149,9 +188,13 @@ __device__ __forceinline__ void chunk_assign(const int32_t* ents, int nent, int 
 
 // One warp: load a chunk's entries (all loads of a batch issued first),
 // validate them into ents[] and, if erank is given, their ranks; count them
-// into hist (shared-memory atomics) if hist is given.
+// into hist (shared-memory atomics) if hist is given.  rank = floor(e / epr)
+// is (e * rank_magic) >> 32 with rank_magic = ceil(2^32 / epr): exact for
+// e, epr <= 2^13 (the error e * (rank_magic - 2^32/epr) / 2^32 < 2^-19 stays
+// below the 1/epr gap to the next integer).
 __device__ __forceinline__ int load_chunk(const int64_t* __restrict__ src, int nent, int E,
-                                          int epr, int32_t* ents, int32_t* erank, int32_t* hist)
+                                          uint64_t rank_magic, int32_t* ents, int32_t* erank,
+                                          int32_t* hist)
 {
     const int lane = threadIdx.x & 31;
     int bad = 0;
@@ -170,7 +213,7 @@ __device__ __forceinline__ int load_chunk(const int64_t* __restrict__ src, int n
                 if (ents)
                     ents[f] = e;
                 if (erank)
-                    erank[f] = e >= 0 ? e / epr : -1;
+                    erank[f] = e >= 0 ? (int32_t)(((uint64_t)e * rank_magic) >> 32) : -1;
                 if (hist && e >= 0)
                     atomicAdd(&hist[e], 1);
             }
@@ -181,7 +224,7 @@ __device__ __forceinline__ int load_chunk(const int64_t* __restrict__ src, int n
 
 // K1.  Shared memory per warp: hist[E], rank_hist[R], entry_rank[32 k].
 __global__ void layout_count_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                    int R, int epr, int64_t nchunks,
+                                    int R, uint64_t rank_magic, int64_t nchunks,
                                     int32_t* __restrict__ chunk_counts,
                                     int32_t* __restrict__ chunk_rank,
                                     uint8_t* __restrict__ is_token_in_rank, int32_t* err)
@@ -205,7 +248,7 @@ __global__ void layout_count_kernel(const int64_t* __restrict__ topk_idx, int T,
     for (int e = lane; e < E; e += 32) hist[e] = 0;
     for (int r = lane; r < R; r += 32) rhist[r] = 0;
     __syncwarp();
-    const int bad = load_chunk(topk_idx + t0 * k, nent, E, epr, nullptr, erank, hist);
+    const int bad = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, nullptr, erank, hist);
     if (bad && lane == 0)
         atomicOr(err, kErrBadIndex);
     __syncwarp();
@@ -286,7 +329,8 @@ layout_scan_kernel(int32_t* __restrict__ chunk_counts, const int32_t* __restrict
 
 // K3.  Shared memory: off[E+1], wsum[32], then per warp run[E] + ents[32 k].
 __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                     int R, int epr, int block_m, int64_t nchunks,
+                                     int R, int epr, uint64_t rank_magic, int block_m,
+                                     int64_t nchunks,
                                      const int32_t* __restrict__ chunk_prefix,
                                      const int32_t* __restrict__ cnt,
                                      int32_t* __restrict__ expert_off_g,
@@ -331,7 +375,7 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
                     runc[e] = v[m];
             }
         }
-        int ignored = load_chunk(topk_idx + t0 * k, nent, E, epr, ents, nullptr, nullptr);
+        int ignored = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, ents, nullptr, nullptr);
         (void)ignored;  // bad indices were flagged by the count pass
     }
     scan_padded(cnt, E, block_m, off, wsum);
@@ -365,7 +409,8 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
 // off[E+1], wsum[32], rank_hist[R], per chunk ents[32 k] + erank[32 k],
 // with nc = max(1, nchunks).
 __global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                    int R, int epr, int block_m, int64_t nchunks,
+                                    int R, int epr, uint64_t rank_magic, int block_m,
+                                    int64_t nchunks,
                                     int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
                                     int32_t* __restrict__ rank_off_g,
                                     int32_t* __restrict__ tokens_per_rank_g,
@@ -399,7 +444,7 @@ __global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T,
     const int ntok = has_chunk ? (int)min((int64_t)kChunkTokens, (int64_t)T - t0) : 0;
     const int nent = ntok * k;
     if (has_chunk) {
-        const int bad = load_chunk(topk_idx + t0 * k, nent, E, epr, ents, erank, hist);
+        const int bad = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, ents, erank, hist);
         if (bad && lane == 0)
             atomicOr(err, kErrBadIndex);
         __syncwarp();
@@ -443,6 +488,225 @@ __global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T,
     chunk_assign(ents, nent, k, t0, hist, dst_row, recv_src);
 }
 
+
+// ------------------------------------------------------------------ fused
+// Grid barrier over the CTAs of a cooperative launch (all co-resident).
+// bar[0] counts arrivals, bar[1] is the generation: the last CTA to arrive
+// resets the count and then bumps the generation, which releases the others.
+// The state is left ready for the next barrier and the next launch.  The wait
+// is bounded: past kSpinLimit polls the CTA sets kErrTimeout and the caller
+// abandons the launch (ep_handle_check then resets the barrier).
+constexpr uint32_t kSpinLimit = 1u << 20;  // polls of ~64 ns sleep + one L2 read
+
+__device__ bool grid_barrier(int32_t* bar, int nblocks, int32_t* err)
+{
+    __shared__ int ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile int32_t* vgen = bar + 1;
+        const int32_t gen = *vgen;
+        __threadfence();
+        int good = 1;
+        if (atomicAdd(bar, 1) == nblocks - 1) {
+            atomicExch(bar, 0);
+            __threadfence();
+            atomicAdd(bar + 1, 1);
+        } else {
+            uint32_t polls = 0;
+            while (*vgen == gen) {
+                if (++polls > kSpinLimit) {
+                    good = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        if (!good)
+            atomicOr(err, kErrTimeout);
+        ok = good;
+    }
+    __syncthreads();
+    return ok != 0;
+}
+
+// One warp scans column col of an [nchunks][ncol] count matrix: exclusive
+// prefix over chunks written in place (if write_prefix); the column total is
+// returned to every lane.  Each batch covers 32 x kBatch consecutive chunks,
+// lane l owning chunks l*kBatch .. l*kBatch + kBatch - 1 of it, so a chunk's
+// prefix = earlier batches' total + lower lanes' sums + its lane's earlier
+// chunks.  All loads of a batch are issued before any is used.
+__device__ int32_t column_scan(int32_t* M, int64_t nchunks, int ncol, int col, bool write_prefix)
+{
+    const int lane = threadIdx.x & 31;
+    int32_t base = 0;
+    for (int64_t b0 = 0; b0 < nchunks; b0 += 32 * kBatch) {
+        const int64_t r0 = b0 + (int64_t)lane * kBatch;
+        int32_t v[kBatch];
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m) v[m] = (r0 + m < nchunks) ? M[(r0 + m) * ncol + col] : 0;
+        int32_t sum = 0;
+#pragma unroll
+        for (int m = 0; m < kBatch; ++m) sum += v[m];
+        int32_t incl = sum;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o)
+                incl += u;
+        }
+        if (write_prefix) {
+            int32_t run = base + incl - sum;
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m)
+                if (r0 + m < nchunks) {
+                    M[(r0 + m) * ncol + col] = run;
+                    run += v[m];
+                }
+        }
+        base += __shfl_sync(kFull, incl, 31);
+    }
+    return base;
+}
+
+// Large batches in one cooperative launch of G CTAs x W warps (all
+// co-resident).  Shared memory: off[E+1], wsum[32], then per warp
+// E + R + 32 k words (phase 1: hist, rank_hist, entry ranks; phase 3: run,
+// entries).  Chunks are taken grid-stride by warp, so G may be smaller than
+// the chunk count.
+__global__ void layout_fused_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
+                                    int R, int epr, uint64_t rank_magic, int block_m,
+                                    int64_t nchunks,
+                                    int32_t* __restrict__ chunk_counts,
+                                    int32_t* __restrict__ chunk_rank, int32_t* __restrict__ cnt_g,
+                                    int32_t* __restrict__ expert_off_g,
+                                    int32_t* __restrict__ rank_off_g,
+                                    int32_t* __restrict__ tokens_per_rank_g,
+                                    int32_t* __restrict__ rows_per_rank_g,
+                                    int32_t* __restrict__ total_rows_g,
+                                    uint8_t* __restrict__ is_token_in_rank,
+                                    int32_t* __restrict__ dst_row, int32_t* __restrict__ recv_src,
+                                    int32_t* err)
+{
+    extern __shared__ int32_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5, nthr = blockDim.x;
+    const int64_t gwarp = (int64_t)blockIdx.x * nwarps + warp;
+    const int64_t nwarps_all = (int64_t)gridDim.x * nwarps;
+    int32_t* off = smem;
+    int32_t* wsum = off + E + 1;
+    int32_t* mine = wsum + 32 + (size_t)warp * (E + R + kChunkTokens * k);
+    int32_t* bar = err + 1;
+
+    // A barrier that timed out earlier leaves its words inconsistent until
+    // ep_handle_check resets them: refuse to run (every CTA reads the same word).
+    __shared__ int stale;
+    if (threadIdx.x == 0)
+        stale = (*(volatile int32_t*)err & kErrTimeout) != 0;
+    __syncthreads();
+    if (stale)
+        return;
+
+    // phase 1: per-chunk histograms, is_token_in_rank, per-chunk rank counts
+    {
+        int32_t* hist = mine;
+        int32_t* rhist = hist + E;
+        int32_t* erank = rhist + R;
+        for (int64_t c = gwarp; c < nchunks; c += nwarps_all) {
+            const int64_t t0 = c * kChunkTokens;
+            const int ntok = (int)min((int64_t)kChunkTokens, (int64_t)T - t0);
+            const int nent = ntok * k;
+            for (int e = lane; e < E; e += 32) hist[e] = 0;
+            for (int r = lane; r < R; r += 32) rhist[r] = 0;
+            __syncwarp();
+            const int bad = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, nullptr, erank, hist);
+            if (bad && lane == 0)
+                atomicOr(err, kErrBadIndex);
+            __syncwarp();
+            chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
+            __syncwarp();
+            for (int e = lane; e < E; e += 32) chunk_counts[c * E + e] = hist[e];
+            for (int r = lane; r < R; r += 32) chunk_rank[c * R + r] = rhist[r];
+            __syncwarp();
+        }
+    }
+    if (!grid_barrier(bar, gridDim.x, err))
+        return;
+
+    // phase 2: one warp per column -- experts (prefix + total), then ranks (total)
+    for (int64_t col = gwarp; col < E + R; col += nwarps_all) {
+        if (col < E) {
+            const int32_t tot = column_scan(chunk_counts, nchunks, E, (int)col, true);
+            if (lane == 0)
+                cnt_g[col] = tot;
+        } else {
+            const int32_t tot = column_scan(chunk_rank, nchunks, R, (int)(col - E), false);
+            if (lane == 0)
+                tokens_per_rank_g[col - E] = tot;
+        }
+    }
+    if (!grid_barrier(bar, gridDim.x, err))
+        return;
+
+    // phase 3: offsets (every CTA), bookkeeping (CTA 0), pad rows, assignment.
+    // A chunk's prefix row (into run) and entries do not depend on the
+    // offsets: the first chunk's loads are issued before the offset scan.
+    int32_t* runc = mine;
+    int32_t* ents = runc + E;
+    auto fetch = [&](int64_t c) {
+        const int64_t t0 = c * kChunkTokens;
+        const int nent = (int)min((int64_t)kChunkTokens, (int64_t)T - t0) * k;
+        for (int base = 0; base < E; base += 32 * kBatch) {
+            int32_t v[kBatch];
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m) {
+                const int e = base + m * 32 + lane;
+                v[m] = e < E ? chunk_counts[c * E + e] : 0;
+            }
+#pragma unroll
+            for (int m = 0; m < kBatch; ++m) {
+                const int e = base + m * 32 + lane;
+                if (e < E)
+                    runc[e] = v[m];
+            }
+        }
+        const int ignored = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, ents, nullptr,
+                                       nullptr);
+        (void)ignored;
+    };
+    if (gwarp < nchunks)
+        fetch(gwarp);
+    scan_padded(cnt_g, E, block_m, off, wsum);
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
+        for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
+        for (int r = threadIdx.x; r < R; r += nthr) {
+            int32_t s = 0;
+            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt_g[e];
+            rows_per_rank_g[r] = s;
+        }
+        if (threadIdx.x == 0)
+            *total_rows_g = off[E];
+    }
+    for (int64_t e = gwarp; e < E; e += nwarps_all)
+        for (int32_t r = off[e] + cnt_g[e] + lane; r < off[e + 1]; r += 32)
+            recv_src[r] = -1;
+
+    for (int64_t c = gwarp; c < nchunks; c += nwarps_all) {
+        if (c != gwarp)
+            fetch(c);
+        const int64_t t0 = c * kChunkTokens;
+        const int nent = (int)min((int64_t)kChunkTokens, (int64_t)T - t0) * k;
+        for (int e = lane; e < E; e += 32) runc[e] += off[e];
+        __syncwarp();
+        chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
+        __syncwarp();
+    }
+}
+
+uint64_t rank_magic_for(int epr) { return ((uint64_t(1) << 32) + (uint64_t)epr - 1) / (uint64_t)epr; }
+
 int warps_for(size_t per_warp_bytes, size_t fixed_bytes)
 {
     size_t w = 4;
@@ -465,7 +729,48 @@ size_t small_layout_smem(int k, int E, int R, int64_t nchunks)
     return sizeof(int32_t) * (size_t)(nc * E + E + E + 1 + 32 + R + nc * 2 * kChunkTokens * k);
 }
 
-cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s)
+// The fused layout: W warps per CTA from the shared-memory budget, G CTAs =
+// min(CTAs the chunks need, CTAs that fit on the GPU at once).
+cudaError_t launch_fused(const Handle& h, const int64_t* topk_idx, int T, int64_t nchunks,
+                         cudaStream_t s)
+{
+    const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
+    const size_t fixed = sizeof(int32_t) * (size_t)(E + 1 + 32);
+    const size_t per_warp = sizeof(int32_t) * (size_t)(E + R + kChunkTokens * k);
+    const int w = warps_for(per_warp, fixed);
+    const size_t smem = fixed + per_warp * w;
+    cudaError_t rc;
+    if ((rc = set_smem((const void*)layout_fused_kernel, smem)) != cudaSuccess)
+        return rc;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+        (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, 32 * w,
+                                                            smem)) != cudaSuccess)
+        return rc;
+    if (per_sm < 1)
+        return cudaErrorCooperativeLaunchTooLarge;
+    const int64_t want = (nchunks + w - 1) / w;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * per_sm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * w);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, T, k, E, R, epr,
+                              rank_magic_for(epr), h.block_m,
+                              nchunks, h.chunk_counts, h.chunk_rank, h.cnt, h.expert_off,
+                              h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
+                              h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
+}
+
+cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s,
+                          bool allow_fused)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
     const int64_t nchunks = ((int64_t)T + kChunkTokens - 1) / kChunkTokens;
@@ -479,10 +784,17 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
                 return rc;
             const unsigned nw = (unsigned)std::max<int64_t>(8, nchunks);
             return launch_pdl(layout_small_kernel, 1, 32 * nw, smem, s, topk_idx, T, k, E, R, epr,
-                              h.block_m, nchunks, h.cnt, h.expert_off, h.rank_off,
+                              rank_magic_for(epr), h.block_m, nchunks, h.cnt, h.expert_off, h.rank_off,
                               h.tokens_per_rank, h.rows_per_rank, h.total_rows,
                               h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
         }
+    }
+
+    if (allow_fused && nchunks > 0) {
+        rc = launch_fused(h, topk_idx, T, nchunks, s);
+        if (rc != cudaErrorCooperativeLaunchTooLarge && rc != cudaErrorNotSupported)
+            return rc;
+        (void)cudaGetLastError();  // clear the refused launch; use three kernels
     }
 
     if (nchunks > 0) {
@@ -493,7 +805,7 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
             return rc;
         const unsigned g1 = (unsigned)((nchunks + w1 - 1) / w1);
         if ((rc = launch_pdl(layout_count_kernel, g1, 32 * w1, smem1, s, topk_idx, T, k, E, R,
-                             epr, nchunks, h.chunk_counts, h.chunk_rank, h.is_token_in_rank,
+                             rank_magic_for(epr), nchunks, h.chunk_counts, h.chunk_rank, h.is_token_in_rank,
                              h.err)) != cudaSuccess)
             return rc;
     }
@@ -511,7 +823,7 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
         return rc;
     const unsigned g3 = (unsigned)std::max<int64_t>(1, (nchunks + w3 - 1) / w3);
     return launch_pdl(layout_assign_kernel, g3, 32 * w3, smem3, s, topk_idx, T, k, E, R, epr,
-                      h.block_m, nchunks, h.chunk_counts, h.cnt, h.expert_off, h.rank_off,
+                      rank_magic_for(epr), h.block_m, nchunks, h.chunk_counts, h.cnt, h.expert_off, h.rank_off,
                       h.rows_per_rank, h.total_rows, h.dst_row, h.recv_src);
 }
 

@@ -117,6 +117,6 @@ extern "C" ep_status_t ep_layout_static_scratch(
     h.T = T;
     h.has_layout = 1;
     h.err_cleared = 1;
-    rc = ep::launch_layout(h, topk_idx, T, s);
+    rc = ep::launch_layout(h, topk_idx, T, s, /*allow_fused=*/false);
     return rc == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }

@@ -45,7 +45,9 @@
  * [-1, E), a receive row beyond the capacity given) set bits in a sticky
  * device error word inside the workspace; the offending rows are skipped,
  * nothing out of bounds is touched, and ep_handle_check reports them.  No
- * kernel traps and no kernel waits on another.
+ * kernel traps.  The one device-side wait -- the grid barrier between the
+ * phases of the single-launch layout, whose CTAs are co-resident by a
+ * cooperative launch -- has an iteration limit and reports EP_ERR_TIMEOUT.
  *
  * Thread safety: calls on one handle must not run concurrently from several
  * host threads; distinct handles are independent.
@@ -71,7 +73,11 @@ typedef enum {
     EP_ERR_BAD_INDEX = 5,            /* a top-k index outside [-1, E) */
     EP_ERR_CUDA = 6,                 /* a CUDA runtime call failed; see ep_last_error_message */
     EP_ERR_STATE = 7,                /* e.g. dispatch/combine before any ep_layout */
-    EP_ERR_NO_MEMORY = 8             /* host malloc of the handle failed */
+    EP_ERR_NO_MEMORY = 8,            /* host malloc of the handle failed */
+    EP_ERR_TIMEOUT = 9               /* a device-side wait (the layout's grid barrier) gave up
+                                        after its iteration limit; that call's outputs are
+                                        invalid.  Reported by ep_handle_check, which also
+                                        resets the barrier. */
 } ep_status_t;
 
 typedef enum {
@@ -89,7 +95,10 @@ typedef enum {
     EP_VIEW_IS_TOKEN_IN_RANK = 5,      /* uint8 [T][R]  1 if token t sends to rank r */
     EP_VIEW_DST_ROW = 6,               /* int32 [T][k]  receive row of slot (t,j), -1 unused */
     EP_VIEW_RECV_SRC = 7,              /* int32 [P]     source token of each row, -1 on pad */
-    EP_VIEW_TOTAL_RECV_ROWS = 8        /* int32 [1]     P, the padded receive rows */
+    EP_VIEW_TOTAL_RECV_ROWS = 8,       /* int32 [1]     P, the padded receive rows */
+    EP_VIEW_ERROR_WORDS = 9            /* int32 [3]     diagnostics: the sticky error bits,
+                                          then the layout grid barrier's count and
+                                          generation (do not write while work is queued) */
 } ep_view_t;
 
 /* Limits of this build. */
@@ -174,9 +183,26 @@ ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void*
 ep_status_t ep_combine(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
                        int H, void* out, void* stream);
 
+/* Dispatch / combine a contiguous range of the last layout's tokens,
+ * [t_begin, t_begin + t_count), 0 <= t_begin <= t_begin + t_count <= T.
+ * Same semantics, formats and errors as ep_dispatch / ep_combine restricted
+ * to those tokens; x_rows, topk_weights_rows and out_rows point at the rows
+ * of token t_begin (x_rows: bf16 [t_count][H]; topk_weights_rows: fp32
+ * [t_count][k]; out_rows: bf16 [t_count][H]).  recv_x, recv_scales and y are
+ * the whole receive-layout buffers.  The ranges of one layout may run in any
+ * order and on different streams: they write disjoint rows.  This lets a
+ * caller overlap the transfer of token chunks (host copies, or an upstream
+ * producer) with dispatch and combine of the chunks already present. */
+ep_status_t ep_dispatch_range(ep_handle_t h, int t_begin, int t_count, const void* x_rows, int H,
+                              ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                              int64_t recv_capacity_rows, void* stream);
+ep_status_t ep_combine_range(ep_handle_t h, int t_begin, int t_count, const void* y,
+                             int64_t y_rows, const float* topk_weights_rows, int H,
+                             void* out_rows, void* stream);
+
 /* Wait for the stream (SYNCHRONISING), read and clear the sticky device
- * error word.  Returns EP_ERR_BAD_INDEX, EP_ERR_CAPACITY (bad index wins if
- * both are set) or EP_OK. */
+ * error word.  Returns EP_ERR_TIMEOUT, EP_ERR_BAD_INDEX or EP_ERR_CAPACITY
+ * (in that order of precedence when several are set) or EP_OK. */
 ep_status_t ep_handle_check(ep_handle_t h, void* stream);
 
 /* ------------------------------------------------------------------------

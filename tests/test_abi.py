@@ -141,6 +141,8 @@ def test_views_point_into_the_workspace(lib):
         spans.append((p, name))
     assert len(set(p for p, _ in spans)) == len(spans)
     assert lib.ep_handle_view(h, 99, None) is None
+    n = ctypes.c_int64()
+    assert lib.ep_handle_view(h, 9, ctypes.byref(n)) and n.value == 3
     lib.ep_handle_destroy(h)
 
 

@@ -163,3 +163,26 @@ def test_layout_deterministic():
     b = gpu_layout(h)
     for key in a:
         assert np.array_equal(np.asarray(a[key]), np.asarray(b[key])), key
+
+
+def test_barrier_timeout_is_reported_and_recovered(oracle):
+    """The cooperative layout's grid barrier has an iteration limit.  Make it
+    run out on purpose (an arrival count that can never complete), check the
+    status, then check that the handle works again after ep_handle_check."""
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV, assert_layout_equal, gpu_layout
+
+    rng = np.random.default_rng(23)
+    idx, _ = random_topk(4096, 256, 8, rng)   # 128 chunks: the cooperative path
+    d_idx = torch.from_numpy(idx).to(DEV)
+    h = ep.ep_handle_create(4096, 8, 256, 8, device=DEV)
+    ep.ep_layout(h, d_idx)
+    assert ep.ep_handle_check(h, raise_on_error=False) == 0
+    words = ep.ep_handle_view(h, "error_words")
+    words[1] = -(1 << 30)                     # arrivals never reach the CTA count
+    ep.ep_layout(h, d_idx)
+    assert ep.ep_handle_check(h, raise_on_error=False) == ep.EP_ERR_TIMEOUT
+    assert words.cpu().tolist() == [0, 0, 0]   # error bits and barrier reset
+    ep.ep_layout(h, d_idx)                    # the barrier was reset: works again
+    assert ep.ep_handle_check(h, raise_on_error=False) == 0
+    assert_layout_equal(gpu_layout(h), oracle.layout(idx, 256, 8))

@@ -57,11 +57,12 @@ def test_full_config_pipeline(oracle, name):
     assert (go == ref["out"]).mean() == 1.0
 
 
-def test_cuda_graph_replay_matches_eager(oracle):
+@pytest.mark.parametrize("name", ["decode", "dsv3"])  # one-CTA and cooperative layouts
+def test_cuda_graph_replay_matches_eager(oracle, name):
     import combine_ep_layout_08_b200 as ep
     from gpu_util import DEV, bf16_to_bits, bits_to_bf16
 
-    w = make_workload("decode", 0)
+    w = make_workload(name, 0, H=1024)
     h = ep.ep_handle_create(w.T, w.k, w.E, w.R, device=DEV)
     x = bits_to_bf16(w.x_bits)
     idx = torch.from_numpy(w.topk_idx).to(DEV)
@@ -117,3 +118,45 @@ def test_pipeline_bitwise_deterministic():
     b = (recv2.view(torch.uint8).cpu().numpy()[rows], sc2.cpu().numpy()[rows], bf16_to_bits(out2))
     for u, v in zip(a, b):
         assert np.array_equal(u.view(np.uint8), v.view(np.uint8))
+
+
+@pytest.mark.parametrize("name,T,H", [("8k", 1000, 1024), ("skewed", 2048, 1024)])
+def test_token_ranges_match_the_whole_call(oracle, name, T, H):
+    """Dispatch and combine of token ranges (uneven, one empty, on two streams)
+    write exactly what the whole-batch calls write."""
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV, bf16_to_bits, bits_to_bf16
+    from workloads import make_x
+
+    w = make_workload(name, 0, T=T, H=H)
+    h = ep.ep_handle_create(w.T, w.k, w.E, w.R, device=DEV)
+    x = bits_to_bf16(w.x_bits)
+    wt = torch.from_numpy(w.topk_weights).to(DEV)
+    ep.ep_layout(h, torch.from_numpy(w.topk_idx).to(DEV))
+    recv_full, sc_full = ep.ep_dispatch(h, x, w.fmt)
+    cap = recv_full.shape[0]
+    lay = oracle.layout(w.topk_idx, w.E, w.R)
+    y = bits_to_bf16(make_x(max(lay.total_rows, 1), H, np.random.default_rng(4)))
+    out_full = ep.ep_combine(h, y, wt)
+    recv = torch.empty_like(recv_full)
+    sc = None if sc_full is None else torch.empty_like(sc_full)
+    out = torch.empty_like(out_full)
+    cuts = [0, 300, 300, 777, T]
+    streams = [torch.cuda.Stream(device=DEV), torch.cuda.Stream(device=DEV)]
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(cuts[:-1], cuts[1:])):
+        with torch.cuda.stream(streams[i % 2]):
+            ep.ep_dispatch_range(h, a, x[a:b], w.fmt, recv, sc)
+            ep.ep_combine_range(h, a, y, wt[a:b], out[a:b])
+    torch.cuda.synchronize()
+    assert ep.ep_handle_check(h, raise_on_error=False) == 0
+    rows = lay.dst_row[lay.dst_row >= 0]
+    assert np.array_equal(recv.view(torch.uint8).cpu().numpy()[rows],
+                          recv_full.view(torch.uint8).cpu().numpy()[rows])
+    if sc is not None:
+        assert np.array_equal(sc.cpu().numpy()[rows], sc_full.cpu().numpy()[rows])
+    assert np.array_equal(bf16_to_bits(out), bf16_to_bits(out_full))
+    assert np.array_equal(bf16_to_bits(out_full), oracle.combine(bf16_to_bits(y), w.topk_weights,
+                                                                 lay.dst_row))
+    with pytest.raises(ep.EPError):
+        ep.ep_dispatch_range(h, T - 10, x[:20], w.fmt, recv, sc)   # past the last token
