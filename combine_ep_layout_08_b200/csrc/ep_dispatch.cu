@@ -18,12 +18,15 @@
 // bytes of a row, so every store instruction covers whole 32-byte sectors.
 // The main kernels move 32-byte vectors (sm_100's 256-bit ld/st.global.v8),
 // halving the store instructions of 16-byte vectors; 16-byte kernels remain
-// for rows that are not 32-byte multiples.  The grid is two waves of resident
-// CTAs striding over units: with a single persistent wave every warp loads,
-// then stores, in lock step with all the others, and measured write
-// bandwidth drops by ~8 %; the second wave staggers those phases.
+// for rows that are not 32-byte multiples.  The grid gives every warp one
+// unit (a grid-stride loop covers grids beyond kMaxGrid): measured on B200,
+// a persistent single wave, in which every warp loads and then stores in
+// lock step with all the others, reaches ~5.4 TB/s; two waves 5.8; one unit
+// per warp, whose CTAs start and retire staggered, 6.1 TB/s.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+
+#include <algorithm>
 
 #include "ep_internal.cuh"
 
@@ -61,8 +64,11 @@ __device__ __forceinline__ void st32(Vec32* p, const Vec32& v)
                  : "memory");
 }
 
-constexpr int kU32 = 2;                 // 32-byte vectors per lane per unit
-constexpr int kUnitVec32 = 32 * kU32;   // 64 vectors x 16 channels = 1024 channels
+constexpr int kU32 = 1;                 // 32-byte vectors per lane per BF16 unit
+constexpr int kUnitVec32 = 32 * kU32;   // 32 vectors x 16 channels = 512 channels
+constexpr int kU32Fp8 = 2;              // FP8 unit: 64 vectors = 1024 channels = 8 blocks
+constexpr int kUnitVec32Fp8 = 32 * kU32Fp8;
+constexpr int64_t kMaxGrid = 1 << 20;
 
 // BF16 dispatch with 32-byte vectors; vpr = H / 16.
 __global__ void __launch_bounds__(kThreads, 8)
@@ -263,22 +269,22 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
     const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
     const int64_t vpr = H / 16;
     const int nblk = H / 128;
-    const int64_t upr = (vpr + kUnitVec32 - 1) / kUnitVec32;
+    const int64_t upr = (vpr + kUnitVec32Fp8 - 1) / kUnitVec32Fp8;
     const int64_t units = (int64_t)T * upr;
 
     for (int64_t u = wg; u < units; u += nw) {
         const int64_t t = u / upr;
         const int64_t unit = u - t * upr;
-        const int64_t v0 = unit * kUnitVec32 + lane;
+        const int64_t v0 = unit * kUnitVec32Fp8 + lane;
         int d = lane < k ? __ldg(dst_row + t * k + lane) : -1;
         if (d >= cap_rows) {
             atomicOr(err, kErrDispatchCap);
             d = -1;
         }
         const Vec32* xs = x + t * vpr;
-        Vec32 a[kU32];
+        Vec32 a[kU32Fp8];
 #pragma unroll
-        for (int i = 0; i < kU32; ++i) {
+        for (int i = 0; i < kU32Fp8; ++i) {
             if (v0 + 32 * i < vpr) {
                 a[i] = ld32_once(xs + v0 + 32 * i);
             } else {
@@ -287,10 +293,10 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
             }
         }
 
-        uint4 q[kU32];
-        float sc[kU32];
+        uint4 q[kU32Fp8];
+        float sc[kU32Fp8];
 #pragma unroll
-        for (int i = 0; i < kU32; ++i) {
+        for (int i = 0; i < kU32Fp8; ++i) {
             float f[16];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -323,7 +329,7 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
         // lane group L % 4 (leader lane 8 (L % 4))
         float my_scale = 0.0f;
 #pragma unroll
-        for (int i = 0; i < kU32; ++i) {
+        for (int i = 0; i < kU32Fp8; ++i) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 const float sv = __shfl_sync(kFull, sc[i], 8 * g);
@@ -331,8 +337,8 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                     my_scale = sv;
             }
         }
-        const int64_t blk = unit * (4 * kU32) + lane;
-        const bool sc_ok = lane < 4 * kU32 && blk < nblk;
+        const int64_t blk = unit * (4 * kU32Fp8) + lane;
+        const bool sc_ok = lane < 4 * kU32Fp8 && blk < nblk;
 
         for (int j = 0; j < k; ++j) {
             const int dj = __shfl_sync(kFull, d, j);
@@ -340,7 +346,7 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                 continue;
             uint4* dq = reinterpret_cast<uint4*>(recv_q + (int64_t)dj * H);
 #pragma unroll
-            for (int i = 0; i < kU32; ++i)
+            for (int i = 0; i < kU32Fp8; ++i)
                 if (v0 + 32 * i < vpr)
                     dq[v0 + 32 * i] = q[i];
             if (sc_ok)
@@ -351,6 +357,14 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
 
 bool aligned32(const void* p) { return ((uintptr_t)p & 31u) == 0; }
 
+// One unit per warp: ceil(units / warps per CTA) CTAs, capped at kMaxGrid.
+unsigned unit_grid(int64_t T, int64_t vec_per_row, int64_t unit_vec)
+{
+    const int64_t units = T * ((vec_per_row + unit_vec - 1) / unit_vec);
+    const int64_t warps = kThreads / 32;
+    return (unsigned)std::min<int64_t>(kMaxGrid, std::max<int64_t>(1, (units + warps - 1) / warps));
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,
@@ -358,22 +372,13 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
 {
     if (h.T == 0)
         return cudaSuccess;
-    int grid = 0;
-    cudaError_t rc;
-    if (H % 16 == 0 && aligned32(x) && aligned32(recv_x)) {
-        if ((rc = persistent_grid((const void*)dispatch_bf16_v32_kernel, kThreads, 0, 8, &grid)) !=
-            cudaSuccess)
-            return rc;
-        return launch_pdl(dispatch_bf16_v32_kernel, 2 * grid, kThreads, 0, s, 
-            static_cast<const Vec32*>(x), h.T, h.k, (int64_t)H / 16, h.dst_row,
-            static_cast<Vec32*>(recv_x), cap_rows, h.err);
-    }
-    if ((rc = persistent_grid((const void*)dispatch_bf16_kernel, kThreads, 0, 8, &grid)) !=
-        cudaSuccess)
-        return rc;
-    return launch_pdl(dispatch_bf16_kernel, 2 * grid, kThreads, 0, s, 
-        static_cast<const uint4*>(x), h.T, h.k, (int64_t)H / 8, h.dst_row,
-        static_cast<uint4*>(recv_x), cap_rows, h.err);
+    if (H % 16 == 0 && aligned32(x) && aligned32(recv_x))
+        return launch_pdl(dispatch_bf16_v32_kernel, unit_grid(h.T, H / 16, kUnitVec32), kThreads,
+                          0, s, static_cast<const Vec32*>(x), h.T, h.k, (int64_t)H / 16,
+                          h.dst_row, static_cast<Vec32*>(recv_x), cap_rows, h.err);
+    return launch_pdl(dispatch_bf16_kernel, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
+                      static_cast<const uint4*>(x), h.T, h.k, (int64_t)H / 8, h.dst_row,
+                      static_cast<uint4*>(recv_x), cap_rows, h.err);
 }
 
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
@@ -381,22 +386,13 @@ cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* rec
 {
     if (h.T == 0)
         return cudaSuccess;
-    int grid = 0;
-    cudaError_t rc;
-    if (aligned32(x)) {
-        if ((rc = persistent_grid((const void*)dispatch_fp8_v32_kernel, kThreads, 0, 8, &grid)) !=
-            cudaSuccess)
-            return rc;
-        return launch_pdl(dispatch_fp8_v32_kernel, 2 * grid, kThreads, 0, s, 
-            static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row, static_cast<uint8_t*>(recv_q),
-            recv_scales, cap_rows, h.err);
-    }
-    if ((rc = persistent_grid((const void*)dispatch_fp8_kernel, kThreads, 0, 8, &grid)) !=
-        cudaSuccess)
-        return rc;
-    return launch_pdl(dispatch_fp8_kernel, 2 * grid, kThreads, 0, s, static_cast<const uint4*>(x), h.T, h.k, H,
-                                                      h.dst_row, static_cast<uint8_t*>(recv_q),
-                                                      recv_scales, cap_rows, h.err);
+    if (aligned32(x))
+        return launch_pdl(dispatch_fp8_v32_kernel, unit_grid(h.T, H / 16, kUnitVec32Fp8),
+                          kThreads, 0, s, static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row,
+                          static_cast<uint8_t*>(recv_q), recv_scales, cap_rows, h.err);
+    return launch_pdl(dispatch_fp8_kernel, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
+                      static_cast<const uint4*>(x), h.T, h.k, H, h.dst_row,
+                      static_cast<uint8_t*>(recv_q), recv_scales, cap_rows, h.err);
 }
 
 }  // namespace ep

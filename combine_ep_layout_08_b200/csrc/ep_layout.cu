@@ -22,9 +22,10 @@
 //              warp replays its chunk in order, ranking equal experts inside
 //              each group of 32 entries with __match_any_sync, to give
 //              dst_row and recv_src; pad rows of recv_src are set to -1.
-// Large batches, one launch (the default): layout_fused_kernel runs the three
-// phases in one cooperative launch, its CTAs separated by two grid barriers;
-// the three kernels remain for launches a cooperative grid cannot serve.
+// Large batches, one launch (the default): layout_tile_kernel runs the three
+// phases in one cooperative launch over 64-token tiles, its CTAs separated by
+// two grid barriers; the three kernels remain for shapes whose tile counts do
+// not fit in shared memory and for the static-scratch entry point.
 // Small batches (at most 32 chunks) run the same three phases inside one CTA
 // (layout_small_kernel), with the chunk counts in shared memory.
 //
@@ -157,6 +158,24 @@ __device__ __forceinline__ void chunk_rank_bytes(const int32_t* erank, int ntok,
             }
         }
     }
+}
+
+// One warp: recv_src[a, b) = -1 (an expert's pad rows), with 16-byte stores
+// over the 4-aligned middle when the array is 16-byte aligned (vec).
+__device__ __forceinline__ void fill_pad(int32_t* recv_src, int32_t a, int32_t b, bool vec)
+{
+    const int lane = threadIdx.x & 31;
+    if (!vec || b - a < 8) {
+        for (int32_t r = a + lane; r < b; r += 32) recv_src[r] = -1;
+        return;
+    }
+    const int32_t a4 = (a + 3) & ~3, b4 = b & ~3;
+    if (lane < a4 - a)
+        recv_src[a + lane] = -1;
+    if (lane < b - b4)
+        recv_src[b4 + lane] = -1;
+    const int4 m1 = make_int4(-1, -1, -1, -1);
+    for (int32_t r = a4 + 4 * lane; r < b4; r += 128) *reinterpret_cast<int4*>(recv_src + r) = m1;
 }
 
 // One warp: replay a chunk's entries (ents in smem, -1 unused) in order and
@@ -391,10 +410,10 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
         if (threadIdx.x == 0)
             *total_rows_g = off[E];
     }
-    // Pad rows of the experts this CTA owns.
-    for (int e = blockIdx.x; e < E; e += gridDim.x)
-        for (int32_t r = off[e] + cnt[e] + (int32_t)threadIdx.x; r < off[e + 1]; r += nthr)
-            recv_src[r] = -1;
+    // Pad rows: one warp per expert over the whole grid.
+    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
+    for (int64_t e = (int64_t)blockIdx.x * nwarps + warp; e < E; e += (int64_t)gridDim.x * nwarps)
+        fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
     if (!has_chunk)
         return;  // no block barrier follows
@@ -404,7 +423,7 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
 }
 
 // Small batches: the three phases in one CTA; warp w < nchunks owns chunk w,
-// and at least 8 warps share the scans and the pad fill.
+// and at least 16 warps share the scans and the pad fill.
 // Shared memory: hist[nc][E] (then per-chunk prefixes, then run), cnt[E],
 // off[E+1], wsum[32], rank_hist[R], per chunk ents[32 k] + erank[32 k],
 // with nc = max(1, nchunks).
@@ -476,10 +495,9 @@ __global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T,
     }
     if (threadIdx.x == 0)
         *total_rows_g = off[E];
-    // pad rows: one warp per expert, lanes on consecutive rows
-    for (int e = warp; e < E; e += nwarps)
-        for (int32_t r = off[e] + cnt[e] + lane; r < off[e + 1]; r += 32)
-            recv_src[r] = -1;
+    // pad rows: one warp per expert
+    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
+    for (int e = warp; e < E; e += nwarps) fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
     if (!has_chunk)
         return;
@@ -491,29 +509,47 @@ __global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T,
 
 // ------------------------------------------------------------------ fused
 // Grid barrier over the CTAs of a cooperative launch (all co-resident).
-// bar[0] counts arrivals, bar[1] is the generation: the last CTA to arrive
-// resets the count and then bumps the generation, which releases the others.
-// The state is left ready for the next barrier and the next launch.  The wait
-// is bounded: past kSpinLimit polls the CTA sets kErrTimeout and the caller
-// abandons the launch (ep_handle_check then resets the barrier).
+// bar[0] counts arrivals, bar[1] is the generation.  Thread 0 of each CTA
+// reads the generation, then arrives with an acq_rel add (releasing the
+// CTA's writes, which __syncthreads made visible to it); the last arrival
+// resets the count and releases the generation bump; the others poll the
+// generation with acquire loads.  The state is left ready for the next
+// barrier and the next launch.  The poll is bounded: past kSpinLimit polls
+// the CTA sets kErrTimeout and the caller abandons the launch
+// (ep_handle_check then resets the barrier).
 constexpr uint32_t kSpinLimit = 1u << 20;  // polls of ~64 ns sleep + one L2 read
+
+__device__ __forceinline__ int32_t ld_acquire(const int32_t* p)
+{
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ int32_t atom_add_acq_rel(int32_t* p, int32_t v)
+{
+    int32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
 
 __device__ bool grid_barrier(int32_t* bar, int nblocks, int32_t* err)
 {
     __shared__ int ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        volatile int32_t* vgen = bar + 1;
-        const int32_t gen = *vgen;
-        __threadfence();
+        const int32_t gen = ld_acquire(bar + 1);
         int good = 1;
-        if (atomicAdd(bar, 1) == nblocks - 1) {
-            atomicExch(bar, 0);
-            __threadfence();
-            atomicAdd(bar + 1, 1);
+        if (atom_add_acq_rel(bar, 1) == nblocks - 1) {
+            asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(bar), "r"(0) : "memory");
+            asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(bar + 1), "r"(1)
+                         : "memory");
         } else {
             uint32_t polls = 0;
-            while (*vgen == gen) {
+            while (ld_acquire(bar + 1) == gen) {
                 if (++polls > kSpinLimit) {
                     good = 0;
                     break;
@@ -521,7 +557,6 @@ __device__ bool grid_barrier(int32_t* bar, int nblocks, int32_t* err)
                 __nanosleep(64);
             }
         }
-        __threadfence();
         if (!good)
             atomicOr(err, kErrTimeout);
         ok = good;
@@ -530,21 +565,21 @@ __device__ bool grid_barrier(int32_t* bar, int nblocks, int32_t* err)
     return ok != 0;
 }
 
-// One warp scans column col of an [nchunks][ncol] count matrix: exclusive
-// prefix over chunks written in place (if write_prefix); the column total is
-// returned to every lane.  Each batch covers 32 x kBatch consecutive chunks,
-// lane l owning chunks l*kBatch .. l*kBatch + kBatch - 1 of it, so a chunk's
+// One warp scans column col of an [nrows][ncol] count matrix: exclusive
+// prefix over rows written in place (if write_prefix); the column total is
+// returned to every lane.  Each batch covers 32 x kBatch consecutive rows,
+// lane l owning rows l*kBatch .. l*kBatch + kBatch - 1 of it, so a row's
 // prefix = earlier batches' total + lower lanes' sums + its lane's earlier
-// chunks.  All loads of a batch are issued before any is used.
-__device__ int32_t column_scan(int32_t* M, int64_t nchunks, int ncol, int col, bool write_prefix)
+// rows.  All loads of a batch are issued before any is used.
+__device__ int32_t column_scan(int32_t* M, int64_t nrows, int ncol, int col, bool write_prefix)
 {
     const int lane = threadIdx.x & 31;
     int32_t base = 0;
-    for (int64_t b0 = 0; b0 < nchunks; b0 += 32 * kBatch) {
+    for (int64_t b0 = 0; b0 < nrows; b0 += 32 * kBatch) {
         const int64_t r0 = b0 + (int64_t)lane * kBatch;
         int32_t v[kBatch];
 #pragma unroll
-        for (int m = 0; m < kBatch; ++m) v[m] = (r0 + m < nchunks) ? M[(r0 + m) * ncol + col] : 0;
+        for (int m = 0; m < kBatch; ++m) v[m] = (r0 + m < nrows) ? M[(r0 + m) * ncol + col] : 0;
         int32_t sum = 0;
 #pragma unroll
         for (int m = 0; m < kBatch; ++m) sum += v[m];
@@ -558,7 +593,7 @@ __device__ int32_t column_scan(int32_t* M, int64_t nchunks, int ncol, int col, b
             int32_t run = base + incl - sum;
 #pragma unroll
             for (int m = 0; m < kBatch; ++m)
-                if (r0 + m < nchunks) {
+                if (r0 + m < nrows) {
                     M[(r0 + m) * ncol + col] = run;
                     run += v[m];
                 }
@@ -568,35 +603,49 @@ __device__ int32_t column_scan(int32_t* M, int64_t nchunks, int ncol, int col, b
     return base;
 }
 
-// Large batches in one cooperative launch of G CTAs x W warps (all
-// co-resident).  Shared memory: off[E+1], wsum[32], then per warp
-// E + R + 32 k words (phase 1: hist, rank_hist, entry ranks; phase 3: run,
-// entries).  Chunks are taken grid-stride by warp, so G may be smaller than
-// the chunk count.
-__global__ void layout_fused_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                    int R, int epr, uint64_t rank_magic, int block_m,
-                                    int64_t nchunks,
-                                    int32_t* __restrict__ chunk_counts,
-                                    int32_t* __restrict__ chunk_rank, int32_t* __restrict__ cnt_g,
-                                    int32_t* __restrict__ expert_off_g,
-                                    int32_t* __restrict__ rank_off_g,
-                                    int32_t* __restrict__ tokens_per_rank_g,
-                                    int32_t* __restrict__ rows_per_rank_g,
-                                    int32_t* __restrict__ total_rows_g,
-                                    uint8_t* __restrict__ is_token_in_rank,
-                                    int32_t* __restrict__ dst_row, int32_t* __restrict__ recv_src,
-                                    int32_t* err)
+// Large batches in one cooperative launch.  A tile is kTileWarps warps x
+// kWarpTokens tokens; the grid (all co-resident) strides over tiles.
+//   phase 1  per tile: CTA-wide shared histogram of the tile's experts,
+//            is_token_in_rank bytes, tile rank counts -> tile_counts /
+//            tile_rank rows in global memory;
+//   phase 2  one warp per column: exclusive prefix of tile_counts over tiles
+//            (in place) and the expert totals; the rank totals;
+//   phase 3  every CTA scans the padded expert sizes into expert_off; per
+//            tile, the warps rebuild their own histograms in shared memory,
+//            a per-expert scan over the warps gives each warp its first free
+//            row per expert, and each warp replays its entries in order.
+// Shared memory (words): phase 1 hist[E] rhist[R] erank[W][kWarpTokens k];
+// phase 3 off[E+1] wsum[32] cnt[E] tpre[E] run[W][E] ents[W][kWarpTokens k].
+constexpr int kTileWarps = 8;
+constexpr int kWarpTokens = 8;
+constexpr int kTileTokens = kTileWarps * kWarpTokens;
+
+__host__ __device__ inline size_t tile_smem_words(int k, int E, int R)
+{
+    const size_t ent = (size_t)kTileWarps * kWarpTokens * k;
+    const size_t p1 = (size_t)E + R + ent;
+    const size_t p3 = (size_t)E + 1 + 32 + E + E + (size_t)kTileWarps * E + ent;
+    return p1 > p3 ? p1 : p3;
+}
+
+__global__ void __launch_bounds__(kTileWarps * 32)
+layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
+                   uint64_t rank_magic, int block_m, int64_t ntiles,
+                   int32_t* __restrict__ tile_counts, int32_t* __restrict__ tile_rank,
+                   int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
+                   int32_t* __restrict__ rank_off_g, int32_t* __restrict__ tokens_per_rank_g,
+                   int32_t* __restrict__ rows_per_rank_g, int32_t* __restrict__ total_rows_g,
+                   uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
+                   int32_t* __restrict__ recv_src, int32_t* err)
 {
     extern __shared__ int32_t smem[];
     pdl_wait();
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5, nthr = blockDim.x;
-    const int64_t gwarp = (int64_t)blockIdx.x * nwarps + warp;
-    const int64_t nwarps_all = (int64_t)gridDim.x * nwarps;
-    int32_t* off = smem;
-    int32_t* wsum = off + E + 1;
-    int32_t* mine = wsum + 32 + (size_t)warp * (E + R + kChunkTokens * k);
+    const int nthr = blockDim.x;
+    const int64_t gwarp = (int64_t)blockIdx.x * kTileWarps + warp;
+    const int64_t nwarps_all = (int64_t)gridDim.x * kTileWarps;
+    const int went = kWarpTokens * k;
     int32_t* bar = err + 1;
 
     // A barrier that timed out earlier leaves its words inconsistent until
@@ -608,40 +657,42 @@ __global__ void layout_fused_kernel(const int64_t* __restrict__ topk_idx, int T,
     if (stale)
         return;
 
-    // phase 1: per-chunk histograms, is_token_in_rank, per-chunk rank counts
+    // ---- phase 1
     {
-        int32_t* hist = mine;
+        int32_t* hist = smem;
         int32_t* rhist = hist + E;
-        int32_t* erank = rhist + R;
-        for (int64_t c = gwarp; c < nchunks; c += nwarps_all) {
-            const int64_t t0 = c * kChunkTokens;
-            const int ntok = (int)min((int64_t)kChunkTokens, (int64_t)T - t0);
-            const int nent = ntok * k;
-            for (int e = lane; e < E; e += 32) hist[e] = 0;
-            for (int r = lane; r < R; r += 32) rhist[r] = 0;
-            __syncwarp();
-            const int bad = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, nullptr, erank, hist);
-            if (bad && lane == 0)
-                atomicOr(err, kErrBadIndex);
-            __syncwarp();
-            chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
-            __syncwarp();
-            for (int e = lane; e < E; e += 32) chunk_counts[c * E + e] = hist[e];
-            for (int r = lane; r < R; r += 32) chunk_rank[c * R + r] = rhist[r];
-            __syncwarp();
+        int32_t* erank = rhist + R + (size_t)warp * went;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            for (int e = threadIdx.x; e < E; e += nthr) hist[e] = 0;
+            for (int r = threadIdx.x; r < R; r += nthr) rhist[r] = 0;
+            __syncthreads();
+            const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
+            const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
+            if (ntok > 0) {
+                const int bad = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, nullptr,
+                                           erank, hist);
+                if (bad && lane == 0)
+                    atomicOr(err, kErrBadIndex);
+                __syncwarp();
+                chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < E; e += nthr) tile_counts[tile * E + e] = hist[e];
+            for (int r = threadIdx.x; r < R; r += nthr) tile_rank[tile * R + r] = rhist[r];
+            __syncthreads();
         }
     }
     if (!grid_barrier(bar, gridDim.x, err))
         return;
 
-    // phase 2: one warp per column -- experts (prefix + total), then ranks (total)
+    // ---- phase 2
     for (int64_t col = gwarp; col < E + R; col += nwarps_all) {
         if (col < E) {
-            const int32_t tot = column_scan(chunk_counts, nchunks, E, (int)col, true);
+            const int32_t tot = column_scan(tile_counts, ntiles, E, (int)col, true);
             if (lane == 0)
                 cnt_g[col] = tot;
         } else {
-            const int32_t tot = column_scan(chunk_rank, nchunks, R, (int)(col - E), false);
+            const int32_t tot = column_scan(tile_rank, ntiles, R, (int)(col - E), false);
             if (lane == 0)
                 tokens_per_rank_g[col - E] = tot;
         }
@@ -649,59 +700,72 @@ __global__ void layout_fused_kernel(const int64_t* __restrict__ topk_idx, int T,
     if (!grid_barrier(bar, gridDim.x, err))
         return;
 
-    // phase 3: offsets (every CTA), bookkeeping (CTA 0), pad rows, assignment.
-    // A chunk's prefix row (into run) and entries do not depend on the
-    // offsets: the first chunk's loads are issued before the offset scan.
-    int32_t* runc = mine;
-    int32_t* ents = runc + E;
-    auto fetch = [&](int64_t c) {
-        const int64_t t0 = c * kChunkTokens;
-        const int nent = (int)min((int64_t)kChunkTokens, (int64_t)T - t0) * k;
-        for (int base = 0; base < E; base += 32 * kBatch) {
-            int32_t v[kBatch];
-#pragma unroll
-            for (int m = 0; m < kBatch; ++m) {
-                const int e = base + m * 32 + lane;
-                v[m] = e < E ? chunk_counts[c * E + e] : 0;
-            }
-#pragma unroll
-            for (int m = 0; m < kBatch; ++m) {
-                const int e = base + m * 32 + lane;
-                if (e < E)
-                    runc[e] = v[m];
-            }
+    // ---- phase 3
+    int32_t* off = smem;
+    int32_t* wsum = off + E + 1;
+    int32_t* cnt = wsum + 32;
+    int32_t* tpre = cnt + E;
+    int32_t* run_all = tpre + E;
+    int32_t* ents_all = run_all + (size_t)kTileWarps * E;
+    int32_t* run = run_all + (size_t)warp * E;
+    int32_t* ents = ents_all + (size_t)warp * went;
+
+    // a tile's loads: this warp's entries (and its histogram into run), the
+    // tile's prefix row into tpre
+    auto fetch = [&](int64_t tile) {
+        for (int e = lane; e < E; e += 32) run[e] = 0;
+        __syncwarp();
+        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
+        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
+        if (ntok > 0) {
+            const int ignored = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, ents,
+                                           nullptr, run);
+            (void)ignored;
         }
-        const int ignored = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, ents, nullptr,
-                                       nullptr);
-        (void)ignored;
+        for (int e = threadIdx.x; e < E; e += nthr) tpre[e] = tile_counts[tile * E + e];
     };
-    if (gwarp < nchunks)
-        fetch(gwarp);
-    scan_padded(cnt_g, E, block_m, off, wsum);
+
+    int64_t tile = blockIdx.x;
+    if (tile < ntiles)
+        fetch(tile);
+    for (int e = threadIdx.x; e < E; e += nthr) cnt[e] = cnt_g[e];
+    __syncthreads();
+    scan_padded(cnt, E, block_m, off, wsum);
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
         for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
         for (int r = threadIdx.x; r < R; r += nthr) {
             int32_t s = 0;
-            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt_g[e];
+            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
             rows_per_rank_g[r] = s;
         }
         if (threadIdx.x == 0)
             *total_rows_g = off[E];
     }
+    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
     for (int64_t e = gwarp; e < E; e += nwarps_all)
-        for (int32_t r = off[e] + cnt_g[e] + lane; r < off[e + 1]; r += 32)
-            recv_src[r] = -1;
+        fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
-    for (int64_t c = gwarp; c < nchunks; c += nwarps_all) {
-        if (c != gwarp)
-            fetch(c);
-        const int64_t t0 = c * kChunkTokens;
-        const int nent = (int)min((int64_t)kChunkTokens, (int64_t)T - t0) * k;
-        for (int e = lane; e < E; e += 32) runc[e] += off[e];
-        __syncwarp();
-        chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
-        __syncwarp();
+    for (; tile < ntiles; tile += gridDim.x) {
+        if (tile != blockIdx.x) {
+            __syncthreads();  // the previous tile is done with run / ents / tpre
+            fetch(tile);
+            __syncthreads();
+        }
+        // run[w][e] = off[e] + tile prefix + the counts of earlier warps
+        for (int e = threadIdx.x; e < E; e += nthr) {
+            int32_t acc = off[e] + tpre[e];
+            for (int w = 0; w < kTileWarps; ++w) {
+                const int32_t h = run_all[(size_t)w * E + e];
+                run_all[(size_t)w * E + e] = acc;
+                acc += h;
+            }
+        }
+        __syncthreads();
+        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
+        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
+        if (ntok > 0)
+            chunk_assign(ents, ntok * k, k, t0, run, dst_row, recv_src);
     }
 }
 
@@ -729,32 +793,30 @@ size_t small_layout_smem(int k, int E, int R, int64_t nchunks)
     return sizeof(int32_t) * (size_t)(nc * E + E + E + 1 + 32 + R + nc * 2 * kChunkTokens * k);
 }
 
-// The fused layout: W warps per CTA from the shared-memory budget, G CTAs =
-// min(CTAs the chunks need, CTAs that fit on the GPU at once).
-cudaError_t launch_fused(const Handle& h, const int64_t* topk_idx, int T, int64_t nchunks,
-                         cudaStream_t s)
+// The single-launch layout: kTileWarps warps per CTA, G CTAs = min(tiles,
+// CTAs that fit on the GPU at once), cooperative so that all are resident.
+cudaError_t launch_fused(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
-    const size_t fixed = sizeof(int32_t) * (size_t)(E + 1 + 32);
-    const size_t per_warp = sizeof(int32_t) * (size_t)(E + R + kChunkTokens * k);
-    const int w = warps_for(per_warp, fixed);
-    const size_t smem = fixed + per_warp * w;
+    const size_t smem = sizeof(int32_t) * tile_smem_words(k, E, R);
+    if (smem > kSmemBudget)
+        return cudaErrorCooperativeLaunchTooLarge;  // the caller uses three kernels
+    const int64_t ntiles = ((int64_t)T + kTileTokens - 1) / kTileTokens;
     cudaError_t rc;
-    if ((rc = set_smem((const void*)layout_fused_kernel, smem)) != cudaSuccess)
+    if ((rc = set_smem((const void*)layout_tile_kernel, smem)) != cudaSuccess)
         return rc;
     int dev = 0, sms = 0, per_sm = 0;
     if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
         (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, 32 * w,
-                                                            smem)) != cudaSuccess)
+        (rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_tile_kernel,
+                                                            32 * kTileWarps, smem)) != cudaSuccess)
         return rc;
     if (per_sm < 1)
         return cudaErrorCooperativeLaunchTooLarge;
-    const int64_t want = (nchunks + w - 1) / w;
-    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * per_sm);
+    const unsigned grid = (unsigned)std::min<int64_t>(ntiles, (int64_t)sms * per_sm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(32 * w);
+    cfg.blockDim = dim3(32 * kTileWarps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -762,11 +824,11 @@ cudaError_t launch_fused(const Handle& h, const int64_t* topk_idx, int T, int64_
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layout_fused_kernel, topk_idx, T, k, E, R, epr,
-                              rank_magic_for(epr), h.block_m,
-                              nchunks, h.chunk_counts, h.chunk_rank, h.cnt, h.expert_off,
-                              h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
-                              h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
+    return cudaLaunchKernelEx(&cfg, layout_tile_kernel, topk_idx, T, k, E, R, epr,
+                              rank_magic_for(epr), h.block_m, ntiles, h.chunk_counts,
+                              h.chunk_rank, h.cnt, h.expert_off, h.rank_off, h.tokens_per_rank,
+                              h.rows_per_rank, h.total_rows, h.is_token_in_rank, h.dst_row,
+                              h.recv_src, h.err);
 }
 
 cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s,
@@ -782,7 +844,7 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
         if (smem <= kSmemBudget) {
             if ((rc = set_smem((const void*)layout_small_kernel, smem)) != cudaSuccess)
                 return rc;
-            const unsigned nw = (unsigned)std::max<int64_t>(8, nchunks);
+            const unsigned nw = (unsigned)std::max<int64_t>(16, nchunks);
             return launch_pdl(layout_small_kernel, 1, 32 * nw, smem, s, topk_idx, T, k, E, R, epr,
                               rank_magic_for(epr), h.block_m, nchunks, h.cnt, h.expert_off, h.rank_off,
                               h.tokens_per_rank, h.rows_per_rank, h.total_rows,
@@ -791,7 +853,7 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
     }
 
     if (allow_fused && nchunks > 0) {
-        rc = launch_fused(h, topk_idx, T, nchunks, s);
+        rc = launch_fused(h, topk_idx, T, s);
         if (rc != cudaErrorCooperativeLaunchTooLarge && rc != cudaErrorNotSupported)
             return rc;
         (void)cudaGetLastError();  // clear the refused launch; use three kernels

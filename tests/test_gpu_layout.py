@@ -52,6 +52,8 @@ FUZZ = [
     (1024, 256, 16, 8, 128, 0.0, True),    # 32 chunks: the one-CTA path's limit
     (1025, 256, 16, 8, 128, 0.0, True),    # 33 chunks: the three-kernel path
     (1000, 2048, 8, 8, 128, 0.0, True),    # 32 chunks but counts too big for one CTA
+    (5000, 8192, 64, 4, 128, 0.0, True),   # tile counts too big for shared memory: 3 kernels
+    (3000, 256, 8, 8, 3, 0.1, True),       # block_m = 3: pad ranges not 4-aligned
 ]
 
 
