@@ -26,8 +26,8 @@
 // phases in one cooperative launch over 64-token tiles, its CTAs separated by
 // two grid barriers; the three kernels remain for shapes whose tile counts do
 // not fit in shared memory and for the static-scratch entry point.
-// Small batches (at most 32 chunks) run the same three phases inside one CTA
-// (layout_small_kernel), with the chunk counts in shared memory.
+// Small batches (T k <= 4096, E <= 1024) run in one CTA of 1024 threads with
+// one entry per thread (layout_small_kernel).
 //
 // The work is latency-bound (at 8K tokens the layout reads 0.5 MB), so each
 // kernel issues all of its global loads before it uses any of them, and every
@@ -422,102 +422,169 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
     chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
 }
 
-// Small batches: the three phases in one CTA; warp w < nchunks owns chunk w,
-// and at least 16 warps share the scans and the pad fill.
-// Shared memory: hist[nc][E] (then per-chunk prefixes, then run), cnt[E],
-// off[E+1], wsum[32], rank_hist[R], per chunk ents[32 k] + erank[32 k],
-// with nc = max(1, nchunks).
-__global__ void layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E,
-                                    int R, int epr, uint64_t rank_magic, int block_m,
-                                    int64_t nchunks,
-                                    int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
-                                    int32_t* __restrict__ rank_off_g,
-                                    int32_t* __restrict__ tokens_per_rank_g,
-                                    int32_t* __restrict__ rows_per_rank_g,
-                                    int32_t* __restrict__ total_rows_g,
-                                    uint8_t* __restrict__ is_token_in_rank,
-                                    int32_t* __restrict__ dst_row, int32_t* __restrict__ recv_src,
-                                    int32_t* err)
+// Small batches (T k <= kSmallEntries, E <= kSmallMaxE): one CTA of 1024
+// threads, one entry per thread per round of 1024 entries (at most
+// kSmallRounds rounds, the entries kept in registers between passes).
+//   pass A  shared-memory histogram, entry ranks, is_token_in_rank bytes (rows
+//           zeroed first; an entry sets its byte), tokens per rank (an entry
+//           counts if no earlier slot of its token has the same rank);
+//   offsets block scan of the padded counts;
+//   pass B  per round: __match_any_sync ranks inside each warp, per-warp
+//           counts in shared memory, a scan over the 32 warps per expert on
+//           top of the running per-expert base, then the positions.
+// Shared memory (words): cnt[E], run[E], wcnt[32][E], off[E+1], wsum[32],
+// rank_hist[R], erank[kSmallEntries].
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallRounds = 4;
+constexpr int kSmallEntries = kSmallThreads * kSmallRounds;
+constexpr int kSmallMaxE = 1024;
+constexpr int64_t kSmallMaxRankBytes = 65536;  // T x R bytes of is_token_in_rank
+
+__host__ __device__ inline size_t small_smem_words(int E, int R)
+{
+    return (size_t)E + E + 32 * (size_t)E + E + 1 + 32 + R + kSmallEntries;
+}
+
+__global__ void __launch_bounds__(kSmallThreads)
+layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
+                    uint64_t rank_magic, int block_m, int32_t* __restrict__ cnt_g,
+                    int32_t* __restrict__ expert_off_g, int32_t* __restrict__ rank_off_g,
+                    int32_t* __restrict__ tokens_per_rank_g,
+                    int32_t* __restrict__ rows_per_rank_g, int32_t* __restrict__ total_rows_g,
+                    uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
+                    int32_t* __restrict__ recv_src, int32_t* err)
 {
     extern __shared__ int32_t smem[];
     pdl_wait();
     pdl_trigger();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5, nthr = blockDim.x;
-    const int nc = (int)max((int64_t)1, nchunks);
-    int32_t* hist_all = smem;                           // [nc][E]
-    int32_t* cnt = hist_all + (size_t)nc * E;           // [E]
-    int32_t* off = cnt + E;                             // [E+1]
-    int32_t* wsum = off + E + 1;                        // [32]
-    int32_t* rhist = wsum + 32;                         // [R]
-    const bool has_chunk = warp < nchunks;
-    int32_t* ents = rhist + R + (size_t)(has_chunk ? warp : 0) * (2 * kChunkTokens * k);
-    int32_t* erank = ents + kChunkTokens * k;
-    int32_t* hist = hist_all + (size_t)(has_chunk ? warp : 0) * E;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int nent = T * k;
+    const int rounds = (nent + kSmallThreads - 1) / kSmallThreads;
+    int32_t* cnt = smem;
+    int32_t* run = cnt + E;
+    int32_t* wcnt = run + E;                     // [32][E]
+    int32_t* off = wcnt + 32 * (size_t)E;
+    int32_t* wsum = off + E + 1;
+    int32_t* rhist = wsum + 32;
+    int32_t* erank = rhist + R;
 
-    for (int i = threadIdx.x; i < nc * E; i += nthr) hist_all[i] = 0;
-    for (int r = threadIdx.x; r < R; r += nthr) rhist[r] = 0;
-    __syncthreads();
-
-    const int64_t t0 = (int64_t)warp * kChunkTokens;
-    const int ntok = has_chunk ? (int)min((int64_t)kChunkTokens, (int64_t)T - t0) : 0;
-    const int nent = ntok * k;
-    if (has_chunk) {
-        const int bad = load_chunk(topk_idx + t0 * k, nent, E, rank_magic, ents, erank, hist);
-        if (bad && lane == 0)
-            atomicOr(err, kErrBadIndex);
-        __syncwarp();
-        chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
-    }
-    __syncthreads();
-
-    // per-expert prefix over chunks, in place; totals into cnt
-    for (int e = threadIdx.x; e < E; e += nthr) {
-        int32_t run = 0;
-        for (int w = 0; w < nc; ++w) {
-            const int32_t h = hist_all[(size_t)w * E + e];
-            hist_all[(size_t)w * E + e] = run;
-            run += h;
+    for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
+    for (int r = tid; r < R; r += kSmallThreads) rhist[r] = 0;
+    {
+        const int64_t bytes = (int64_t)T * R;
+        uint8_t* itr = is_token_in_rank;
+        if (((uintptr_t)itr & 15u) == 0) {
+            for (int64_t i = (int64_t)tid * 16; i + 16 <= bytes; i += 16 * kSmallThreads)
+                *reinterpret_cast<int4*>(itr + i) = make_int4(0, 0, 0, 0);
+            for (int64_t i = (bytes & ~int64_t(15)) + tid; i < bytes; i += kSmallThreads) itr[i] = 0;
+        } else {
+            for (int64_t i = tid; i < bytes; i += kSmallThreads) itr[i] = 0;
         }
-        cnt[e] = run;
     }
     __syncthreads();
-    scan_padded(cnt, E, block_m, off, wsum);
 
-    for (int e = threadIdx.x; e < E; e += nthr) cnt_g[e] = cnt[e];
-    for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
-    for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
-    for (int r = threadIdx.x; r < R; r += nthr) {
+    // pass A
+    int e_r[kSmallRounds];
+    int bad = 0;
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        const int f = q * kSmallThreads + tid;
+        e_r[q] = (q < rounds && f < nent) ? to_expert(topk_idx[f], E, bad) : -2;
+    }
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        const int f = q * kSmallThreads + tid;
+        const int e = e_r[q];
+        if (e >= 0) {
+            const int rk = (int)(((uint64_t)e * rank_magic) >> 32);
+            atomicAdd(&cnt[e], 1);
+            erank[f] = rk;
+            is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
+        } else if (e == -1) {
+            erank[f] = -1;
+        }
+    }
+    if (__syncthreads_or(bad) && tid == 0)
+        atomicOr(err, kErrBadIndex);
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        const int f = q * kSmallThreads + tid;
+        if (e_r[q] >= 0) {
+            const int rk = erank[f];
+            const int t = f / k, j = f - t * k;
+            bool first = true;
+            for (int jj = 0; jj < j; ++jj) first &= (erank[t * k + jj] != rk);
+            if (first)
+                atomicAdd(&rhist[rk], 1);
+        }
+    }
+    __syncthreads();
+
+    // offsets and bookkeeping
+    scan_padded(cnt, E, block_m, off, wsum);
+    for (int e = tid; e < E; e += kSmallThreads) {
+        cnt_g[e] = cnt[e];
+        run[e] = off[e];
+    }
+    for (int e = tid; e <= E; e += kSmallThreads) expert_off_g[e] = off[e];
+    for (int r = tid; r <= R; r += kSmallThreads) rank_off_g[r] = off[r * epr];
+    for (int r = tid; r < R; r += kSmallThreads) {
         int32_t s = 0;
         for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
         rows_per_rank_g[r] = s;
         tokens_per_rank_g[r] = rhist[r];
     }
-    if (threadIdx.x == 0)
+    if (tid == 0)
         *total_rows_g = off[E];
-    // pad rows: one warp per expert
     const bool vec = ((uintptr_t)recv_src & 15u) == 0;
-    for (int e = warp; e < E; e += nwarps) fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
+    for (int e = warp; e < E; e += kSmallThreads / 32) fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
-    if (!has_chunk)
-        return;
-    for (int e = lane; e < E; e += 32) hist[e] += off[e];
-    __syncwarp();
-    chunk_assign(ents, nent, k, t0, hist, dst_row, recv_src);
+    // pass B
+    const unsigned lt = lanemask_lt();
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        if (q < rounds) {
+            for (int i = tid; i < 32 * E; i += kSmallThreads) wcnt[i] = 0;
+            __syncthreads();
+            const int e = e_r[q];
+            const unsigned peers = __match_any_sync(kFull, e);
+            if (e >= 0 && (peers & lt) == 0)
+                wcnt[warp * E + e] = __popc(peers);
+            __syncthreads();
+            for (int x = tid; x < E; x += kSmallThreads) {
+                int32_t acc = run[x];
+                for (int w = 0; w < 32; ++w) {
+                    const int32_t c = wcnt[w * E + x];
+                    wcnt[w * E + x] = acc;
+                    acc += c;
+                }
+                run[x] = acc;
+            }
+            __syncthreads();
+            const int f = q * kSmallThreads + tid;
+            if (f < nent) {
+                const int pos = e >= 0 ? wcnt[warp * E + e] + __popc(peers & lt) : -1;
+                dst_row[f] = pos;
+                if (pos >= 0)
+                    recv_src[pos] = f / k;
+            }
+        }
+    }
 }
-
 
 // ------------------------------------------------------------------ fused
 // Grid barrier over the CTAs of a cooperative launch (all co-resident).
-// bar[0] counts arrivals, bar[1] is the generation.  Thread 0 of each CTA
-// reads the generation, then arrives with an acq_rel add (releasing the
-// CTA's writes, which __syncthreads made visible to it); the last arrival
-// resets the count and releases the generation bump; the others poll the
-// generation with acquire loads.  The state is left ready for the next
-// barrier and the next launch.  The poll is bounded: past kSpinLimit polls
-// the CTA sets kErrTimeout and the caller abandons the launch
-// (ep_handle_check then resets the barrier).
-constexpr uint32_t kSpinLimit = 1u << 20;  // polls of ~64 ns sleep + one L2 read
+// bar[0] is an arrival counter that only grows (32-bit wrap-around, compared
+// by signed difference); bar[1] is its value when the current launch began.
+// Each CTA reads the base at its start; barrier b of the launch waits until
+// the counter reaches base + b G; the last arrival of the last barrier
+// stores the next launch's base (every CTA read the old one before
+// arriving).  Waiters watch the counter itself: the last arrival's add is the
+// release, one L2 round trip earlier than a separate release flag.  Graph
+// replays need no host state, and G may differ between launches.  The poll
+// is bounded: past kSpinLimit polls the CTA sets kErrTimeout and the caller
+// abandons the launch (ep_handle_check then resets both words).
+constexpr uint32_t kSpinLimit = 1u << 22;  // polls of one L2 read each
 
 __device__ __forceinline__ int32_t ld_acquire(const int32_t* p)
 {
@@ -536,25 +603,29 @@ __device__ __forceinline__ int32_t atom_add_acq_rel(int32_t* p, int32_t v)
     return old;
 }
 
-__device__ bool grid_barrier(int32_t* bar, int nblocks, int32_t* err)
+__device__ __forceinline__ int32_t signed_gap(int32_t a, int32_t b)
+{
+    return (int32_t)((uint32_t)a - (uint32_t)b);
+}
+
+__device__ bool grid_barrier(int32_t* bar, int32_t target, bool last_of_launch, int32_t* err)
 {
     __shared__ int ok;
     __syncthreads();
     if (threadIdx.x == 0) {
-        const int32_t gen = ld_acquire(bar + 1);
         int good = 1;
-        if (atom_add_acq_rel(bar, 1) == nblocks - 1) {
-            asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(bar), "r"(0) : "memory");
-            asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(bar + 1), "r"(1)
-                         : "memory");
+        const int32_t old = atom_add_acq_rel(bar, 1);
+        if (signed_gap(old, target) == -1) {
+            if (last_of_launch)
+                asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(bar + 1), "r"(target)
+                             : "memory");
         } else {
             uint32_t polls = 0;
-            while (ld_acquire(bar + 1) == gen) {
+            while (signed_gap(ld_acquire(bar), target) < 0) {
                 if (++polls > kSpinLimit) {
                     good = 0;
                     break;
                 }
-                __nanosleep(64);
             }
         }
         if (!good)
@@ -605,17 +676,21 @@ __device__ int32_t column_scan(int32_t* M, int64_t nrows, int ncol, int col, boo
 
 // Large batches in one cooperative launch.  A tile is kTileWarps warps x
 // kWarpTokens tokens; the grid (all co-resident) strides over tiles.
-//   phase 1  per tile: CTA-wide shared histogram of the tile's experts,
-//            is_token_in_rank bytes, tile rank counts -> tile_counts /
-//            tile_rank rows in global memory;
+//   phase 1  per tile: each warp loads its tokens' entries into shared memory
+//            and counts them into its own histogram row; the tile's counts
+//            (sum of the rows), is_token_in_rank bytes and rank counts ->
+//            tile_counts / tile_rank rows in global memory;
 //   phase 2  one warp per column: exclusive prefix of tile_counts over tiles
 //            (in place) and the expert totals; the rank totals;
 //   phase 3  every CTA scans the padded expert sizes into expert_off; per
-//            tile, the warps rebuild their own histograms in shared memory,
-//            a per-expert scan over the warps gives each warp its first free
-//            row per expert, and each warp replays its entries in order.
-// Shared memory (words): phase 1 hist[E] rhist[R] erank[W][kWarpTokens k];
-// phase 3 off[E+1] wsum[32] cnt[E] tpre[E] run[W][E] ents[W][kWarpTokens k].
+//            tile, a per-expert scan over the warp rows (on top of the tile
+//            prefix) gives each warp its first free row per expert, and each
+//            warp replays its entries in order.
+// When every CTA owns one tile, the entries and warp rows stay in shared
+// memory from phase 1 to phase 3; otherwise phase 3 rebuilds them per tile.
+// Shared memory (words): ents[W][kWarpTokens k], run[W][E] (kept), then
+// phase 1: rank_hist[R], erank[W][kWarpTokens k]; phase 3: off[E+1],
+// wsum[32], cnt[E], tpre[E].
 constexpr int kTileWarps = 8;
 constexpr int kWarpTokens = 8;
 constexpr int kTileTokens = kTileWarps * kWarpTokens;
@@ -623,9 +698,10 @@ constexpr int kTileTokens = kTileWarps * kWarpTokens;
 __host__ __device__ inline size_t tile_smem_words(int k, int E, int R)
 {
     const size_t ent = (size_t)kTileWarps * kWarpTokens * k;
-    const size_t p1 = (size_t)E + R + ent;
-    const size_t p3 = (size_t)E + 1 + 32 + E + E + (size_t)kTileWarps * E + ent;
-    return p1 > p3 ? p1 : p3;
+    const size_t kept = ent + (size_t)kTileWarps * E;
+    const size_t p1 = (size_t)R + ent;
+    const size_t p3 = (size_t)E + 1 + 32 + E + E;
+    return kept + (p1 > p3 ? p1 : p3);
 }
 
 __global__ void __launch_bounds__(kTileWarps * 32)
@@ -646,43 +722,68 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
     const int64_t gwarp = (int64_t)blockIdx.x * kTileWarps + warp;
     const int64_t nwarps_all = (int64_t)gridDim.x * kTileWarps;
     const int went = kWarpTokens * k;
+    const bool resident = ntiles <= (int64_t)gridDim.x;  // one tile per CTA
     int32_t* bar = err + 1;
 
+    int32_t* ents_all = smem;
+    int32_t* run_all = ents_all + (size_t)kTileWarps * went;
+    int32_t* scratch = run_all + (size_t)kTileWarps * E;
+    int32_t* ents = ents_all + (size_t)warp * went;
+    int32_t* run = run_all + (size_t)warp * E;
+
     // A barrier that timed out earlier leaves its words inconsistent until
-    // ep_handle_check resets them: refuse to run (every CTA reads the same word).
+    // ep_handle_check resets them: refuse to run (every CTA reads the same
+    // word).  Every CTA reads the launch's barrier base here, before any
+    // CTA can finish the last barrier and store the next one.
     __shared__ int stale;
-    if (threadIdx.x == 0)
+    __shared__ int32_t bar_base;
+    if (threadIdx.x == 0) {
         stale = (*(volatile int32_t*)err & kErrTimeout) != 0;
+        bar_base = *(volatile int32_t*)(bar + 1);
+    }
     __syncthreads();
     if (stale)
         return;
+    const int32_t G = (int32_t)gridDim.x;
+
+    // a tile's entries into ents and each warp's histogram into its run row
+    auto load_tile = [&](int64_t tile, int32_t* erank) {
+        for (int e = lane; e < E; e += 32) run[e] = 0;
+        __syncwarp();
+        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
+        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
+        int bad = 0;
+        if (ntok > 0)
+            bad = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, ents, erank, run);
+        __syncwarp();
+        return bad;
+    };
 
     // ---- phase 1
     {
-        int32_t* hist = smem;
-        int32_t* rhist = hist + E;
+        int32_t* rhist = scratch;
         int32_t* erank = rhist + R + (size_t)warp * went;
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            for (int e = threadIdx.x; e < E; e += nthr) hist[e] = 0;
             for (int r = threadIdx.x; r < R; r += nthr) rhist[r] = 0;
             __syncthreads();
+            const int bad = load_tile(tile, erank);
+            if (bad && lane == 0)
+                atomicOr(err, kErrBadIndex);
             const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
             const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
-            if (ntok > 0) {
-                const int bad = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, nullptr,
-                                           erank, hist);
-                if (bad && lane == 0)
-                    atomicOr(err, kErrBadIndex);
-                __syncwarp();
+            if (ntok > 0)
                 chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
-            }
             __syncthreads();
-            for (int e = threadIdx.x; e < E; e += nthr) tile_counts[tile * E + e] = hist[e];
+            for (int e = threadIdx.x; e < E; e += nthr) {
+                int32_t h = 0;
+                for (int w = 0; w < kTileWarps; ++w) h += run_all[(size_t)w * E + e];
+                tile_counts[tile * E + e] = h;
+            }
             for (int r = threadIdx.x; r < R; r += nthr) tile_rank[tile * R + r] = rhist[r];
             __syncthreads();
         }
     }
-    if (!grid_barrier(bar, gridDim.x, err))
+    if (!grid_barrier(bar, bar_base + G, false, err))
         return;
 
     // ---- phase 2
@@ -697,38 +798,21 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
                 tokens_per_rank_g[col - E] = tot;
         }
     }
-    if (!grid_barrier(bar, gridDim.x, err))
+    if (!grid_barrier(bar, bar_base + 2 * G, true, err))
         return;
 
     // ---- phase 3
-    int32_t* off = smem;
+    int32_t* off = scratch;
     int32_t* wsum = off + E + 1;
     int32_t* cnt = wsum + 32;
     int32_t* tpre = cnt + E;
-    int32_t* run_all = tpre + E;
-    int32_t* ents_all = run_all + (size_t)kTileWarps * E;
-    int32_t* run = run_all + (size_t)warp * E;
-    int32_t* ents = ents_all + (size_t)warp * went;
-
-    // a tile's loads: this warp's entries (and its histogram into run), the
-    // tile's prefix row into tpre
-    auto fetch = [&](int64_t tile) {
-        for (int e = lane; e < E; e += 32) run[e] = 0;
-        __syncwarp();
-        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
-        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
-        if (ntok > 0) {
-            const int ignored = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, ents,
-                                           nullptr, run);
-            (void)ignored;
-        }
-        for (int e = threadIdx.x; e < E; e += nthr) tpre[e] = tile_counts[tile * E + e];
-    };
-
     int64_t tile = blockIdx.x;
-    if (tile < ntiles)
-        fetch(tile);
-    for (int e = threadIdx.x; e < E; e += nthr) cnt[e] = cnt_g[e];
+    for (int e = threadIdx.x; e < E; e += nthr) {
+        cnt[e] = cnt_g[e];
+        tpre[e] = tile_counts[tile * E + e];  // tile < ntiles: G <= ntiles
+    }
+    if (!resident)
+        (void)load_tile(tile, nullptr);
     __syncthreads();
     scan_padded(cnt, E, block_m, off, wsum);
     if (blockIdx.x == 0) {
@@ -749,7 +833,8 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
     for (; tile < ntiles; tile += gridDim.x) {
         if (tile != blockIdx.x) {
             __syncthreads();  // the previous tile is done with run / ents / tpre
-            fetch(tile);
+            (void)load_tile(tile, nullptr);
+            for (int e = threadIdx.x; e < E; e += nthr) tpre[e] = tile_counts[tile * E + e];
             __syncthreads();
         }
         // run[w][e] = off[e] + tile prefix + the counts of earlier warps
@@ -786,12 +871,6 @@ cudaError_t set_smem(const void* fn, size_t bytes)
 }
 
 }  // namespace
-
-size_t small_layout_smem(int k, int E, int R, int64_t nchunks)
-{
-    const int64_t nc = std::max<int64_t>(1, nchunks);
-    return sizeof(int32_t) * (size_t)(nc * E + E + E + 1 + 32 + R + nc * 2 * kChunkTokens * k);
-}
 
 // The single-launch layout: kTileWarps warps per CTA, G CTAs = min(tiles,
 // CTAs that fit on the GPU at once), cooperative so that all are resident.
@@ -838,18 +917,16 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
     const int64_t nchunks = ((int64_t)T + kChunkTokens - 1) / kChunkTokens;
     cudaError_t rc;
 
-    // one CTA when the batch is small and its counts fit in shared memory
-    if (nchunks <= 32) {
-        const size_t smem = small_layout_smem(k, E, R, nchunks);
-        if (smem <= kSmemBudget) {
-            if ((rc = set_smem((const void*)layout_small_kernel, smem)) != cudaSuccess)
-                return rc;
-            const unsigned nw = (unsigned)std::max<int64_t>(16, nchunks);
-            return launch_pdl(layout_small_kernel, 1, 32 * nw, smem, s, topk_idx, T, k, E, R, epr,
-                              rank_magic_for(epr), h.block_m, nchunks, h.cnt, h.expert_off, h.rank_off,
-                              h.tokens_per_rank, h.rows_per_rank, h.total_rows,
-                              h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
-        }
+    // one CTA, one entry per thread, when the batch is small
+    if ((int64_t)T * k <= kSmallEntries && E <= kSmallMaxE &&
+        (int64_t)T * R <= kSmallMaxRankBytes) {
+        const size_t smem = sizeof(int32_t) * small_smem_words(E, R);
+        if ((rc = set_smem((const void*)layout_small_kernel, smem)) != cudaSuccess)
+            return rc;
+        return launch_pdl(layout_small_kernel, 1, kSmallThreads, smem, s, topk_idx, T, k, E, R,
+                          epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off, h.rank_off,
+                          h.tokens_per_rank, h.rows_per_rank, h.total_rows, h.is_token_in_rank,
+                          h.dst_row, h.recv_src, h.err);
     }
 
     if (allow_fused && nchunks > 0) {

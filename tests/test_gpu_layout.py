@@ -49,9 +49,11 @@ FUZZ = [
     (64, 8192, 8192, 4, 128, 0.0, True),   # maximum E, R = E
     (4096, 256, 256, 8, 128, 0.5, True),   # many unused slots
     (20000, 256, 8, 8, 128, 0.0, True),    # many chunks
-    (1024, 256, 16, 8, 128, 0.0, True),    # 32 chunks: the one-CTA path's limit
-    (1025, 256, 16, 8, 128, 0.0, True),    # 33 chunks: the three-kernel path
-    (1000, 2048, 8, 8, 128, 0.0, True),    # 32 chunks but counts too big for one CTA
+    (512, 256, 16, 8, 128, 0.1, True),     # 4096 entries: the one-CTA path's limit
+    (513, 256, 16, 8, 128, 0.0, True),     # 4104 entries: the tiled path
+    (400, 1024, 64, 8, 128, 0.0, True),    # one-CTA path at its largest E
+    (300, 1024, 1024, 4, 128, 0.0, True),  # T x R too many bytes for one CTA: tiled
+    (1000, 2048, 8, 8, 128, 0.0, True),    # E above the one-CTA limit
     (5000, 8192, 64, 4, 128, 0.0, True),   # tile counts too big for shared memory: 3 kernels
     (3000, 256, 8, 8, 3, 0.1, True),       # block_m = 3: pad ranges not 4-aligned
 ]
