@@ -71,6 +71,10 @@ def _load():
             lib.oracle_expert_scale_fp8.restype = None
             lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, P]
             lib.oracle_combine.restype = i32
+            lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, P]
+            lib.oracle_dispatch_backward.restype = i32
+            lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
+            lib.oracle_combine_backward.restype = i32
             for name in ("oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
                          "oracle_f32_to_bf16_array"):
                 getattr(lib, name).argtypes = [P, P, i64]
@@ -247,6 +251,43 @@ def combine(y_bits: np.ndarray, topk_weights: np.ndarray, dst_row: np.ndarray) -
     if rc != OK:
         raise OracleError(rc, "oracle_combine")
     return out
+
+
+# ---------------------------------------------------------------- backward
+
+def dispatch_backward(grad_recv_bits: np.ndarray, dst_row: np.ndarray) -> np.ndarray:
+    """grad_x[t] = bf16(sum over used slots of grad_recv[dst_row[t, j]]), fp32 in slot order."""
+    g = np.ascontiguousarray(grad_recv_bits, dtype=np.uint16)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    rows, H = g.shape
+    T, k = dst_row.shape
+    out = np.zeros((T, H), np.uint16)
+    if rows == 0:
+        g = np.zeros((1, H), np.uint16)
+    rc = _load().oracle_dispatch_backward(_p(g), rows, _p(dst_row), T, k, H, _p(out))
+    if rc != OK:
+        raise OracleError(rc, "oracle_dispatch_backward")
+    return out
+
+
+def combine_backward(grad_out_bits: np.ndarray, y_bits: np.ndarray, topk_weights: np.ndarray,
+                     dst_row: np.ndarray):
+    """(grad_y bits [rows, H] with pad rows zero, grad_w f32 [T, k])."""
+    g = np.ascontiguousarray(grad_out_bits, dtype=np.uint16)
+    y = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(topk_weights, dtype=np.float32)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    rows, H = y.shape
+    T, k = dst_row.shape
+    gy = np.zeros((max(rows, 1), H), np.uint16)
+    gw = np.zeros((T, k), np.float32)
+    if rows == 0:
+        y = np.zeros((1, H), np.uint16)
+    rc = _load().oracle_combine_backward(_p(g), _p(y), rows, _p(w), _p(dst_row), T, k, H,
+                                         _p(gy), _p(gw))
+    if rc != OK:
+        raise OracleError(rc, "oracle_combine_backward")
+    return gy[:rows], gw
 
 
 def pipeline(x_bits, topk_idx, topk_weights, E, R, fmt, c, block_m=128):
