@@ -344,6 +344,52 @@ def graph_latency_us(s, reps=200):
     return us
 
 
+def time_backward(dev, flush, seed, steps):
+    """Backward of the 8k step: ep_dispatch_backward (a k-row sum per token)
+    and ep_combine_backward (k scaled rows written, k dot products), each
+    timed with CUDA events, L2 flushed before each launch."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from workloads import make_workload
+
+    w = make_workload(MAIN_WORKLOAD, seed, H=16)  # routing only; rows are drawn below
+    H = 7168
+    h = ep.ep_handle_create(w.T, w.k, w.E, w.R, w.block_m, device=dev)
+    ep.ep_layout(h, torch.from_numpy(w.topk_idx).to(dev))
+    cap = ep.ep_recv_rows_upper_bound(w.T, w.k, w.E, w.block_m)
+    g = torch.randn((cap, H), device=dev).to(torch.bfloat16)
+    go = torch.randn((w.T, H), device=dev).to(torch.bfloat16)
+    y = torch.randn((cap, H), device=dev).to(torch.bfloat16)
+    wt = torch.from_numpy(w.topk_weights).to(dev)
+    gx = torch.empty((w.T, H), dtype=torch.bfloat16, device=dev)
+    gy = torch.empty_like(y)
+    res = {}
+    for name, fn, nbytes in (
+            ("dispatch_backward", lambda: ep.ep_dispatch_backward(h, g, gx),
+             w.T * w.k * 2 * H + w.T * 2 * H),
+            ("combine_backward", lambda: ep.ep_combine_backward(h, go, y, wt, gy),
+             w.T * 2 * H + 2 * w.T * w.k * 2 * H + w.T * w.k * 4)):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        res[name + "_us"] = round(ms * 1e3, 2)
+        res[name + "_GBps"] = round(nbytes / (ms / 1e3) / 1e9, 1)
+    ep.ep_handle_check(h)
+    res["workload"] = "8k routing, H=7168, bf16 gradients (random rows)"
+    return res
+
+
 # ----------------------------------------------------------------- CPU arm
 
 def cpu_oracle_step(w, tokens, y_full=None):
@@ -536,6 +582,11 @@ def main():
             secondary[name] = ent
             del s2
             torch.cuda.empty_cache()
+
+    if not args.no_secondary:
+        secondary["8k_backward"] = time_backward(dev, flush, args.seed + rank,
+                                                 max(3, min(args.steps, 50)))
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -27,7 +27,7 @@ import torch
 __all__ = [
     "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
     "ep_layout", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
-    "ep_dispatch_range", "ep_combine_range",
+    "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
@@ -96,6 +96,8 @@ def load_library():
             "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
             "ep_combine": ([P, P, I64, P, I, P, P], I),
             "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
+            "ep_dispatch_backward": ([P, P, I64, I, P, P], I),
+            "ep_combine_backward": ([P, P, P, I64, P, I, P, I64, P, P], I),
             "ep_combine_range": ([P, I, I, P, I64, P, I, P, P], I),
             "ep_handle_check": ([P, P], I),
             "ep_strerror": ([I], ctypes.c_char_p),
@@ -335,6 +337,45 @@ def ep_combine_range(h: EPHandle, t_begin: int, y: torch.Tensor, topk_weights_ro
         _check(load_library().ep_combine_range(
             h.handle, t_begin, n, _ptr(y), y.shape[0], _ptr(topk_weights_rows), H, _ptr(out_rows),
             _stream(h.device)), "ep_combine_range")
+
+
+def ep_dispatch_backward(h: EPHandle, grad_recv: torch.Tensor,
+                         grad_x: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """grad_x[t] = sum over the used slots of grad_recv[dst_row[t, j]] (bf16 [T, H])."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch_backward")
+    if grad_recv.dtype != torch.bfloat16 or grad_recv.dim() != 2 or not grad_recv.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_backward: grad_recv must be bf16 [rows, H]")
+    H = grad_recv.shape[1]
+    if grad_x is None:
+        grad_x = torch.empty((h.T, H), dtype=torch.bfloat16, device=grad_recv.device)
+    with _on(h):
+        _check(load_library().ep_dispatch_backward(h.handle, _ptr(grad_recv), grad_recv.shape[0],
+                                                   H, _ptr(grad_x), _stream(h.device)),
+               "ep_dispatch_backward")
+    return grad_x
+
+
+def ep_combine_backward(h: EPHandle, grad_out: torch.Tensor, y: torch.Tensor,
+                        topk_weights: torch.Tensor, grad_y: Optional[torch.Tensor] = None):
+    """(grad_y bf16 in the receive layout, grad_weights f32 [T, k]) for ep_combine."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_combine_backward")
+    for name, t in (("grad_out", grad_out), ("y", y)):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
+            raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: %s must be bf16 2-D" % name)
+    if (topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (h.T, h.k)
+            or not topk_weights.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: topk_weights must be f32 [T, k]")
+    H = y.shape[1]
+    if grad_y is None:
+        grad_y = torch.empty_like(y)
+    grad_w = torch.empty((h.T, h.k), dtype=torch.float32, device=y.device)
+    with _on(h):
+        _check(load_library().ep_combine_backward(
+            h.handle, _ptr(grad_out), _ptr(y), y.shape[0], _ptr(topk_weights), H, _ptr(grad_y),
+            grad_y.shape[0], _ptr(grad_w), _stream(h.device)), "ep_combine_backward")
+    return grad_y, grad_w
 
 
 def ep_handle_check(h: EPHandle, raise_on_error: bool = True) -> int:

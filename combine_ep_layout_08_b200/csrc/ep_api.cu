@@ -388,6 +388,44 @@ ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const voi
                         out_rows, stream, "ep_combine_range");
 }
 
+ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t grad_rows, int H,
+                                 void* grad_x, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 8 != 0 || grad_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (h->T > 0 && (!grad_x || (!grad_recv && grad_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(grad_recv, 16) || !ep::aligned(grad_x, 16))
+        return EP_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = ep::launch_combine(*h, grad_recv, grad_rows, nullptr, H, grad_x, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_backward");
+}
+
+ep_status_t ep_combine_backward(ep_handle_t hh, const void* grad_out, const void* y,
+                                int64_t y_rows, const float* topk_weights, int H, void* grad_y,
+                                int64_t grad_y_rows, float* grad_weights, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0 || grad_y_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (h->T > 0 && (!grad_out || !topk_weights || !grad_weights || (!y && y_rows > 0) ||
+                     (!grad_y && grad_y_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(grad_out, 16) || !ep::aligned(y, 16) || !ep::aligned(grad_y, 16) ||
+        !ep::aligned(topk_weights, 4) || !ep::aligned(grad_weights, 4))
+        return EP_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = ep::launch_combine_backward(*h, grad_out, y, y_rows, topk_weights, H, grad_y,
+                                                 grad_y_rows, grad_weights, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine_backward");
+}
+
 ep_status_t ep_handle_check(ep_handle_t hh, void* stream)
 {
     Handle* h = ep::as_handle(hh);

@@ -1,0 +1,143 @@
+// ep_backward.cu -- gradients of dispatch and combine on sm_100a.
+//
+// The pages name training as a use of expert-parallel dispatch/combine
+// ("DeepEP：让大模型「专家们」高效协作的通信高速公路", section 核心使用场景;
+// "DeepEP是什麼？…", high-throughput mode for training and prefill) without
+// defining gradients.  These are the gradients of the forward definitions:
+//
+//   dispatch backward: grad_x[t] = sum over used slots of grad_recv[dst_row[t][j]],
+//     fp32 in slot order j = 0..k-1, bf16 out -- the combine kernel with unit
+//     weights (ep_combine.cu);
+//   combine backward:  grad_y[dst_row[t][j]] = bf16(w[t][j] * grad_out[t])
+//                      grad_w[t][j] = sum_h grad_out[t][h] * y[dst_row[t][j]][h]
+//     (this file).
+//
+// combine_backward_kernel: one CTA per token.  Each thread takes 16-byte
+// vectors of the row (8 channels), reads grad_out once and the k rows of y,
+// writes the k scaled rows of grad_y and keeps k fp32 partial dot products
+// (fused multiply-adds, its channels in order).  The partials are reduced
+// with a fixed xor-shuffle tree inside each warp and then in warp order, so
+// the result is bitwise repeatable (its rounding differs from a sequential
+// sum by at most the fp32 summation bound).  Slots are taken 8 at a time.
+// HBM traffic per token: 2H + 2kH read, 2kH written (+ 4k bytes of grad_w).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kMaxThreads = 256;
+constexpr int kSlotBatch = 8;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return a | (b << 16);
+}
+
+__global__ void __launch_bounds__(kMaxThreads)
+combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restrict__ y,
+                        int64_t y_rows, const float* __restrict__ weights, int T, int k,
+                        int64_t vpr, const int32_t* __restrict__ dst_row,
+                        uint4* __restrict__ grad_y, int64_t grad_y_rows,
+                        float* __restrict__ grad_w, int32_t* err)
+{
+    __shared__ int32_t s_row[EP_MAX_TOPK];
+    __shared__ float s_w[EP_MAX_TOPK];
+    __shared__ float s_red[kMaxThreads / 32][kSlotBatch];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int64_t t = blockIdx.x;
+    if (t >= T)
+        return;
+    if ((int)threadIdx.x < k) {
+        int32_t d = dst_row[t * k + threadIdx.x];
+        if (d >= y_rows || d >= grad_y_rows) {
+            atomicOr(err, kErrCombineCap);
+            d = -1;
+        }
+        s_row[threadIdx.x] = d;
+        s_w[threadIdx.x] = weights[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    const uint4* g_row = grad_out + t * vpr;
+
+    for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
+        const int nj = min(kSlotBatch, k - j0);
+        float part[kSlotBatch];
+#pragma unroll
+        for (int jj = 0; jj < kSlotBatch; ++jj) part[jj] = 0.0f;
+        for (int64_t v = threadIdx.x; v < vpr; v += blockDim.x) {
+            const uint4 gv = g_row[v];
+            const float g[8] = {bf16_lo(gv.x), bf16_hi(gv.x), bf16_lo(gv.y), bf16_hi(gv.y),
+                                bf16_lo(gv.z), bf16_hi(gv.z), bf16_lo(gv.w), bf16_hi(gv.w)};
+            uint4 yv[kSlotBatch];
+#pragma unroll
+            for (int jj = 0; jj < kSlotBatch; ++jj) {
+                const int d = jj < nj ? s_row[j0 + jj] : -1;
+                if (d >= 0)
+                    yv[jj] = __ldcs(y + (int64_t)d * vpr + v);
+            }
+#pragma unroll
+            for (int jj = 0; jj < kSlotBatch; ++jj) {
+                const int d = jj < nj ? s_row[j0 + jj] : -1;
+                if (d < 0)
+                    continue;
+                const float f[8] = {bf16_lo(yv[jj].x), bf16_hi(yv[jj].x), bf16_lo(yv[jj].y),
+                                    bf16_hi(yv[jj].y), bf16_lo(yv[jj].z), bf16_hi(yv[jj].z),
+                                    bf16_lo(yv[jj].w), bf16_hi(yv[jj].w)};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) part[jj] = __fmaf_rn(g[c], f[c], part[jj]);
+                const float w = s_w[j0 + jj];
+                uint4 o;
+                o.x = pack_bf16x2(__fmul_rn(w, g[0]), __fmul_rn(w, g[1]));
+                o.y = pack_bf16x2(__fmul_rn(w, g[2]), __fmul_rn(w, g[3]));
+                o.z = pack_bf16x2(__fmul_rn(w, g[4]), __fmul_rn(w, g[5]));
+                o.w = pack_bf16x2(__fmul_rn(w, g[6]), __fmul_rn(w, g[7]));
+                grad_y[(int64_t)d * vpr + v] = o;
+            }
+        }
+        // fixed-order reduction: xor tree in the warp, then warps in order
+#pragma unroll
+        for (int jj = 0; jj < kSlotBatch; ++jj)
+            for (int o = 16; o > 0; o >>= 1) part[jj] += __shfl_xor_sync(kFull, part[jj], o);
+        if (lane == 0)
+#pragma unroll
+            for (int jj = 0; jj < kSlotBatch; ++jj) s_red[warp][jj] = part[jj];
+        __syncthreads();
+        if ((int)threadIdx.x < nj) {
+            float sum = 0.0f;
+            for (int w = 0; w < nwarps; ++w) sum += s_red[w][threadIdx.x];
+            grad_w[t * k + j0 + threadIdx.x] = s_row[j0 + threadIdx.x] >= 0 ? sum : 0.0f;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
+                                    int64_t y_rows, const float* w, int H, void* grad_y,
+                                    int64_t grad_y_rows, float* grad_w, cudaStream_t s)
+{
+    if (h.T == 0)
+        return cudaSuccess;
+    const int64_t vpr = H / 8;
+    const int threads = (int)std::min<int64_t>(kMaxThreads, 32 * ((vpr + 31) / 32));
+    return launch_pdl(combine_backward_kernel, (unsigned)h.T, (unsigned)threads, 0, s,
+                      static_cast<const uint4*>(grad_out), static_cast<const uint4*>(y), y_rows, w,
+                      h.T, h.k, vpr, h.dst_row, static_cast<uint4*>(grad_y), grad_y_rows, grad_w,
+                      h.err);
+}
+
+}  // namespace ep

@@ -10,6 +10,9 @@
 // accumulator, one fused multiply-add per used slot in slot order
 // j = 0..k-1, round-to-nearest-even to bf16 at the end.
 //
+// With a null weight pointer every weight is 1 (fma(1, y, acc) rounds like
+// acc + y): that is the backward of dispatch, grad_x[t] = sum of the k rows.
+//
 // HBM-bound: k row reads (k x 2H bytes) and one row write per token.  Work
 // unit: one warp x (token, 32 x U 16-byte vectors of the row).  When every
 // slot of the token is used and in range (the common case), all k x U loads
@@ -99,7 +102,7 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
         float w = 0.0f;
         if (lane < k) {
             d = __ldg(dst_row + t * k + lane);
-            w = __ldg(weights + t * k + lane);
+            w = weights ? __ldg(weights + t * k + lane) : 1.0f;  // null: unit weights
         }
         if (d >= y_rows) {
             atomicOr(err, kErrCombineCap);

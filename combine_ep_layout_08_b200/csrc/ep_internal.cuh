@@ -93,7 +93,10 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
                                 float* recv_scales, int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
-                           int H, void* out, cudaStream_t s);
+                           int H, void* out, cudaStream_t s);  // w == nullptr: unit weights
+cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
+                                    int64_t y_rows, const float* w, int H, void* grad_y,
+                                    int64_t grad_y_rows, float* grad_w, cudaStream_t s);
 
 // Persistent-grid size: min(resident blocks per SM from the occupancy API,
 // max_per_sm) x the SM count of the current device, cached per kernel and

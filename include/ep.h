@@ -200,6 +200,37 @@ ep_status_t ep_combine_range(ep_handle_t h, int t_begin, int t_count, const void
                              int64_t y_rows, const float* topk_weights_rows, int H,
                              void* out_rows, void* stream);
 
+/* Backward of ep_dispatch for the last layout: grad_x[t] = sum over the used
+ * slots of grad_recv[dst_row[t][j]], accumulated in fp32 in slot order
+ * j = 0..k-1, rounded to bf16 (the forward sent x[t] to each of those rows).
+ * grad_recv: device bf16 [grad_rows][H] in the receive layout (for an FP8
+ * dispatch: the gradient with respect to the dequantised rows); grad_x:
+ * device bf16 [T][H].  16-byte aligned, H % 8 == 0.  A row >= grad_rows is
+ * skipped and sets EP_ERR_CAPACITY.
+ *
+ * The pages name training as a use (pomoai page, 核心使用场景; yololab page,
+ * high-throughput mode) but define no gradients; these are the gradients of
+ * the forward definitions. */
+ep_status_t ep_dispatch_backward(ep_handle_t h, const void* grad_recv, int64_t grad_rows, int H,
+                                 void* grad_x, void* stream);
+
+/* Backward of ep_combine for the last layout, given grad_out (device bf16
+ * [T][H]) and the forward's y (device bf16 [y_rows][H]) and topk_weights
+ * (device fp32 [T][k]):
+ *   grad_y[dst_row[t][j]][h] = bf16_rn(w[t][j] * grad_out[t][h])   (one fp32 product)
+ *   grad_weights[t][j]       = sum_h grad_out[t][h] * y[dst_row[t][j]][h]   (fp32)
+ * grad_y: device bf16 [grad_y_rows][H] in the receive layout (pad rows keep
+ * their contents); grad_weights: device fp32 [T][k], 0 for unused slots.
+ * The dot products use fused multiply-adds per thread and a fixed reduction
+ * tree: bitwise repeatable, within the fp32 summation bound
+ * H * 2^-24 * sum |grad_out * y| of the exact value.  16-byte aligned
+ * bf16 arrays, 4-byte aligned fp32 arrays, H % 8 == 0.  A row beyond
+ * y_rows or grad_y_rows is skipped (grad_weights 0) and sets
+ * EP_ERR_CAPACITY. */
+ep_status_t ep_combine_backward(ep_handle_t h, const void* grad_out, const void* y,
+                                int64_t y_rows, const float* topk_weights, int H, void* grad_y,
+                                int64_t grad_y_rows, float* grad_weights, void* stream);
+
 /* Wait for the stream (SYNCHRONISING), read and clear the sticky device
  * error word.  Returns EP_ERR_TIMEOUT, EP_ERR_BAD_INDEX or EP_ERR_CAPACITY
  * (in that order of precedence when several are set) or EP_OK. */

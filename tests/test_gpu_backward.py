@@ -1,0 +1,109 @@
+"""GPU parity of the backward entry points against the oracle.
+
+ep_dispatch_backward: bit-exact (fp32 sum in slot order, like combine).
+ep_combine_backward: grad_y bit-exact on every used row (one fp32 product,
+then bf16); pad rows keep their sentinel; grad_weights within the fp32
+summation bound H * 2^-24 * sum|grad_out * y| (plus the oracle's one
+rounding) of the oracle's fp64 dot product, and bitwise repeatable.
+"""
+import numpy as np
+import pytest
+import torch
+
+from workloads import make_workload, make_x, random_topk
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(idx, E, R, B=128):
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV
+
+    T, k = idx.shape
+    h = ep.ep_handle_create(max(T, 1), k, E, R, B, device=DEV)
+    ep.ep_layout(h, torch.from_numpy(idx).to(DEV))
+    return h
+
+
+@pytest.mark.parametrize("T,H,E,R,k,p_unused", [
+    (1, 8, 4, 2, 2, 0.0),
+    (200, 1032, 32, 8, 8, 0.1),     # 129 vectors: a ragged unit
+    (64, 7168, 256, 8, 8, 0.0),
+    (50, 512, 64, 8, 20, 0.2),      # k > 8: the general path
+])
+def test_dispatch_backward_bit_exact(oracle, T, H, E, R, k, p_unused):
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import bf16_to_bits, bits_to_bf16
+
+    rng = np.random.default_rng(T + H + k)
+    idx, _ = random_topk(T, E, k, rng, p_unused=p_unused)
+    lay = oracle.layout(idx, E, R)
+    g = make_x(max(lay.total_rows, 1), H, rng)
+    h = _setup(idx, E, R)
+    gx = ep.ep_dispatch_backward(h, bits_to_bf16(g))
+    ep.ep_handle_check(h)
+    assert np.array_equal(bf16_to_bits(gx), oracle.dispatch_backward(g, lay.dst_row))
+
+
+def _combine_backward_case(oracle, idx, E, R, H, rng, w=None):
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV, bf16_to_bits, bits_to_bf16
+
+    T, k = idx.shape
+    lay = oracle.layout(idx, E, R)
+    P = lay.total_rows
+    y = make_x(max(P, 1), H, rng)
+    g = make_x(T, H, rng)
+    if w is None:
+        w = rng.random((T, k)).astype(np.float32)
+    h = _setup(idx, E, R)
+    gy_dev = torch.full((max(P, 1), H), 0, dtype=torch.int16, device=DEV)
+    gy_dev.fill_(0x5A5A)
+    gy_dev = gy_dev.view(torch.bfloat16)
+    gy, gw = ep.ep_combine_backward(h, bits_to_bf16(g), bits_to_bf16(y),
+                                    torch.from_numpy(w).to(DEV), grad_y=gy_dev)
+    ep.ep_handle_check(h)
+    gy_ref, gw_ref = oracle.combine_backward(g, y, w, lay.dst_row)
+    got = bf16_to_bits(gy)
+    rows = lay.dst_row[lay.dst_row >= 0]
+    assert np.array_equal(got[rows], gy_ref[rows])
+    pad = np.setdiff1d(np.arange(P), rows)
+    assert np.all(got[pad] == 0x5A5A), "a pad row of grad_y was written"
+    gw_got = gw.cpu().numpy()
+    yf = oracle.bf16_to_f32(y).astype(np.float64)
+    gf = oracle.bf16_to_f32(g).astype(np.float64)
+    for t in range(T):
+        for j in range(k):
+            d = lay.dst_row[t, j]
+            if d < 0:
+                assert gw_got[t, j] == 0.0
+                continue
+            bound = H * 2.0 ** -24 * float(np.abs(gf[t] * yf[d]).sum()) + 2.0 ** -24 * abs(gw_ref[t, j])
+            assert abs(float(gw_got[t, j]) - float(gw_ref[t, j])) <= bound + 1e-30, (t, j)
+    # bitwise repeatable
+    _, gw2 = ep.ep_combine_backward(h, bits_to_bf16(g), bits_to_bf16(y),
+                                    torch.from_numpy(w).to(DEV))
+    assert np.array_equal(gw2.cpu().numpy().view(np.uint32), gw_got.view(np.uint32))
+    return gw_got, gw_ref
+
+
+@pytest.mark.parametrize("T,H,E,R,k,p_unused", [
+    (1, 8, 4, 2, 2, 0.0),
+    (120, 1032, 32, 8, 8, 0.1),
+    (48, 7168, 256, 8, 8, 0.0),
+    (40, 2048, 64, 8, 20, 0.2),      # k > 8: slots in batches of 8
+    (30, 64, 16, 4, 1, 0.0),
+])
+def test_combine_backward(oracle, T, H, E, R, k, p_unused):
+    rng = np.random.default_rng(3 * T + H + k)
+    idx, _ = random_topk(T, E, k, rng, p_unused=p_unused)
+    _combine_backward_case(oracle, idx, E, R, H, rng)
+
+
+def test_combine_backward_full_dsv3_shape(oracle):
+    w = make_workload("dsv3", 0, T=512)
+    rng = np.random.default_rng(77)
+    gw, ref = _combine_backward_case(oracle, w.topk_idx, w.E, w.R, w.H, rng, w.topk_weights)
+    # typical error is far inside the worst-case bound
+    rel = np.abs(gw - ref) / np.maximum(np.abs(ref), 1e-6)
+    assert np.median(rel) < 1e-5
