@@ -75,6 +75,12 @@ def _load():
             lib.oracle_dispatch_backward.restype = i32
             lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
             lib.oracle_combine_backward.restype = i32
+            lib.oracle_dispatch_weights.argtypes = [P, P, i64, i32, P, i64]
+            lib.oracle_dispatch_weights.restype = i32
+            lib.oracle_zero_pad_rows.argtypes = [P, i64, P, i64]
+            lib.oracle_zero_pad_rows.restype = None
+            lib.oracle_dispatch_fp8_mn.argtypes = [P, i64, i32, i64, P, P, P, i64, i64]
+            lib.oracle_dispatch_fp8_mn.restype = i32
             for name in ("oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
                          "oracle_f32_to_bf16_array"):
                 getattr(lib, name).argtypes = [P, P, i64]
@@ -288,6 +294,47 @@ def combine_backward(grad_out_bits: np.ndarray, y_bits: np.ndarray, topk_weights
     if rc != OK:
         raise OracleError(rc, "oracle_combine_backward")
     return gy[:rows], gw
+
+
+# ---------------------------------------------------------------- GEMM-ready layout
+
+def dispatch_weights(topk_weights: np.ndarray, dst_row: np.ndarray, recv_rows: int,
+                     fill: float = 0.0) -> np.ndarray:
+    """recv_w[dst_row[t, j]] = w[t, j]; pad rows keep `fill`."""
+    w = np.ascontiguousarray(topk_weights, dtype=np.float32)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    T, k = dst_row.shape
+    out = np.full(max(recv_rows, 1), fill, np.float32)
+    rc = _load().oracle_dispatch_weights(_p(w), _p(dst_row), T, k, _p(out), recv_rows)
+    if rc != OK:
+        raise OracleError(rc, "oracle_dispatch_weights")
+    return out[:recv_rows]
+
+
+def zero_pad_rows(recv_src: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """A copy of `rows` (any dtype, [P, ...]) with every pad row zeroed."""
+    recv_src = np.ascontiguousarray(recv_src, dtype=np.int32)
+    out = np.ascontiguousarray(rows).copy()
+    P = recv_src.shape[0]
+    if P:
+        _load().oracle_zero_pad_rows(_p(recv_src), P, _p(out.view(np.uint8)),
+                                     out.nbytes // out.shape[0])
+    return out
+
+
+def dispatch_fp8_mn(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int, ld: int):
+    """FP8 dispatch with MN-major scales: (recv_q [P, H], scales_mn [H/128, ld])."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    T, H = x_bits.shape
+    k = dst_row.shape[1]
+    q = np.zeros((max(recv_rows, 1), H), np.uint8)
+    s = np.zeros((H // 128, max(ld, 1)), np.float32)
+    rc = _load().oracle_dispatch_fp8_mn(_p(x_bits), T, k, H, _p(dst_row), _p(q), _p(s), ld,
+                                        recv_rows)
+    if rc != OK:
+        raise OracleError(rc, "oracle_dispatch_fp8_mn")
+    return q[:recv_rows], s[:, :ld]
 
 
 def pipeline(x_bits, topk_idx, topk_weights, E, R, fmt, c, block_m=128):

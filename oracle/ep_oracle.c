@@ -506,3 +506,74 @@ int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t
         }
     return OR_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* GEMM-ready receive layout.  The pages say high-throughput and low-    */
+/* latency kernels share one "GEMM layout" (DeepEP v2 release notes,     */
+/* "Có gì mới trong v2"; the pomoai page, ElasticBuffer paragraph)       */
+/* without defining it; these are the readings taken for an expert GEMM  */
+/* that consumes the receive buffer directly.                            */
+/* ------------------------------------------------------------------ */
+
+/* Per-row routing weight: recv_w[dst_row[t][j]] = w[t][j] for every used
+ * slot; pad rows are not written. */
+int oracle_dispatch_weights(const float* w, const int32_t* dst_row, int64_t T, int k,
+                            float* recv_w, int64_t recv_cap)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int64_t d = dst_row[t * k + j];
+            if (d < 0)
+                continue;
+            if (d >= recv_cap)
+                return OR_ERR_CAPACITY;
+            recv_w[d] = w[t * k + j];
+        }
+    return OR_OK;
+}
+
+/* Zero the pad rows of a row buffer in the receive layout: every row r < P
+ * with recv_src[r] == -1 gets row_bytes zero bytes. */
+void oracle_zero_pad_rows(const int32_t* recv_src, int64_t P, uint8_t* rows, int64_t row_bytes)
+{
+    for (int64_t r = 0; r < P; ++r)
+        if (recv_src[r] < 0)
+            memset(rows + r * row_bytes, 0, (size_t)row_bytes);
+}
+
+/* MN-major FP8 scales: the same scales as oracle_dispatch_fp8, stored as
+ * scales_mn[b][row] with leading dimension ld (b = 128-channel block). */
+int oracle_dispatch_fp8_mn(const uint16_t* x, int64_t T, int k, int64_t H,
+                           const int32_t* dst_row, uint8_t* recv_q, float* scales_mn,
+                           int64_t ld, int64_t recv_cap)
+{
+    if (H % 128 != 0 || ld < recv_cap)
+        return OR_ERR_ARG;
+    const int64_t nb = H / 128;
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    if (!q || !s) {
+        free(q);
+        free(s);
+        return OR_ERR_ARG;
+    }
+    int rc = OR_OK;
+    for (int64_t t = 0; t < T && rc == OR_OK; ++t) {
+        oracle_quantize_token_fp8(x + t * H, H, q, s);
+        for (int j = 0; j < k; ++j) {
+            int64_t d = dst_row[t * k + j];
+            if (d < 0)
+                continue;
+            if (d >= recv_cap) {
+                rc = OR_ERR_CAPACITY;
+                break;
+            }
+            memcpy(recv_q + d * H, q, (size_t)H);
+            for (int64_t b = 0; b < nb; ++b)
+                scales_mn[b * ld + d] = s[b];
+        }
+    }
+    free(q);
+    free(s);
+    return rc;
+}
