@@ -28,6 +28,7 @@ __all__ = [
     "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
     "ep_layout", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
     "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
+    "ep_dispatch_weights", "ep_zero_pad_rows",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
@@ -47,7 +48,8 @@ EP_ERR_TIMEOUT = 9
 
 EP_FMT_BF16 = 0
 EP_FMT_FP8_E4M3_1X128 = 1
-_FMTS = {"bf16": EP_FMT_BF16, "fp8": EP_FMT_FP8_E4M3_1X128}
+EP_FMT_FP8_E4M3_1X128_MN = 2
+_FMTS = {"bf16": EP_FMT_BF16, "fp8": EP_FMT_FP8_E4M3_1X128, "fp8_mn": EP_FMT_FP8_E4M3_1X128_MN}
 
 VIEWS = {
     "num_tokens_per_expert": (0, torch.int32),
@@ -97,6 +99,8 @@ def load_library():
             "ep_combine": ([P, P, I64, P, I, P, P], I),
             "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
             "ep_dispatch_backward": ([P, P, I64, I, P, P], I),
+            "ep_dispatch_weights": ([P, P, P, I64, P], I),
+            "ep_zero_pad_rows": ([P, P, I64, I64, P], I),
             "ep_combine_backward": ([P, P, P, I64, P, I, P, I64, P, P], I),
             "ep_combine_range": ([P, I, I, P, I64, P, I, P, P], I),
             "ep_handle_check": ([P, P], I),
@@ -260,11 +264,15 @@ def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
     if recv_x is None:
         cap = capacity_rows if capacity_rows is not None else \
             ep_recv_rows_upper_bound(T, h.k, h.E, h.block_m)
+        if f == EP_FMT_FP8_E4M3_1X128_MN:
+            cap = (cap + 3) // 4 * 4
         dt = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
         recv_x = torch.empty((cap, H), dtype=dt, device=x.device)
     cap = recv_x.shape[0]
     if f == EP_FMT_FP8_E4M3_1X128 and recv_scales is None:
         recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+    if f == EP_FMT_FP8_E4M3_1X128_MN and recv_scales is None:
+        recv_scales = torch.empty((H // 128, cap), dtype=torch.float32, device=x.device)
     want = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
     if recv_x.dtype != want or recv_x.shape[1] != H or not recv_x.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_x must be contiguous %s [*, %d]"
@@ -273,11 +281,15 @@ def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
         if (recv_scales.dtype != torch.float32 or recv_scales.shape[0] < cap
                 or recv_scales.shape[1] != H // 128 or not recv_scales.is_contiguous()):
             raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_scales must be f32 [cap, H/128]")
+    if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128_MN:
+        if (recv_scales.dtype != torch.float32 or tuple(recv_scales.shape) != (H // 128, cap)
+                or not recv_scales.is_contiguous()):
+            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_scales must be f32 [H/128, cap]")
     with _on(h):
         _check(load_library().ep_dispatch(h.handle, _ptr(x), H, f, _ptr(recv_x),
                                           _ptr(recv_scales) if f else ctypes.c_void_p(0), cap,
                                           _stream(h.device)), "ep_dispatch")
-    return recv_x, (recv_scales if f == EP_FMT_FP8_E4M3_1X128 else None)
+    return recv_x, (recv_scales if f != EP_FMT_BF16 else None)
 
 
 def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,
@@ -376,6 +388,39 @@ def ep_combine_backward(h: EPHandle, grad_out: torch.Tensor, y: torch.Tensor,
             h.handle, _ptr(grad_out), _ptr(y), y.shape[0], _ptr(topk_weights), H, _ptr(grad_y),
             grad_y.shape[0], _ptr(grad_w), _stream(h.device)), "ep_combine_backward")
     return grad_y, grad_w
+
+
+def ep_dispatch_weights(h: EPHandle, topk_weights: torch.Tensor,
+                        recv_weights: Optional[torch.Tensor] = None,
+                        capacity_rows: Optional[int] = None) -> torch.Tensor:
+    """recv_weights[dst_row[t, j]] = topk_weights[t, j] (f32, receive layout)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch_weights")
+    if (topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (h.T, h.k)
+            or not topk_weights.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_weights: topk_weights must be f32 [T, k]")
+    if recv_weights is None:
+        cap = capacity_rows if capacity_rows is not None else \
+            ep_recv_rows_upper_bound(h.T, h.k, h.E, h.block_m)
+        recv_weights = torch.zeros(cap, dtype=torch.float32, device=topk_weights.device)
+    with _on(h):
+        _check(load_library().ep_dispatch_weights(h.handle, _ptr(topk_weights), _ptr(recv_weights),
+                                                  recv_weights.shape[0], _stream(h.device)),
+               "ep_dispatch_weights")
+    return recv_weights
+
+
+def ep_zero_pad_rows(h: EPHandle, rows: torch.Tensor) -> torch.Tensor:
+    """Zero the pad rows (receive layout) of a contiguous [capacity, ...] tensor in place."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_zero_pad_rows")
+    if not rows.is_contiguous() or rows.dim() < 1:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_zero_pad_rows: rows must be contiguous")
+    row_bytes = rows[0].numel() * rows.element_size() if rows.shape[0] else 1
+    with _on(h):
+        _check(load_library().ep_zero_pad_rows(h.handle, _ptr(rows), row_bytes, rows.shape[0],
+                                               _stream(h.device)), "ep_zero_pad_rows")
+    return rows
 
 
 def ep_handle_check(h: EPHandle, raise_on_error: bool = True) -> int:

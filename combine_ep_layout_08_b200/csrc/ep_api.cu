@@ -307,15 +307,18 @@ ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, in
         return EP_ERR_STATE;
     if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
         return EP_ERR_INVALID_ARG;
-    if (fmt != EP_FMT_BF16 && fmt != EP_FMT_FP8_E4M3_1X128)
+    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
+    if (fmt != EP_FMT_BF16 && !fp8)
         return EP_ERR_INVALID_ARG;
     if (fmt == EP_FMT_BF16 && H % 8 != 0)
         return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_FP8_E4M3_1X128 && H % 128 != 0)
+    if (fp8 && H % 128 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_FP8_E4M3_1X128_MN && recv_capacity_rows % 4 != 0)
         return EP_ERR_INVALID_ARG;
     if (t_count > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
         return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_FP8_E4M3_1X128 && t_count > 0 && recv_capacity_rows > 0 && !recv_scales)
+    if (fp8 && t_count > 0 && recv_capacity_rows > 0 && !recv_scales)
         return EP_ERR_INVALID_ARG;
     if (!ep::aligned(x, 16) || !ep::aligned(recv_x, 16) || !ep::aligned(recv_scales, 16))
         return EP_ERR_ALIGNMENT;
@@ -325,8 +328,10 @@ ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, in
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t rc = (fmt == EP_FMT_BF16)
                          ? ep::launch_dispatch_bf16(sub, x, H, recv_x, recv_capacity_rows, s)
-                         : ep::launch_dispatch_fp8(sub, x, H, recv_x, recv_scales,
-                                                   recv_capacity_rows, s);
+                         : ep::launch_dispatch_fp8(
+                               sub, x, H, recv_x, recv_scales,
+                               fmt == EP_FMT_FP8_E4M3_1X128_MN ? recv_capacity_rows : 0,
+                               recv_capacity_rows, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
 }
 
@@ -386,6 +391,39 @@ ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const voi
 {
     return combine_impl(ep::as_handle(hh), t_begin, t_count, y, y_rows, topk_weights_rows, H,
                         out_rows, stream, "ep_combine_range");
+}
+
+ep_status_t ep_dispatch_weights(ep_handle_t hh, const float* topk_weights, float* recv_weights,
+                                int64_t recv_capacity_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || recv_capacity_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (h->T > 0 && (!topk_weights || (!recv_weights && recv_capacity_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(topk_weights, 4) || !ep::aligned(recv_weights, 4))
+        return EP_ERR_ALIGNMENT;
+    cudaError_t rc = ep::launch_dispatch_weights(*h, topk_weights, recv_weights,
+                                                 recv_capacity_rows,
+                                                 static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_weights");
+}
+
+ep_status_t ep_zero_pad_rows(ep_handle_t hh, void* rows, int64_t row_bytes, int64_t capacity_rows,
+                             void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || row_bytes <= 0 || capacity_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (!rows && capacity_rows > 0)
+        return EP_ERR_INVALID_ARG;
+    cudaError_t rc = ep::launch_zero_pad_rows(*h, rows, row_bytes, capacity_rows,
+                                              static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_zero_pad_rows");
 }
 
 ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t grad_rows, int H,

@@ -151,6 +151,14 @@ dispatch_bf16_kernel(const uint4* __restrict__ x, int T, int k, int64_t vpr,
     }
 }
 
+// Scale of (row, block): row-major [row][nblk] when ld == 0, else MN-major
+// [block][ld] (each block's scales contiguous over rows, for GEMMs that read
+// scales along M).
+__device__ __forceinline__ int64_t scale_index(int64_t row, int64_t blk, int nblk, int64_t ld)
+{
+    return ld == 0 ? row * nblk + blk : blk * ld + row;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
@@ -169,7 +177,8 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d)
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
                     const int32_t* __restrict__ dst_row, uint8_t* __restrict__ recv_q,
-                    float* __restrict__ recv_scales, int64_t cap_rows, int32_t* err)
+                    float* __restrict__ recv_scales, int64_t scales_ld, int64_t cap_rows,
+                    int32_t* err)
 {
     pdl_wait();
     pdl_trigger();
@@ -245,7 +254,7 @@ dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
                 if (v0 + 32 * i < vpr)
                     dq[v0 + 32 * i] = q[i];
             if (sc_ok)
-                recv_scales[(int64_t)dj * nblk + blk] = my_scale;
+                recv_scales[scale_index(dj, blk, nblk, scales_ld)] = my_scale;
         }
     }
 }
@@ -260,7 +269,8 @@ dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                         const int32_t* __restrict__ dst_row, uint8_t* __restrict__ recv_q,
-                        float* __restrict__ recv_scales, int64_t cap_rows, int32_t* err)
+                        float* __restrict__ recv_scales, int64_t scales_ld, int64_t cap_rows,
+                        int32_t* err)
 {
     pdl_wait();
     pdl_trigger();
@@ -350,7 +360,7 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                 if (v0 + 32 * i < vpr)
                     dq[v0 + 32 * i] = q[i];
             if (sc_ok)
-                recv_scales[(int64_t)dj * nblk + blk] = my_scale;
+                recv_scales[scale_index(dj, blk, nblk, scales_ld)] = my_scale;
         }
     }
 }
@@ -382,17 +392,19 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
 }
 
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
-                                float* recv_scales, int64_t cap_rows, cudaStream_t s)
+                                float* recv_scales, int64_t scales_ld, int64_t cap_rows,
+                                cudaStream_t s)
 {
     if (h.T == 0)
         return cudaSuccess;
     if (aligned32(x))
         return launch_pdl(dispatch_fp8_v32_kernel, unit_grid(h.T, H / 16, kUnitVec32Fp8),
                           kThreads, 0, s, static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row,
-                          static_cast<uint8_t*>(recv_q), recv_scales, cap_rows, h.err);
+                          static_cast<uint8_t*>(recv_q), recv_scales, scales_ld, cap_rows,
+                          h.err);
     return launch_pdl(dispatch_fp8_kernel, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
                       static_cast<const uint4*>(x), h.T, h.k, H, h.dst_row,
-                      static_cast<uint8_t*>(recv_q), recv_scales, cap_rows, h.err);
+                      static_cast<uint8_t*>(recv_q), recv_scales, scales_ld, cap_rows, h.err);
 }
 
 }  // namespace ep

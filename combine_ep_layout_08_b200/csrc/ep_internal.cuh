@@ -91,7 +91,12 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
 cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,
                                  int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
-                                float* recv_scales, int64_t cap_rows, cudaStream_t s);
+                                float* recv_scales, int64_t scales_ld, int64_t cap_rows,
+                                cudaStream_t s);  // scales_ld 0: row-major scales
+cudaError_t launch_dispatch_weights(const Handle& h, const float* w, float* recv_w,
+                                    int64_t cap_rows, cudaStream_t s);
+cudaError_t launch_zero_pad_rows(const Handle& h, void* rows, int64_t row_bytes, int64_t cap_rows,
+                                 cudaStream_t s);
 cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
                            int H, void* out, cudaStream_t s);  // w == nullptr: unit weights
 cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,

@@ -81,8 +81,13 @@ typedef enum {
 } ep_status_t;
 
 typedef enum {
-    EP_FMT_BF16 = 0,            /* receive rows are the bf16 input rows */
-    EP_FMT_FP8_E4M3_1X128 = 1   /* e4m3 rows + one fp32 scale per 128 channels */
+    EP_FMT_BF16 = 0,              /* receive rows are the bf16 input rows */
+    EP_FMT_FP8_E4M3_1X128 = 1,    /* e4m3 rows + one fp32 scale per 128 channels,
+                                     scales row-major [rows][H/128] */
+    EP_FMT_FP8_E4M3_1X128_MN = 2  /* the same codes and scales, scales MN-major
+                                     [H/128][recv_capacity_rows]: each block's scales
+                                     contiguous over rows (recv_capacity_rows % 4 == 0,
+                                     so every block's column starts 16-byte aligned) */
 } ep_fmt_t;
 
 /* Views of the layout held in the workspace (see ep_handle_view). */
@@ -199,6 +204,27 @@ ep_status_t ep_dispatch_range(ep_handle_t h, int t_begin, int t_count, const voi
 ep_status_t ep_combine_range(ep_handle_t h, int t_begin, int t_count, const void* y,
                              int64_t y_rows, const float* topk_weights_rows, int H,
                              void* out_rows, void* stream);
+
+/* GEMM-ready receive layout.  The pages say the high-throughput and
+ * low-latency kernels share one "GEMM layout" (DeepEP v2 release notes, "Có
+ * gì mới trong v2") without defining it; these helpers complete the reading
+ * taken here for an expert GEMM that consumes the receive buffer directly.
+ *
+ * ep_dispatch_weights: recv_weights[dst_row[t][j]] = topk_weights[t][j] for
+ * every used slot of the last layout (device fp32 [T][k] in, device fp32
+ * [recv_capacity_rows] out, 4-byte aligned; pad rows are not written), so the
+ * expert op can scale its rows.  A row >= recv_capacity_rows sets
+ * EP_ERR_CAPACITY.
+ *
+ * ep_zero_pad_rows: set every pad row of a buffer in the receive layout to
+ * zero bytes (rows: device, capacity_rows rows of row_bytes bytes; 16-byte
+ * stores when row_bytes % 16 == 0 and rows is 16-byte aligned), so a GEMM
+ * over whole 128-row blocks reads zeros there.  Works for recv_x, row-major
+ * scales, y or grad_y.  A pad row >= capacity_rows sets EP_ERR_CAPACITY. */
+ep_status_t ep_dispatch_weights(ep_handle_t h, const float* topk_weights, float* recv_weights,
+                                int64_t recv_capacity_rows, void* stream);
+ep_status_t ep_zero_pad_rows(ep_handle_t h, void* rows, int64_t row_bytes, int64_t capacity_rows,
+                             void* stream);
 
 /* Backward of ep_dispatch for the last layout: grad_x[t] = sum over the used
  * slots of grad_recv[dst_row[t][j]], accumulated in fp32 in slot order
