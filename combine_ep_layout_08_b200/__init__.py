@@ -26,7 +26,7 @@ import torch
 
 __all__ = [
     "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
-    "ep_layout", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
+    "ep_layout", "ep_layout_dispatch", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
     "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_weights", "ep_zero_pad_rows",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
@@ -93,6 +93,7 @@ def load_library():
             "ep_handle_create": ([P, SZ, I, I, I, I, I, ctypes.POINTER(P)], I),
             "ep_handle_destroy": ([P], None),
             "ep_layout": ([P, P, I, P], I),
+            "ep_layout_dispatch": ([P, P, I, P, I, I, P, P, I64, P], I),
             "ep_handle_view": ([P, I, ctypes.POINTER(I64)], P),
             "ep_handle_read_counts": ([P, P, P, P, P, P], I),
             "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
@@ -249,47 +250,78 @@ def ep_handle_read_counts(h: EPHandle) -> dict:
                 total_recv_rows=int(d[0]))
 
 
-def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
-                recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
-                capacity_rows: Optional[int] = None):
-    """Scatter bf16 x [T, H] into the receive layout.  Returns (recv_x, recv_scales);
-    recv_scales is None for BF16.  Buffers not given are allocated with
-    capacity_rows rows (default: the no-sync upper bound)."""
-    if h.T is None:
-        raise EPError(EP_ERR_STATE, "ep_dispatch")
-    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != h.T or not x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: x must be contiguous bf16 [T, H]")
-    T, H = x.shape
-    f = _FMTS[fmt]
+def _recv_buffers(h: EPHandle, T: int, H: int, f: int, device, recv_x, recv_scales,
+                  capacity_rows):
+    """Allocate missing receive buffers (default capacity: the no-sync bound)
+    and check the given ones."""
     if recv_x is None:
         cap = capacity_rows if capacity_rows is not None else \
             ep_recv_rows_upper_bound(T, h.k, h.E, h.block_m)
         if f == EP_FMT_FP8_E4M3_1X128_MN:
             cap = (cap + 3) // 4 * 4
         dt = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
-        recv_x = torch.empty((cap, H), dtype=dt, device=x.device)
+        recv_x = torch.empty((cap, H), dtype=dt, device=device)
     cap = recv_x.shape[0]
     if f == EP_FMT_FP8_E4M3_1X128 and recv_scales is None:
-        recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=x.device)
+        recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=device)
     if f == EP_FMT_FP8_E4M3_1X128_MN and recv_scales is None:
-        recv_scales = torch.empty((H // 128, cap), dtype=torch.float32, device=x.device)
+        recv_scales = torch.empty((H // 128, cap), dtype=torch.float32, device=device)
     want = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
     if recv_x.dtype != want or recv_x.shape[1] != H or not recv_x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_x must be contiguous %s [*, %d]"
-                      % (want, H))
+        raise EPError(EP_ERR_INVALID_ARG, "recv_x must be contiguous %s [*, %d]" % (want, H))
     if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128:
         if (recv_scales.dtype != torch.float32 or recv_scales.shape[0] < cap
                 or recv_scales.shape[1] != H // 128 or not recv_scales.is_contiguous()):
-            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_scales must be f32 [cap, H/128]")
+            raise EPError(EP_ERR_INVALID_ARG, "recv_scales must be f32 [cap, H/128]")
     if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128_MN:
         if (recv_scales.dtype != torch.float32 or tuple(recv_scales.shape) != (H // 128, cap)
                 or not recv_scales.is_contiguous()):
-            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: recv_scales must be f32 [H/128, cap]")
+            raise EPError(EP_ERR_INVALID_ARG, "recv_scales must be f32 [H/128, cap]")
+    return recv_x, (recv_scales if f != EP_FMT_BF16 else None)
+
+
+def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
+                recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
+                capacity_rows: Optional[int] = None):
+    """Scatter bf16 x [T, H] into the receive layout.  Returns (recv_x, recv_scales);
+    recv_scales is None for BF16.  Buffers not given are allocated with
+    capacity_rows rows (default: the no-sync upper bound).  fmt: "bf16", "fp8"
+    (row-major scales [cap, H/128]) or "fp8_mn" (MN-major scales [H/128, cap])."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != h.T or not x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: x must be contiguous bf16 [T, H]")
+    T, H = x.shape
+    f = _FMTS[fmt]
+    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
     with _on(h):
         _check(load_library().ep_dispatch(h.handle, _ptr(x), H, f, _ptr(recv_x),
-                                          _ptr(recv_scales) if f else ctypes.c_void_p(0), cap,
+                                          _ptr(recv_scales), recv_x.shape[0],
                                           _stream(h.device)), "ep_dispatch")
-    return recv_x, (recv_scales if f != EP_FMT_BF16 else None)
+    return recv_x, recv_scales
+
+
+def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor, fmt: str = "bf16",
+                       recv_x: Optional[torch.Tensor] = None,
+                       recv_scales: Optional[torch.Tensor] = None,
+                       capacity_rows: Optional[int] = None):
+    """ep_layout then ep_dispatch, in one launch for decode-sized batches."""
+    if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or topk_idx.shape[1] != h.k:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be int64 [T, %d]" % h.k)
+    if not topk_idx.is_cuda or not topk_idx.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be contiguous CUDA")
+    T = topk_idx.shape[0]
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != T or not x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: x must be contiguous bf16 [T, H]")
+    H = x.shape[1]
+    f = _FMTS[fmt]
+    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
+    with _on(h):
+        _check(load_library().ep_layout_dispatch(
+            h.handle, _ptr(topk_idx), T, _ptr(x), H, f, _ptr(recv_x), _ptr(recv_scales),
+            recv_x.shape[0], _stream(h.device)), "ep_layout_dispatch")
+    h.T = T
+    return recv_x, recv_scales
 
 
 def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,

@@ -136,6 +136,111 @@ cudaError_t persistent_grid(const void* kernel, int block_threads, size_t dyn_sm
 
 using ep::Handle;
 
+namespace {
+
+// Dispatch / combine of the tokens [t_begin, t_begin + t_count) of the last
+// layout: the kernels see a shallow copy of the handle whose token count and
+// dst_row start at the range.
+// Argument checks of a dispatch of t_count tokens (no launch).
+ep_status_t dispatch_check(int t_count, const void* x, int H, ep_fmt_t fmt, const void* recv_x,
+                           const float* recv_scales, int64_t recv_capacity_rows)
+{
+    if (H <= 0 || recv_capacity_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
+    if (fmt != EP_FMT_BF16 && !fp8)
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_BF16 && H % 8 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (fp8 && H % 128 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (fmt == EP_FMT_FP8_E4M3_1X128_MN && recv_capacity_rows % 4 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (t_count > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (fp8 && t_count > 0 && recv_capacity_rows > 0 && !recv_scales)
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(x, 16) || !ep::aligned(recv_x, 16) || !ep::aligned(recv_scales, 16))
+        return EP_ERR_ALIGNMENT;
+    return EP_OK;
+}
+
+// Dispatch / combine of the tokens [t_begin, t_begin + t_count) of the last
+// layout: the kernels see a shallow copy of the handle whose token count and
+// dst_row start at the range.
+ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, int H,
+                          ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                          int64_t recv_capacity_rows, void* stream, const char* what)
+{
+    if (!h)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    const ep_status_t st =
+        dispatch_check(t_count, x, H, fmt, recv_x, recv_scales, recv_capacity_rows);
+    if (st != EP_OK)
+        return st;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = (fmt == EP_FMT_BF16)
+                         ? ep::launch_dispatch_bf16(sub, x, H, recv_x, recv_capacity_rows, s)
+                         : ep::launch_dispatch_fp8(
+                               sub, x, H, recv_x, recv_scales,
+                               fmt == EP_FMT_FP8_E4M3_1X128_MN ? recv_capacity_rows : 0,
+                               recv_capacity_rows, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
+}
+
+ep_status_t layout_check(Handle* h, const int64_t* topk_idx, int T)
+{
+    if (!h || T < 0 || T > h->max_tokens || (T > 0 && !topk_idx))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(topk_idx, 8))
+        return EP_ERR_ALIGNMENT;
+    return EP_OK;
+}
+
+// The workspace starts with unknown contents: zero the error word and the
+// grid barrier's words once, on the first layout of the handle.
+ep_status_t clear_error_words_once(Handle* h, cudaStream_t s)
+{
+    if (h->err_cleared)
+        return EP_OK;
+    cudaError_t rc = cudaMemsetAsync(h->err, 0, 3 * sizeof(int32_t), s);
+    if (rc != cudaSuccess)
+        return ep::cuda_fail(rc, "clearing the error words");
+    h->err_cleared = 1;
+    return EP_OK;
+}
+
+ep_status_t combine_impl(Handle* h, int t_begin, int t_count, const void* y, int64_t y_rows,
+                         const float* topk_weights, int H, void* out, void* stream,
+                         const char* what)
+{
+    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    if (t_count > 0 && (!out || !topk_weights || (!y && y_rows > 0)))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(y, 16) || !ep::aligned(out, 16) || !ep::aligned(topk_weights, 4))
+        return EP_ERR_ALIGNMENT;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t rc = ep::launch_combine(sub, y, y_rows, topk_weights, H, out, s);
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t ep_workspace_bytes(int max_tokens, int num_topk, int num_experts, int num_ranks,
@@ -213,19 +318,12 @@ void ep_handle_destroy(ep_handle_t hh)
 ep_status_t ep_layout(ep_handle_t hh, const int64_t* topk_idx, int T, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    if (!h || T < 0 || T > h->max_tokens || (T > 0 && !topk_idx))
-        return EP_ERR_INVALID_ARG;
-    if (!ep::aligned(topk_idx, 8))
-        return EP_ERR_ALIGNMENT;
+    ep_status_t st = layout_check(h, topk_idx, T);
+    if (st != EP_OK)
+        return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (!h->err_cleared) {
-        // The workspace starts with unknown contents: zero the error word and
-        // the grid barrier's words once.
-        cudaError_t rc = cudaMemsetAsync(h->err, 0, 3 * sizeof(int32_t), s);
-        if (rc != cudaSuccess)
-            return ep::cuda_fail(rc, "ep_layout (clear error word)");
-        h->err_cleared = 1;
-    }
+    if ((st = clear_error_words_once(h, s)) != EP_OK)
+        return st;
     cudaError_t rc = ep::launch_layout(*h, topk_idx, T, s);
     if (rc != cudaSuccess) {
         h->has_layout = 0;
@@ -234,6 +332,39 @@ ep_status_t ep_layout(ep_handle_t hh, const int64_t* topk_idx, int T, void* stre
     h->T = T;
     h->has_layout = 1;
     return EP_OK;
+}
+
+ep_status_t ep_layout_dispatch(ep_handle_t hh, const int64_t* topk_idx, int T, const void* x,
+                               int H, ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                               int64_t recv_capacity_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    ep_status_t st = layout_check(h, topk_idx, T);
+    if (st != EP_OK)
+        return st;
+    if ((st = dispatch_check(T, x, H, fmt, recv_x, recv_scales, recv_capacity_rows)) != EP_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool fp8 = fmt != EP_FMT_BF16;
+    const bool v32 = H % 16 == 0 && ep::aligned(x, 32) && (fp8 || ep::aligned(recv_x, 32));
+    if (T > 0 && v32 && ep::fused_layout_dispatch_fits(*h, T)) {
+        if ((st = clear_error_words_once(h, s)) != EP_OK)
+            return st;
+        cudaError_t rc = ep::launch_layout_dispatch(
+            *h, topk_idx, T, x, H, fp8, recv_x, recv_scales,
+            fmt == EP_FMT_FP8_E4M3_1X128_MN ? recv_capacity_rows : 0, recv_capacity_rows, s);
+        if (rc != cudaSuccess) {
+            h->has_layout = 0;
+            return ep::cuda_fail(rc, "ep_layout_dispatch");
+        }
+        h->T = T;
+        h->has_layout = 1;
+        return EP_OK;
+    }
+    if ((st = ep_layout(hh, topk_idx, T, stream)) != EP_OK)
+        return st;
+    return dispatch_impl(h, 0, T, x, H, fmt, recv_x, recv_scales, recv_capacity_rows, stream,
+                         "ep_layout_dispatch");
 }
 
 const void* ep_handle_view(ep_handle_t hh, ep_view_t what, int64_t* count)
@@ -290,76 +421,7 @@ ep_status_t ep_handle_read_counts(ep_handle_t hh, int32_t* num_tokens_per_expert
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_handle_read_counts");
 }
 
-}  // extern "C"
 
-namespace {
-
-// Dispatch / combine of the tokens [t_begin, t_begin + t_count) of the last
-// layout: the kernels see a shallow copy of the handle whose token count and
-// dst_row start at the range.
-ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, int H,
-                          ep_fmt_t fmt, void* recv_x, float* recv_scales,
-                          int64_t recv_capacity_rows, void* stream, const char* what)
-{
-    if (!h || H <= 0 || recv_capacity_rows < 0)
-        return EP_ERR_INVALID_ARG;
-    if (!h->has_layout)
-        return EP_ERR_STATE;
-    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
-        return EP_ERR_INVALID_ARG;
-    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
-    if (fmt != EP_FMT_BF16 && !fp8)
-        return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_BF16 && H % 8 != 0)
-        return EP_ERR_INVALID_ARG;
-    if (fp8 && H % 128 != 0)
-        return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_FP8_E4M3_1X128_MN && recv_capacity_rows % 4 != 0)
-        return EP_ERR_INVALID_ARG;
-    if (t_count > 0 && (!x || (!recv_x && recv_capacity_rows > 0)))
-        return EP_ERR_INVALID_ARG;
-    if (fp8 && t_count > 0 && recv_capacity_rows > 0 && !recv_scales)
-        return EP_ERR_INVALID_ARG;
-    if (!ep::aligned(x, 16) || !ep::aligned(recv_x, 16) || !ep::aligned(recv_scales, 16))
-        return EP_ERR_ALIGNMENT;
-    Handle sub = *h;
-    sub.T = t_count;
-    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = (fmt == EP_FMT_BF16)
-                         ? ep::launch_dispatch_bf16(sub, x, H, recv_x, recv_capacity_rows, s)
-                         : ep::launch_dispatch_fp8(
-                               sub, x, H, recv_x, recv_scales,
-                               fmt == EP_FMT_FP8_E4M3_1X128_MN ? recv_capacity_rows : 0,
-                               recv_capacity_rows, s);
-    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
-}
-
-ep_status_t combine_impl(Handle* h, int t_begin, int t_count, const void* y, int64_t y_rows,
-                         const float* topk_weights, int H, void* out, void* stream,
-                         const char* what)
-{
-    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
-        return EP_ERR_INVALID_ARG;
-    if (!h->has_layout)
-        return EP_ERR_STATE;
-    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
-        return EP_ERR_INVALID_ARG;
-    if (t_count > 0 && (!out || !topk_weights || (!y && y_rows > 0)))
-        return EP_ERR_INVALID_ARG;
-    if (!ep::aligned(y, 16) || !ep::aligned(out, 16) || !ep::aligned(topk_weights, 4))
-        return EP_ERR_ALIGNMENT;
-    Handle sub = *h;
-    sub.T = t_count;
-    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = ep::launch_combine(sub, y, y_rows, topk_weights, H, out, s);
-    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
-}
-
-}  // namespace
-
-extern "C" {
 
 ep_status_t ep_dispatch(ep_handle_t hh, const void* x, int H, ep_fmt_t fmt, void* recv_x,
                         float* recv_scales, int64_t recv_capacity_rows, void* stream)

@@ -1,0 +1,167 @@
+// ep_dispatch_units.cuh -- the per-unit bodies of the 256-bit dispatch
+// kernels, shared by ep_dispatch.cu and the fused layout + dispatch kernel.
+// A unit is one warp's share of one token row: BF16 512 channels (32 lanes x
+// one 32-byte vector), FP8 1024 channels (32 lanes x two 32-byte vectors = 8
+// blocks of 128).  `d` is this lane's destination row for slot j = lane
+// (lanes >= k, unused slots and rows beyond the capacity pass -1).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace units {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// 32-byte vector and its 256-bit global load (read-once, no L1 allocation)
+// and store.
+struct alignas(32) Vec32 {
+    uint32_t w[8];
+};
+
+__device__ __forceinline__ Vec32 ld32_once(const Vec32* p)
+{
+    Vec32 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                   "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st32(Vec32* p, const Vec32& v)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                 "r"(v.w[7])
+                 : "memory");
+}
+
+constexpr int kUnitVec32 = 32;      // BF16 unit: 32 vectors x 16 channels = 512 channels
+constexpr int kU32Fp8 = 2;          // FP8 unit: 2 vectors per lane
+constexpr int kUnitVec32Fp8 = 32 * kU32Fp8;  // 64 vectors = 1024 channels = 8 blocks
+
+// Scale of (row, block): row-major [row][nblk] when ld == 0, else MN-major
+// [block][ld] (each block's scales contiguous over rows, for GEMMs that read
+// scales along M).
+__device__ __forceinline__ int64_t scale_index(int64_t row, int64_t blk, int nblk, int64_t ld)
+{
+    return ld == 0 ? row * nblk + blk : blk * ld + row;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d)
+{
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+}
+
+// BF16: the lane's 32-byte vector of the unit is read once and written to
+// each of the k destination rows; consecutive lanes write consecutive bytes.
+__device__ __forceinline__ void bf16_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
+                                          int d, int k, Vec32* __restrict__ recv)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t v = unit * kUnitVec32 + lane;
+    Vec32 val;
+    if (v < vpr)
+        val = ld32_once(xs + v);
+    for (int j = 0; j < k; ++j) {
+        const int dj = __shfl_sync(kFull, d, j);
+        if (dj >= 0 && v < vpr)
+            st32(recv + (int64_t)dj * vpr + v, val);
+    }
+}
+
+// FP8: lane vector i of the unit covers channels 16 v .. 16 v + 15 with
+// v = unit * 64 + 32 i + lane, so each 128-channel block is one group of 8
+// lanes (xor 4, 2, 1 reduction) and the unit's blocks 4i .. 4i + 3 sit in
+// lane groups 0-3 of vector i.  Each lane writes its 16 codes as one 16-byte
+// store; the unit's 8 scales are gathered into lanes 0-7 and written as one
+// 32-byte run per destination row (row-major scales).  xs: the token row in
+// 32-byte vectors, vpr = H / 16.
+__device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
+                                         int d, int k, int H, uint8_t* __restrict__ recv_q,
+                                         float* __restrict__ recv_scales, int64_t scales_ld)
+{
+    const int lane = threadIdx.x & 31;
+    const int nblk = H / 128;
+    const int64_t v0 = unit * kUnitVec32Fp8 + lane;
+    Vec32 a[kU32Fp8];
+#pragma unroll
+    for (int i = 0; i < kU32Fp8; ++i) {
+        if (v0 + 32 * i < vpr) {
+            a[i] = ld32_once(xs + v0 + 32 * i);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) a[i].w[c] = 0u;
+        }
+    }
+    uint4 q[kU32Fp8];
+    float sc[kU32Fp8];
+#pragma unroll
+    for (int i = 0; i < kU32Fp8; ++i) {
+        float f[16];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            f[2 * c] = bf16_lo(a[i].w[c]);
+            f[2 * c + 1] = bf16_hi(a[i].w[c]);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m = fmaxf(m, fabsf(f[c]));
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+        if (m == 0.0f) {
+            sc[i] = 0.0f;
+            q[i] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            const float s = __fdiv_rn(m, 448.0f);
+            sc[i] = s;
+            q[i].x = e4m3x4(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s), __fdiv_rn(f[2], s),
+                            __fdiv_rn(f[3], s));
+            q[i].y = e4m3x4(__fdiv_rn(f[4], s), __fdiv_rn(f[5], s), __fdiv_rn(f[6], s),
+                            __fdiv_rn(f[7], s));
+            q[i].z = e4m3x4(__fdiv_rn(f[8], s), __fdiv_rn(f[9], s), __fdiv_rn(f[10], s),
+                            __fdiv_rn(f[11], s));
+            q[i].w = e4m3x4(__fdiv_rn(f[12], s), __fdiv_rn(f[13], s), __fdiv_rn(f[14], s),
+                            __fdiv_rn(f[15], s));
+        }
+    }
+    // lane L < 8 takes the scale of block L of the unit: vector L / 4, lane
+    // group L % 4 (leader lane 8 (L % 4))
+    float my_scale = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kU32Fp8; ++i) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const float sv = __shfl_sync(kFull, sc[i], 8 * g);
+            if (lane == 4 * i + g)
+                my_scale = sv;
+        }
+    }
+    const int64_t blk = unit * (4 * kU32Fp8) + lane;
+    const bool sc_ok = lane < 4 * kU32Fp8 && blk < nblk;
+    for (int j = 0; j < k; ++j) {
+        const int dj = __shfl_sync(kFull, d, j);
+        if (dj < 0)
+            continue;
+        uint4* dq = reinterpret_cast<uint4*>(recv_q + (int64_t)dj * H);
+#pragma unroll
+        for (int i = 0; i < kU32Fp8; ++i)
+            if (v0 + 32 * i < vpr)
+                dq[v0 + 32 * i] = q[i];
+        if (sc_ok)
+            recv_scales[scale_index(dj, blk, nblk, scales_ld)] = my_scale;
+    }
+}
+
+}  // namespace units
+}  // namespace ep

@@ -88,6 +88,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
 // grid barrier words at h.err[1..2], zero-initialised).
 cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s,
                           bool allow_fused = true);
+// Layout + dispatch in one launch for small batches (fused_layout_dispatch_fits);
+// the dispatch side needs the 256-bit path (H % 16 == 0, x / recv_x 32-byte aligned).
+bool fused_layout_dispatch_fits(const Handle& h, int T);
+cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int T, const void* x,
+                                   int H, bool fp8, void* recv_x, float* recv_scales,
+                                   int64_t scales_ld, int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* recv_x,
                                  int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,

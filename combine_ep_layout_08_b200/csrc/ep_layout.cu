@@ -36,6 +36,7 @@
 // memory.
 #include <algorithm>
 
+#include "ep_dispatch_units.cuh"
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -445,6 +446,24 @@ __host__ __device__ inline size_t small_smem_words(int E, int R)
     return (size_t)E + E + 32 * (size_t)E + E + 1 + 32 + R + kSmallEntries;
 }
 
+// The dispatch half of the fused small-batch kernel (layout + dispatch in
+// one launch): what ep_dispatch would be given.
+struct FusedDispatch {
+    const void* x;
+    int H;
+    int fp8;             // 0: BF16 copy; 1: FP8 e4m3 1x128
+    void* recv_x;
+    float* recv_scales;
+    int64_t scales_ld;   // FP8: 0 row-major scales, else MN-major leading dimension
+    int64_t cap_rows;
+};
+
+// kFused = false: the layout alone, one CTA.  kFused = true: every CTA of
+// the grid computes the same layout in its shared memory (deterministic, so
+// identical); CTA 0 publishes it; the pad rows of recv_src are spread over
+// the CTAs; then every warp of the grid dispatches (token, unit) pieces with
+// the positions in its own shared memory -- no grid-wide wait.
+template <bool kFused>
 __global__ void __launch_bounds__(kSmallThreads)
 layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
                     uint64_t rank_magic, int block_m, int32_t* __restrict__ cnt_g,
@@ -452,12 +471,13 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
                     int32_t* __restrict__ tokens_per_rank_g,
                     int32_t* __restrict__ rows_per_rank_g, int32_t* __restrict__ total_rows_g,
                     uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
-                    int32_t* __restrict__ recv_src, int32_t* err)
+                    int32_t* __restrict__ recv_src, int32_t* err, FusedDispatch fd)
 {
     extern __shared__ int32_t smem[];
     pdl_wait();
     pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5;
+    const bool leader = !kFused || blockIdx.x == 0;
     const int nent = T * k;
     const int rounds = (nent + kSmallThreads - 1) / kSmallThreads;
     int32_t* cnt = smem;
@@ -466,11 +486,11 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     int32_t* off = wcnt + 32 * (size_t)E;
     int32_t* wsum = off + E + 1;
     int32_t* rhist = wsum + 32;
-    int32_t* erank = rhist + R;
+    int32_t* erank = rhist + R;                  // entry ranks, then (fused) positions
 
     for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
     for (int r = tid; r < R; r += kSmallThreads) rhist[r] = 0;
-    {
+    if (leader) {
         const int64_t bytes = (int64_t)T * R;
         uint8_t* itr = is_token_in_rank;
         if (((uintptr_t)itr & 15u) == 0) {
@@ -499,48 +519,57 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             const int rk = (int)(((uint64_t)e * rank_magic) >> 32);
             atomicAdd(&cnt[e], 1);
             erank[f] = rk;
-            is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
+            if (leader)
+                is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
         } else if (e == -1) {
             erank[f] = -1;
         }
     }
-    if (__syncthreads_or(bad) && tid == 0)
+    if (__syncthreads_or(bad) && tid == 0 && leader)
         atomicOr(err, kErrBadIndex);
+    if (leader) {
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
-        const int f = q * kSmallThreads + tid;
-        if (e_r[q] >= 0) {
-            const int rk = erank[f];
-            const int t = f / k, j = f - t * k;
-            bool first = true;
-            for (int jj = 0; jj < j; ++jj) first &= (erank[t * k + jj] != rk);
-            if (first)
-                atomicAdd(&rhist[rk], 1);
+        for (int q = 0; q < kSmallRounds; ++q) {
+            const int f = q * kSmallThreads + tid;
+            if (e_r[q] >= 0) {
+                const int rk = erank[f];
+                const int t = f / k, j = f - t * k;
+                bool first = true;
+                for (int jj = 0; jj < j; ++jj) first &= (erank[t * k + jj] != rk);
+                if (first)
+                    atomicAdd(&rhist[rk], 1);
+            }
         }
     }
     __syncthreads();
 
     // offsets and bookkeeping
     scan_padded(cnt, E, block_m, off, wsum);
-    for (int e = tid; e < E; e += kSmallThreads) {
-        cnt_g[e] = cnt[e];
-        run[e] = off[e];
+    for (int e = tid; e < E; e += kSmallThreads) run[e] = off[e];
+    if (leader) {
+        for (int e = tid; e < E; e += kSmallThreads) cnt_g[e] = cnt[e];
+        for (int e = tid; e <= E; e += kSmallThreads) expert_off_g[e] = off[e];
+        for (int r = tid; r <= R; r += kSmallThreads) rank_off_g[r] = off[r * epr];
+        for (int r = tid; r < R; r += kSmallThreads) {
+            int32_t s = 0;
+            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
+            rows_per_rank_g[r] = s;
+            tokens_per_rank_g[r] = rhist[r];
+        }
+        if (tid == 0)
+            *total_rows_g = off[E];
     }
-    for (int e = tid; e <= E; e += kSmallThreads) expert_off_g[e] = off[e];
-    for (int r = tid; r <= R; r += kSmallThreads) rank_off_g[r] = off[r * epr];
-    for (int r = tid; r < R; r += kSmallThreads) {
-        int32_t s = 0;
-        for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
-        rows_per_rank_g[r] = s;
-        tokens_per_rank_g[r] = rhist[r];
-    }
-    if (tid == 0)
-        *total_rows_g = off[E];
+    // pad rows: one warp per expert, experts spread over the CTAs
     const bool vec = ((uintptr_t)recv_src & 15u) == 0;
-    for (int e = warp; e < E; e += kSmallThreads / 32) fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
+    const int G = kFused ? (int)gridDim.x : 1;
+    const int cta = kFused ? (int)blockIdx.x : 0;
+    for (int64_t e = cta + (int64_t)warp * G; e < E; e += (int64_t)G * (kSmallThreads / 32))
+        fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
     // pass B
     const unsigned lt = lanemask_lt();
+    int tpe = 1;  // threads per expert in the warp-count scan: a power of two, <= 32
+    while (tpe < 32 && 2 * tpe * E <= kSmallThreads) tpe *= 2;
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
         if (q < rounds) {
@@ -551,24 +580,71 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             if (e >= 0 && (peers & lt) == 0)
                 wcnt[warp * E + e] = __popc(peers);
             __syncthreads();
-            for (int x = tid; x < E; x += kSmallThreads) {
-                int32_t acc = run[x];
-                for (int w = 0; w < 32; ++w) {
-                    const int32_t c = wcnt[w * E + x];
-                    wcnt[w * E + x] = acc;
-                    acc += c;
+            // per expert, exclusive scan of the 32 warp counts on top of run:
+            // tpe threads per expert (consecutive lanes), each over 32 / tpe warps
+            {
+                const int x = tid / tpe, p = tid - x * tpe, wpp = 32 / tpe;
+                int32_t part = 0;
+                if (x < E)
+                    for (int w = p * wpp; w < (p + 1) * wpp; ++w) part += wcnt[w * E + x];
+                int32_t incl = part;
+                for (int o = 1; o < tpe; o <<= 1) {
+                    const int32_t u = __shfl_up_sync(kFull, incl, o, tpe);
+                    if (p >= o)
+                        incl += u;
                 }
-                run[x] = acc;
+                if (x < E) {
+                    int32_t acc = run[x] + incl - part;
+                    for (int w = p * wpp; w < (p + 1) * wpp; ++w) {
+                        const int32_t c = wcnt[w * E + x];
+                        wcnt[w * E + x] = acc;
+                        acc += c;
+                    }
+                }
+                __syncthreads();
+                if (x < E && p == tpe - 1)
+                    run[x] = run[x] + incl;
             }
             __syncthreads();
             const int f = q * kSmallThreads + tid;
             if (f < nent) {
                 const int pos = e >= 0 ? wcnt[warp * E + e] + __popc(peers & lt) : -1;
-                dst_row[f] = pos;
-                if (pos >= 0)
-                    recv_src[pos] = f / k;
+                if (kFused)
+                    erank[f] = pos;  // every entry's rank was consumed in pass A
+                if (leader) {
+                    dst_row[f] = pos;
+                    if (pos >= 0)
+                        recv_src[pos] = f / k;
+                }
             }
         }
+    }
+    if (!kFused)
+        return;
+
+    // dispatch: (token, unit) pieces over all warps of the grid
+    __syncthreads();
+    const int lane = tid & 31;
+    const int64_t gw = (int64_t)blockIdx.x * (kSmallThreads / 32) + warp;
+    const int64_t nw = (int64_t)gridDim.x * (kSmallThreads / 32);
+    const int64_t vpr = fd.H / 16;
+    const int64_t uvec = fd.fp8 ? units::kUnitVec32Fp8 : units::kUnitVec32;
+    const int64_t upr = (vpr + uvec - 1) / uvec;
+    const units::Vec32* x = static_cast<const units::Vec32*>(fd.x);
+    for (int64_t u = gw; u < (int64_t)T * upr; u += nw) {
+        const int64_t t = u / upr;
+        int d = lane < k ? erank[t * k + lane] : -1;
+        if (d >= fd.cap_rows) {
+            if (leader)
+                atomicOr(err, kErrDispatchCap);
+            d = -1;
+        }
+        if (fd.fp8)
+            units::fp8_unit(x + t * vpr, vpr, u - t * upr, d, k, fd.H,
+                            static_cast<uint8_t*>(fd.recv_x), fd.recv_scales, fd.scales_ld);
+        else
+            units::bf16_unit(x + t * vpr, vpr, u - t * upr, d, k,
+                             static_cast<units::Vec32*>(fd.recv_x));
     }
 }
 
@@ -921,12 +997,12 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
     if ((int64_t)T * k <= kSmallEntries && E <= kSmallMaxE &&
         (int64_t)T * R <= kSmallMaxRankBytes) {
         const size_t smem = sizeof(int32_t) * small_smem_words(E, R);
-        if ((rc = set_smem((const void*)layout_small_kernel, smem)) != cudaSuccess)
+        if ((rc = set_smem((const void*)layout_small_kernel<false>, smem)) != cudaSuccess)
             return rc;
-        return launch_pdl(layout_small_kernel, 1, kSmallThreads, smem, s, topk_idx, T, k, E, R,
-                          epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off, h.rank_off,
-                          h.tokens_per_rank, h.rows_per_rank, h.total_rows, h.is_token_in_rank,
-                          h.dst_row, h.recv_src, h.err);
+        return launch_pdl(layout_small_kernel<false>, 1, kSmallThreads, smem, s, topk_idx, T, k,
+                          E, R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off,
+                          h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
+                          h.is_token_in_rank, h.dst_row, h.recv_src, h.err, FusedDispatch{});
     }
 
     if (allow_fused && nchunks > 0) {
@@ -964,6 +1040,35 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
     return launch_pdl(layout_assign_kernel, g3, 32 * w3, smem3, s, topk_idx, T, k, E, R, epr,
                       rank_magic_for(epr), h.block_m, nchunks, h.chunk_counts, h.cnt, h.expert_off, h.rank_off,
                       h.rows_per_rank, h.total_rows, h.dst_row, h.recv_src);
+}
+
+bool fused_layout_dispatch_fits(const Handle& h, int T)
+{
+    return (int64_t)T * h.k <= kSmallEntries && h.E <= kSmallMaxE &&
+           (int64_t)T * h.R <= kSmallMaxRankBytes;
+}
+
+cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int T, const void* x,
+                                   int H, bool fp8, void* recv_x, float* recv_scales,
+                                   int64_t scales_ld, int64_t cap_rows, cudaStream_t s)
+{
+    const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
+    const size_t smem = sizeof(int32_t) * small_smem_words(E, R);
+    cudaError_t rc;
+    if ((rc = set_smem((const void*)layout_small_kernel<true>, smem)) != cudaSuccess)
+        return rc;
+    int dev = 0, sms = 0;
+    if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+        (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return rc;
+    // one CTA per SM: the layout is replicated (cheap at these sizes) so that
+    // the dispatch -- FP8 division and row stores -- spreads over the GPU
+    const unsigned grid = (unsigned)std::max(1, sms);
+    FusedDispatch fd{x, H, fp8 ? 1 : 0, recv_x, recv_scales, scales_ld, cap_rows};
+    return launch_pdl(layout_small_kernel<true>, grid, kSmallThreads, smem, s, topk_idx, T, k, E,
+                      R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off, h.rank_off,
+                      h.tokens_per_rank, h.rows_per_rank, h.total_rows, h.is_token_in_rank,
+                      h.dst_row, h.recv_src, h.err, fd);
 }
 
 }  // namespace ep

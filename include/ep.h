@@ -146,6 +146,22 @@ void ep_handle_destroy(ep_handle_t h);
  * [-1, E) sets EP_ERR_BAD_INDEX in the sticky error word and is treated as -1. */
 ep_status_t ep_layout(ep_handle_t h, const int64_t* topk_idx, int T, void* stream);
 
+/* Layout followed by dispatch, the low-latency path for decode-sized batches
+ * (the pages' low-latency mode serves decode and small batches, where launch
+ * latency matters most: "DeepEP是什麼？…", section 高吞吐與低延遲工作負載).
+ * Same arguments, results and errors as ep_layout(h, topk_idx, T, stream)
+ * followed by ep_dispatch(h, x, H, fmt, recv_x, recv_scales,
+ * recv_capacity_rows, stream).  When the batch is small (T*k <= 4096,
+ * E <= 1024, T*R <= 65536) and rows take 32-byte vectors (H % 16 == 0; x,
+ * and for BF16 recv_x, 32-byte aligned), both run in ONE launch: every CTA
+ * computes the same layout in its shared memory, CTA 0 publishes it, and all
+ * CTAs dispatch from their own copy -- no grid-wide wait.  Otherwise the two
+ * launches of the separate calls run.  All arguments are checked before
+ * anything is enqueued. */
+ep_status_t ep_layout_dispatch(ep_handle_t h, const int64_t* topk_idx, int T, const void* x, int H,
+                               ep_fmt_t fmt, void* recv_x, float* recv_scales,
+                               int64_t recv_capacity_rows, void* stream);
+
 /* Device pointer of a layout view inside the workspace (host; no CUDA call);
  * *count (if not NULL) receives its number of elements for the last layout
  * (P for EP_VIEW_RECV_SRC is only known on the device, so its count is the
