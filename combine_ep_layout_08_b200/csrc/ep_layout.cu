@@ -26,8 +26,9 @@
 // phases in one cooperative launch over 64-token tiles, its CTAs separated by
 // two grid barriers; the three kernels remain for shapes whose tile counts do
 // not fit in shared memory and for the static-scratch entry point.
-// Small batches (T k <= 4096, E <= 1024) run in one CTA of 1024 threads with
-// one entry per thread (layout_small_kernel).
+// Small batches (T k <= 4096, E <= 1024, shared memory permitting) run with
+// one entry per thread in CTAs of 1024 threads that each compute the whole
+// layout (layout_small_kernel).
 //
 // The work is latency-bound (at 8K tokens the layout reads 0.5 MB), so each
 // kernel issues all of its global loads before it uses any of them, and every
@@ -423,27 +424,50 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
     chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
 }
 
-// Small batches (T k <= kSmallEntries, E <= kSmallMaxE): one CTA of 1024
-// threads, one entry per thread per round of 1024 entries (at most
-// kSmallRounds rounds, the entries kept in registers between passes).
-//   pass A  shared-memory histogram, entry ranks, is_token_in_rank bytes (rows
-//           zeroed first; an entry sets its byte), tokens per rank (an entry
-//           counts if no earlier slot of its token has the same rank);
-//   offsets block scan of the padded counts;
-//   pass B  per round: __match_any_sync ranks inside each warp, per-warp
-//           counts in shared memory, a scan over the 32 warps per expert on
-//           top of the running per-expert base, then the positions.
-// Shared memory (words): cnt[E], run[E], wcnt[32][E], off[E+1], wsum[32],
-// rank_hist[R], erank[kSmallEntries].
+// Small batches (T k <= kSmallEntries, E <= kSmallMaxE): CTAs of 1024
+// threads take the entries 1024 at a time (a round, at most kSmallRounds),
+// one per thread, kept in registers.  Entry f of round q belongs to virtual
+// warp v = f / 32 = 32 q + warp.  Every CTA of the grid computes the whole
+// layout in its own shared memory (deterministic, so all agree) and CTA 0
+// writes it out; the pad rows of recv_src -- most of the bytes at decode
+// sizes -- are spread over the CTAs, since one SM alone stores only some
+// tens of GB/s.  Five block barriers:
+//   1  topk_idx loaded (issued before anything else), the count table, rank
+//      counters and is_token_in_rank zeroed;
+//   2  per round, __match_any_sync groups equal experts inside the warp; the
+//      first lane of a group stores the group size in vtab[e][v]; entry
+//      ranks, is_token_in_rank bytes, rows per rank (one shared atomic per
+//      group of equal ranks);
+//   3  per expert, tpe threads scan vtab[e][*] over the virtual warps in place
+//      (exclusive), the last of them holding cnt[e]; the padded counts are
+//      scanned across the warp; tokens per rank (an entry counts when no
+//      earlier slot of its token has the same rank);
+//   4  each warp scans the 32 warp totals itself and stores off[e];
+//   5  position = off[e] + vtab[e][v] + rank among the equal lanes.
+// Shared memory: vtab uint16 [E][nv] (nv = 32 rounds), then 32-bit words
+// cnt[E], off[E+1], wsum[32], rhist[R], rrows[R], erank[1024 rounds].
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallRounds = 4;
 constexpr int kSmallEntries = kSmallThreads * kSmallRounds;
 constexpr int kSmallMaxE = 1024;
 constexpr int64_t kSmallMaxRankBytes = 65536;  // T x R bytes of is_token_in_rank
 
-__host__ __device__ inline size_t small_smem_words(int E, int R)
+__host__ __device__ inline int small_rounds(int64_t nent)
 {
-    return (size_t)E + E + 32 * (size_t)E + E + 1 + 32 + R + kSmallEntries;
+    return nent <= kSmallThreads ? 1 : (int)((nent + kSmallThreads - 1) / kSmallThreads);
+}
+
+__host__ __device__ inline size_t small_smem_bytes(int E, int R, int rounds)
+{
+    return 2 * (size_t)E * 32 * rounds +
+           sizeof(int32_t) * ((size_t)E + E + 1 + 32 + 2 * (size_t)R + (size_t)kSmallThreads * rounds);
+}
+
+bool small_fits(int64_t T, int k, int E, int R)
+{
+    const int64_t nent = T * k;
+    return nent <= kSmallEntries && E <= kSmallMaxE && T * R <= kSmallMaxRankBytes &&
+           small_smem_bytes(E, R, small_rounds(nent)) <= kSmemBudget;
 }
 
 // The dispatch half of the fused small-batch kernel (layout + dispatch in
@@ -458,11 +482,33 @@ struct FusedDispatch {
     int64_t cap_rows;
 };
 
-// kFused = false: the layout alone, one CTA.  kFused = true: every CTA of
-// the grid computes the same layout in its shared memory (deterministic, so
-// identical); CTA 0 publishes it; the pad rows of recv_src are spread over
-// the CTAs; then every warp of the grid dispatches (token, unit) pieces with
-// the positions in its own shared memory -- no grid-wide wait.
+__device__ __forceinline__ int32_t sum_u16x8(int4 v)
+{
+    const uint32_t w[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
+    int32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += (int32_t)(w[i] & 0xffffu) + (int32_t)(w[i] >> 16);
+    return s;
+}
+
+// Exclusive prefix of 8 packed uint16 counts starting at acc; returns the
+// running sum after them.
+__device__ __forceinline__ int32_t exscan_u16x8(int4& v, int32_t acc)
+{
+    uint32_t w[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int32_t lo = (int32_t)(w[i] & 0xffffu), hi = (int32_t)(w[i] >> 16);
+        w[i] = (uint32_t)acc | ((uint32_t)(acc + lo) << 16);
+        acc += lo + hi;
+    }
+    v = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
+    return acc;
+}
+
+// kFused = false: the layout alone.  kFused = true: then every warp of the
+// grid dispatches (token, unit) pieces with the positions in its own shared
+// memory -- no grid-wide wait.
 template <bool kFused>
 __global__ void __launch_bounds__(kSmallThreads)
 layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
@@ -473,23 +519,38 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
                     uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
                     int32_t* __restrict__ recv_src, int32_t* err, FusedDispatch fd)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) unsigned char small_smem[];
     pdl_wait();
     pdl_trigger();
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const bool leader = !kFused || blockIdx.x == 0;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool leader = blockIdx.x == 0;
     const int nent = T * k;
-    const int rounds = (nent + kSmallThreads - 1) / kSmallThreads;
-    int32_t* cnt = smem;
-    int32_t* run = cnt + E;
-    int32_t* wcnt = run + E;                     // [32][E]
-    int32_t* off = wcnt + 32 * (size_t)E;
+    const int rounds = small_rounds(nent);
+    const int nv = 32 * rounds;
+    uint16_t* vtab = reinterpret_cast<uint16_t*>(small_smem);  // [E][nv]
+    int32_t* cnt = reinterpret_cast<int32_t*>(small_smem + 2 * (size_t)E * nv);
+    int32_t* off = cnt + E;
     int32_t* wsum = off + E + 1;
     int32_t* rhist = wsum + 32;
-    int32_t* erank = rhist + R;                  // entry ranks, then (fused) positions
+    int32_t* rrows = rhist + R;
+    int32_t* erank = rrows + R;  // entry ranks, then (fused) positions
 
-    for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
-    for (int r = tid; r < R; r += kSmallThreads) rhist[r] = 0;
+    // 1: loads first; zeroing while they are in flight
+    int64_t raw[kSmallRounds];
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        const int f = q * kSmallThreads + tid;
+        raw[q] = (q < rounds && f < nent) ? topk_idx[f] : -1;
+    }
+    {
+        int4* z = reinterpret_cast<int4*>(vtab);
+        const int n16 = (int)(((size_t)E * nv) / 8);  // E nv halfwords, a multiple of 32
+        for (int i = tid; i < n16; i += kSmallThreads) z[i] = make_int4(0, 0, 0, 0);
+    }
+    for (int r = tid; r < R; r += kSmallThreads) {
+        rhist[r] = 0;
+        rrows[r] = 0;
+    }
     if (leader) {
         const int64_t bytes = (int64_t)T * R;
         uint8_t* itr = is_token_in_rank;
@@ -501,37 +562,82 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             for (int64_t i = tid; i < bytes; i += kSmallThreads) itr[i] = 0;
         }
     }
-    __syncthreads();
-
-    // pass A
     int e_r[kSmallRounds];
     int bad = 0;
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
-        const int f = q * kSmallThreads + tid;
-        e_r[q] = (q < rounds && f < nent) ? to_expert(topk_idx[f], E, bad) : -2;
-    }
-#pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
-        const int f = q * kSmallThreads + tid;
-        const int e = e_r[q];
-        if (e >= 0) {
-            const int rk = (int)(((uint64_t)e * rank_magic) >> 32);
-            atomicAdd(&cnt[e], 1);
-            erank[f] = rk;
-            if (leader)
-                is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
-        } else if (e == -1) {
-            erank[f] = -1;
-        }
-    }
+    for (int q = 0; q < kSmallRounds; ++q) e_r[q] = to_expert(raw[q], E, bad);
     if (__syncthreads_or(bad) && tid == 0 && leader)
         atomicOr(err, kErrBadIndex);
+
+    // 2: equal experts inside each warp
+    const unsigned lt = lanemask_lt();
+    int rin[kSmallRounds];
+#pragma unroll
+    for (int q = 0; q < kSmallRounds; ++q) {
+        rin[q] = 0;
+        if (q < rounds) {
+            const int f = q * kSmallThreads + tid;
+            const int e = e_r[q];
+            const unsigned peers = __match_any_sync(kFull, e);
+            rin[q] = __popc(peers & lt);
+            const int rk = e >= 0 ? (int)(((uint64_t)e * rank_magic) >> 32) : -1;
+            if (e >= 0 && rin[q] == 0)
+                vtab[(size_t)e * nv + q * 32 + warp] = (uint16_t)__popc(peers);
+            const unsigned rpeers = __match_any_sync(kFull, rk);
+            if (rk >= 0 && (rpeers & lt) == 0)
+                atomicAdd(&rrows[rk], __popc(rpeers));
+            if (f < nent) {
+                erank[f] = rk;
+                if (leader && rk >= 0)
+                    is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
+            }
+        }
+    }
+    __syncthreads();
+
+    // 3: per expert, tpe consecutive threads over nv / tpe virtual warps each
+    int tpe = 1;
+    while (2 * tpe * E <= kSmallThreads && (nv / (2 * tpe)) % 8 == 0) tpe *= 2;
+    const int x = tid / tpe, p = tid - x * tpe;
+    const int chunk = nv / tpe;  // a multiple of 8 halfwords: whole int4s
+    int32_t padded = 0;
+    {
+        int4* row = reinterpret_cast<int4*>(vtab + (size_t)x * nv + p * chunk);
+        int32_t part = 0;
+        if (x < E)
+            for (int i = 0; i < chunk / 8; ++i) part += sum_u16x8(row[i]);
+        int32_t incl = part;
+        for (int o = 1; o < tpe; o <<= 1) {
+            const int32_t u = __shfl_up_sync(kFull, incl, o, tpe);
+            if (p >= o)
+                incl += u;
+        }
+        if (x < E) {
+            int32_t acc = incl - part;
+            for (int i = 0; i < chunk / 8; ++i) {
+                int4 v = row[i];
+                acc = exscan_u16x8(v, acc);
+                row[i] = v;
+            }
+            if (p == tpe - 1) {
+                cnt[x] = incl;
+                padded = pad_up(incl, block_m);
+            }
+        }
+    }
+    int32_t pincl = padded;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(kFull, pincl, o);
+        if (lane >= o)
+            pincl += u;
+    }
+    if (lane == 31)
+        wsum[warp] = pincl;
     if (leader) {
 #pragma unroll
         for (int q = 0; q < kSmallRounds; ++q) {
             const int f = q * kSmallThreads + tid;
-            if (e_r[q] >= 0) {
+            if (q < rounds && f < nent && e_r[q] >= 0) {
                 const int rk = erank[f];
                 const int t = f / k, j = f - t * k;
                 bool first = true;
@@ -543,107 +649,81 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     }
     __syncthreads();
 
-    // offsets and bookkeeping
-    scan_padded(cnt, E, block_m, off, wsum);
-    for (int e = tid; e < E; e += kSmallThreads) run[e] = off[e];
+    // 4: expert offsets
+    {
+        const int32_t v = wsum[lane];
+        int32_t inc = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o)
+                inc += u;
+        }
+        const int32_t base = __shfl_sync(kFull, inc - v, warp);
+        if (x < E && p == tpe - 1) {
+            off[x] = base + pincl - padded;
+            if (x == E - 1)
+                off[E] = base + pincl;
+        }
+    }
+    __syncthreads();
+
+    // 5: outputs (CTA 0), pad rows (all CTAs), positions
     if (leader) {
         for (int e = tid; e < E; e += kSmallThreads) cnt_g[e] = cnt[e];
         for (int e = tid; e <= E; e += kSmallThreads) expert_off_g[e] = off[e];
         for (int r = tid; r <= R; r += kSmallThreads) rank_off_g[r] = off[r * epr];
         for (int r = tid; r < R; r += kSmallThreads) {
-            int32_t s = 0;
-            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
-            rows_per_rank_g[r] = s;
+            rows_per_rank_g[r] = rrows[r];
             tokens_per_rank_g[r] = rhist[r];
         }
         if (tid == 0)
             *total_rows_g = off[E];
     }
-    // pad rows: one warp per expert, experts spread over the CTAs
-    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
-    const int G = kFused ? (int)gridDim.x : 1;
-    const int cta = kFused ? (int)blockIdx.x : 0;
-    for (int64_t e = cta + (int64_t)warp * G; e < E; e += (int64_t)G * (kSmallThreads / 32))
-        fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
-
-    // pass B
-    const unsigned lt = lanemask_lt();
-    int tpe = 1;  // threads per expert in the warp-count scan: a power of two, <= 32
-    while (tpe < 32 && 2 * tpe * E <= kSmallThreads) tpe *= 2;
+    {
+        const bool vec = ((uintptr_t)recv_src & 15u) == 0;
+        const int G = (int)gridDim.x;
+        for (int64_t e = blockIdx.x + (int64_t)warp * G; e < E; e += (int64_t)G * (kSmallThreads / 32))
+            fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
+    }
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
-        if (q < rounds) {
-            for (int i = tid; i < 32 * E; i += kSmallThreads) wcnt[i] = 0;
-            __syncthreads();
+        const int f = q * kSmallThreads + tid;
+        if (q < rounds && f < nent) {
             const int e = e_r[q];
-            const unsigned peers = __match_any_sync(kFull, e);
-            if (e >= 0 && (peers & lt) == 0)
-                wcnt[warp * E + e] = __popc(peers);
-            __syncthreads();
-            // per expert, exclusive scan of the 32 warp counts on top of run:
-            // tpe threads per expert (consecutive lanes), each over 32 / tpe warps
-            {
-                const int x = tid / tpe, p = tid - x * tpe, wpp = 32 / tpe;
-                int32_t part = 0;
-                if (x < E)
-                    for (int w = p * wpp; w < (p + 1) * wpp; ++w) part += wcnt[w * E + x];
-                int32_t incl = part;
-                for (int o = 1; o < tpe; o <<= 1) {
-                    const int32_t u = __shfl_up_sync(kFull, incl, o, tpe);
-                    if (p >= o)
-                        incl += u;
-                }
-                if (x < E) {
-                    int32_t acc = run[x] + incl - part;
-                    for (int w = p * wpp; w < (p + 1) * wpp; ++w) {
-                        const int32_t c = wcnt[w * E + x];
-                        wcnt[w * E + x] = acc;
-                        acc += c;
-                    }
-                }
-                __syncthreads();
-                if (x < E && p == tpe - 1)
-                    run[x] = run[x] + incl;
-            }
-            __syncthreads();
-            const int f = q * kSmallThreads + tid;
-            if (f < nent) {
-                const int pos = e >= 0 ? wcnt[warp * E + e] + __popc(peers & lt) : -1;
-                if (kFused)
-                    erank[f] = pos;  // every entry's rank was consumed in pass A
-                if (leader) {
-                    dst_row[f] = pos;
-                    if (pos >= 0)
-                        recv_src[pos] = f / k;
-                }
+            const int pos = e >= 0 ? off[e] + vtab[(size_t)e * nv + q * 32 + warp] + rin[q] : -1;
+            if (kFused)
+                erank[f] = pos;  // the ranks were last read before barrier 3
+            if (leader) {
+                dst_row[f] = pos;
+                if (pos >= 0)
+                    recv_src[pos] = f / k;
             }
         }
     }
     if (!kFused)
         return;
 
-    // dispatch: (token, unit) pieces over all warps of the grid
+    // dispatch: (token, unit) pieces dealt to the CTAs in turn, so that the
+    // row stores spread over every SM
     __syncthreads();
-    const int lane = tid & 31;
-    const int64_t gw = (int64_t)blockIdx.x * (kSmallThreads / 32) + warp;
-    const int64_t nw = (int64_t)gridDim.x * (kSmallThreads / 32);
+    const int64_t G = gridDim.x;
     const int64_t vpr = fd.H / 16;
     const int64_t uvec = fd.fp8 ? units::kUnitVec32Fp8 : units::kUnitVec32;
     const int64_t upr = (vpr + uvec - 1) / uvec;
-    const units::Vec32* x = static_cast<const units::Vec32*>(fd.x);
-    for (int64_t u = gw; u < (int64_t)T * upr; u += nw) {
+    const units::Vec32* xv = static_cast<const units::Vec32*>(fd.x);
+    for (int64_t u = (int64_t)warp * G + blockIdx.x; u < (int64_t)T * upr;
+         u += G * (kSmallThreads / 32)) {
         const int64_t t = u / upr;
         int d = lane < k ? erank[t * k + lane] : -1;
         if (d >= fd.cap_rows) {
-            if (leader)
-                atomicOr(err, kErrDispatchCap);
+            atomicOr(err, kErrDispatchCap);
             d = -1;
         }
         if (fd.fp8)
-            units::fp8_unit(x + t * vpr, vpr, u - t * upr, d, k, fd.H,
+            units::fp8_unit(xv + t * vpr, vpr, u - t * upr, d, k, fd.H,
                             static_cast<uint8_t*>(fd.recv_x), fd.recv_scales, fd.scales_ld);
         else
-            units::bf16_unit(x + t * vpr, vpr, u - t * upr, d, k,
+            units::bf16_unit(xv + t * vpr, vpr, u - t * upr, d, k,
                              static_cast<units::Vec32*>(fd.recv_x));
     }
 }
@@ -993,14 +1073,19 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
     const int64_t nchunks = ((int64_t)T + kChunkTokens - 1) / kChunkTokens;
     cudaError_t rc;
 
-    // one CTA, one entry per thread, when the batch is small
-    if ((int64_t)T * k <= kSmallEntries && E <= kSmallMaxE &&
-        (int64_t)T * R <= kSmallMaxRankBytes) {
-        const size_t smem = sizeof(int32_t) * small_smem_words(E, R);
+    // one entry per thread when the batch is small; one warp per expert's pad
+    // rows, so ceil(E / 32) CTAs, each computing the same layout
+    if (small_fits(T, k, E, R)) {
+        const size_t smem = small_smem_bytes(E, R, small_rounds((int64_t)T * k));
         if ((rc = set_smem((const void*)layout_small_kernel<false>, smem)) != cudaSuccess)
             return rc;
-        return launch_pdl(layout_small_kernel<false>, 1, kSmallThreads, smem, s, topk_idx, T, k,
-                          E, R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off,
+        int dev = 0, sms = 0;
+        if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+            (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return rc;
+        const unsigned grid = (unsigned)std::max(1, std::min(sms, (E + 31) / 32));
+        return launch_pdl(layout_small_kernel<false>, grid, kSmallThreads, smem, s, topk_idx, T,
+                          k, E, R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off,
                           h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
                           h.is_token_in_rank, h.dst_row, h.recv_src, h.err, FusedDispatch{});
     }
@@ -1044,8 +1129,7 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
 
 bool fused_layout_dispatch_fits(const Handle& h, int T)
 {
-    return (int64_t)T * h.k <= kSmallEntries && h.E <= kSmallMaxE &&
-           (int64_t)T * h.R <= kSmallMaxRankBytes;
+    return small_fits(T, h.k, h.E, h.R);
 }
 
 cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int T, const void* x,
@@ -1053,7 +1137,7 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
                                    int64_t scales_ld, int64_t cap_rows, cudaStream_t s)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
-    const size_t smem = sizeof(int32_t) * small_smem_words(E, R);
+    const size_t smem = small_smem_bytes(E, R, small_rounds((int64_t)T * k));
     cudaError_t rc;
     if ((rc = set_smem((const void*)layout_small_kernel<true>, smem)) != cudaSuccess)
         return rc;
