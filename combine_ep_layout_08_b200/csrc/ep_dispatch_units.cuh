@@ -1,8 +1,9 @@
 // ep_dispatch_units.cuh -- the per-unit bodies of the 256-bit dispatch
 // kernels, shared by ep_dispatch.cu and the fused layout + dispatch kernel.
 // A unit is one warp's share of one token row: BF16 512 channels (32 lanes x
-// one 32-byte vector), FP8 1024 channels (32 lanes x two 32-byte vectors = 8
-// blocks of 128).  `d` is this lane's destination row for slot j = lane
+// one 32-byte vector), FP8 512 kU channels (32 lanes x kU 32-byte vectors =
+// 4 kU blocks of 128; kU = 2 in the dispatch kernels, 1 in the fused
+// small-batch kernel, where more and shorter units spread the latency).  `d` is this lane's destination row for slot j = lane
 // (lanes >= k, unused slots and rows beyond the capacity pass -1).
 #pragma once
 
@@ -41,7 +42,7 @@ __device__ __forceinline__ void st32(Vec32* p, const Vec32& v)
 }
 
 constexpr int kUnitVec32 = 32;      // BF16 unit: 32 vectors x 16 channels = 512 channels
-constexpr int kU32Fp8 = 2;          // FP8 unit: 2 vectors per lane
+constexpr int kU32Fp8 = 2;          // FP8 unit of the dispatch kernels: 2 vectors per lane
 constexpr int kUnitVec32Fp8 = 32 * kU32Fp8;  // 64 vectors = 1024 channels = 8 blocks
 
 // Scale of (row, block): row-major [row][nblk] when ld == 0, else MN-major
@@ -80,22 +81,23 @@ __device__ __forceinline__ void bf16_unit(const Vec32* __restrict__ xs, int64_t 
 }
 
 // FP8: lane vector i of the unit covers channels 16 v .. 16 v + 15 with
-// v = unit * 64 + 32 i + lane, so each 128-channel block is one group of 8
+// v = unit * 32 kU + 32 i + lane, so each 128-channel block is one group of 8
 // lanes (xor 4, 2, 1 reduction) and the unit's blocks 4i .. 4i + 3 sit in
 // lane groups 0-3 of vector i.  Each lane writes its 16 codes as one 16-byte
-// store; the unit's 8 scales are gathered into lanes 0-7 and written as one
-// 32-byte run per destination row (row-major scales).  xs: the token row in
-// 32-byte vectors, vpr = H / 16.
+// store; the unit's 4 kU scales are gathered into lanes 0 .. 4 kU - 1 and
+// written as one run per destination row (row-major scales).  xs: the token
+// row in 32-byte vectors, vpr = H / 16.
+template <int kU = kU32Fp8>
 __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
                                          int d, int k, int H, uint8_t* __restrict__ recv_q,
                                          float* __restrict__ recv_scales, int64_t scales_ld)
 {
     const int lane = threadIdx.x & 31;
     const int nblk = H / 128;
-    const int64_t v0 = unit * kUnitVec32Fp8 + lane;
-    Vec32 a[kU32Fp8];
+    const int64_t v0 = unit * (32 * kU) + lane;
+    Vec32 a[kU];
 #pragma unroll
-    for (int i = 0; i < kU32Fp8; ++i) {
+    for (int i = 0; i < kU; ++i) {
         if (v0 + 32 * i < vpr) {
             a[i] = ld32_once(xs + v0 + 32 * i);
         } else {
@@ -103,10 +105,10 @@ __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t v
             for (int c = 0; c < 8; ++c) a[i].w[c] = 0u;
         }
     }
-    uint4 q[kU32Fp8];
-    float sc[kU32Fp8];
+    uint4 q[kU];
+    float sc[kU];
 #pragma unroll
-    for (int i = 0; i < kU32Fp8; ++i) {
+    for (int i = 0; i < kU; ++i) {
         float f[16];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -139,7 +141,7 @@ __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t v
     // group L % 4 (leader lane 8 (L % 4))
     float my_scale = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kU32Fp8; ++i) {
+    for (int i = 0; i < kU; ++i) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const float sv = __shfl_sync(kFull, sc[i], 8 * g);
@@ -147,15 +149,15 @@ __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t v
                 my_scale = sv;
         }
     }
-    const int64_t blk = unit * (4 * kU32Fp8) + lane;
-    const bool sc_ok = lane < 4 * kU32Fp8 && blk < nblk;
+    const int64_t blk = unit * (4 * kU) + lane;
+    const bool sc_ok = lane < 4 * kU && blk < nblk;
     for (int j = 0; j < k; ++j) {
         const int dj = __shfl_sync(kFull, d, j);
         if (dj < 0)
             continue;
         uint4* dq = reinterpret_cast<uint4*>(recv_q + (int64_t)dj * H);
 #pragma unroll
-        for (int i = 0; i < kU32Fp8; ++i)
+        for (int i = 0; i < kU; ++i)
             if (v0 + 32 * i < vpr)
                 dq[v0 + 32 * i] = q[i];
         if (sc_ok)

@@ -451,6 +451,7 @@ constexpr int kSmallRounds = 4;
 constexpr int kSmallEntries = kSmallThreads * kSmallRounds;
 constexpr int kSmallMaxE = 1024;
 constexpr int64_t kSmallMaxRankBytes = 65536;  // T x R bytes of is_token_in_rank
+constexpr int kFusedU32Fp8 = 1;                // fused FP8 pieces: 512 channels
 
 __host__ __device__ inline int small_rounds(int64_t nent)
 {
@@ -505,6 +506,24 @@ __device__ __forceinline__ int32_t exscan_u16x8(int4& v, int32_t acc)
     v = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
     return acc;
 }
+
+// Lanes of the warp whose key equals this lane's, for keys in [-1, 2^nbits - 1)
+// (nbits uniform over the warp): the AND over the key bits of the matching
+// ballot -- nbits ballots, where __match_any_sync slows down with the number
+// of distinct keys (up to 32 here).
+__device__ __forceinline__ unsigned match_key(int key, int nbits)
+{
+    const unsigned v = (unsigned)(key + 1);
+    unsigned m = kFull;
+    for (int b = 0; b < nbits; ++b) {
+        const unsigned bit = (v >> b) & 1u;
+        const unsigned bal = __ballot_sync(kFull, bit);
+        m &= bit ? bal : ~bal;
+    }
+    return m;
+}
+
+__host__ __device__ inline int bit_width(unsigned v) { int n = 0; while (v >> n) ++n; return n; }
 
 // kFused = false: the layout alone.  kFused = true: then every warp of the
 // grid dispatches (token, unit) pieces with the positions in its own shared
@@ -569,8 +588,12 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     if (__syncthreads_or(bad) && tid == 0 && leader)
         atomicOr(err, kErrBadIndex);
 
-    // 2: equal experts inside each warp
+    // 2: equal experts inside each warp.  When k divides 32 a token's slots
+    // share a warp, and tokens per rank are counted here from the rank groups
+    // (an entry counts when no lower slot of its token is in its group).
     const unsigned lt = lanemask_lt();
+    const int ebits = bit_width((unsigned)E), rbits = bit_width((unsigned)R);
+    const bool tok_in_warp = (32 % k) == 0;
     int rin[kSmallRounds];
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
@@ -578,14 +601,21 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
         if (q < rounds) {
             const int f = q * kSmallThreads + tid;
             const int e = e_r[q];
-            const unsigned peers = __match_any_sync(kFull, e);
+            const unsigned peers = match_key(e, ebits);
             rin[q] = __popc(peers & lt);
             const int rk = e >= 0 ? (int)(((uint64_t)e * rank_magic) >> 32) : -1;
             if (e >= 0 && rin[q] == 0)
                 vtab[(size_t)e * nv + q * 32 + warp] = (uint16_t)__popc(peers);
-            const unsigned rpeers = __match_any_sync(kFull, rk);
+            const unsigned rpeers = match_key(rk, rbits);
             if (rk >= 0 && (rpeers & lt) == 0)
                 atomicAdd(&rrows[rk], __popc(rpeers));
+            if (leader && tok_in_warp) {
+                const int j = lane % k;
+                const bool first = rk >= 0 && (rpeers & (((1u << j) - 1u) << (lane - j))) == 0;
+                const unsigned grp = rpeers & __ballot_sync(kFull, first);
+                if (first && (grp & lt) == 0)
+                    atomicAdd(&rhist[rk], __popc(grp));
+            }
             if (f < nent) {
                 erank[f] = rk;
                 if (leader && rk >= 0)
@@ -633,7 +663,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     }
     if (lane == 31)
         wsum[warp] = pincl;
-    if (leader) {
+    if (leader && !tok_in_warp) {
 #pragma unroll
         for (int q = 0; q < kSmallRounds; ++q) {
             const int f = q * kSmallThreads + tid;
@@ -708,7 +738,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     __syncthreads();
     const int64_t G = gridDim.x;
     const int64_t vpr = fd.H / 16;
-    const int64_t uvec = fd.fp8 ? units::kUnitVec32Fp8 : units::kUnitVec32;
+    const int64_t uvec = fd.fp8 ? 32 * kFusedU32Fp8 : units::kUnitVec32;
     const int64_t upr = (vpr + uvec - 1) / uvec;
     const units::Vec32* xv = static_cast<const units::Vec32*>(fd.x);
     for (int64_t u = (int64_t)warp * G + blockIdx.x; u < (int64_t)T * upr;
@@ -720,7 +750,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             d = -1;
         }
         if (fd.fp8)
-            units::fp8_unit(xv + t * vpr, vpr, u - t * upr, d, k, fd.H,
+            units::fp8_unit<kFusedU32Fp8>(xv + t * vpr, vpr, u - t * upr, d, k, fd.H,
                             static_cast<uint8_t*>(fd.recv_x), fd.recv_scales, fd.scales_ld);
         else
             units::bf16_unit(xv + t * vpr, vpr, u - t * upr, d, k,

@@ -48,6 +48,9 @@ FUZZ = [
     (2000, 2048, 64, 8, 128, 0.0, True),   # large E
     (64, 8192, 8192, 4, 128, 0.0, True),   # maximum E, R = E
     (4096, 256, 256, 8, 128, 0.5, True),   # many unused slots
+    (200, 64, 8, 6, 16, 0.1, True),        # small batch, k does not divide 32
+    (150, 40, 5, 20, 8, 0.1, True),        # small batch, three rounds of 1024 entries
+    (100, 1024, 8, 9, 128, 0.0, False),    # small batch, E = 1024, duplicates
     (20000, 256, 8, 8, 128, 0.0, True),    # many chunks
     (512, 256, 16, 8, 128, 0.1, True),     # 4096 entries: the one-CTA path's limit
     (513, 256, 16, 8, 128, 0.0, True),     # 4104 entries: the tiled path
