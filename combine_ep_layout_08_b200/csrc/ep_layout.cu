@@ -431,37 +431,49 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
 // layout in its own shared memory (deterministic, so all agree) and CTA 0
 // writes it out; the pad rows of recv_src -- most of the bytes at decode
 // sizes -- are spread over the CTAs, since one SM alone stores only some
-// tens of GB/s.  Five block barriers:
-//   1  topk_idx loaded (issued before anything else), the count table, rank
-//      counters and is_token_in_rank zeroed;
-//   2  per round, __match_any_sync groups equal experts inside the warp; the
-//      first lane of a group stores the group size in vtab[e][v]; entry
-//      ranks, is_token_in_rank bytes, rows per rank (one shared atomic per
-//      group of equal ranks);
+// tens of GB/s.  Shared-memory atomics are avoided on the common path: many
+// warps adding to the same few counters back up the shared-memory pipe.
+// Five block barriers:
+//   1  tables zeroed (before the dependent-launch wait: shared memory only),
+//      topk_idx loaded, is_token_in_rank zeroed;
+//   2  per round, equal experts inside the warp (ballots over the key bits);
+//      the first lane of a group stores the group size in vtab[e][v]; entry
+//      ranks and is_token_in_rank bytes.  When k divides 32 a token's slots
+//      share the warp: an entry is the first of its token in its rank when no
+//      lower slot of the token has its rank, and the first lane of each rank
+//      group of such entries stores their number in ttab[r][v] (R <= 128);
 //   3  per expert, tpe threads scan vtab[e][*] over the virtual warps in place
-//      (exclusive), the last of them holding cnt[e]; the padded counts are
-//      scanned across the warp; tokens per rank (an entry counts when no
-//      earlier slot of its token has the same rank);
-//   4  each warp scans the 32 warp totals itself and stores off[e];
+//      (exclusive), the last of them holding cnt[e]; padded and plain counts
+//      scanned across the warp; tokens per rank summed from ttab (or, for
+//      other shapes, counted with shared atomics);
+//   4  each warp scans the 32 warp totals itself and stores off[e] and the
+//      unpadded offsets uoff[e] (rows per rank are their differences);
 //   5  position = off[e] + vtab[e][v] + rank among the equal lanes.
-// Shared memory: vtab uint16 [E][nv] (nv = 32 rounds), then 32-bit words
-// cnt[E], off[E+1], wsum[32], rhist[R], rrows[R], erank[1024 rounds].
+// Shared memory: vtab uint16 [E][nv] (nv = 32 rounds), ttab uint16 [R][nv]
+// when R <= kSmallTabR, then 32-bit words cnt[E], off[E+1], uoff[E+1],
+// wsum[2][32], rhist[R], erank[1024 rounds].
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallRounds = 4;
 constexpr int kSmallEntries = kSmallThreads * kSmallRounds;
 constexpr int kSmallMaxE = 1024;
 constexpr int64_t kSmallMaxRankBytes = 65536;  // T x R bytes of is_token_in_rank
 constexpr int kFusedU32Fp8 = 1;                // fused FP8 pieces: 512 channels
+constexpr int kSmallTabR = 128;                // largest R with a tokens-per-rank table
 
 __host__ __device__ inline int small_rounds(int64_t nent)
 {
     return nent <= kSmallThreads ? 1 : (int)((nent + kSmallThreads - 1) / kSmallThreads);
 }
 
+__host__ __device__ inline size_t small_ttab_halves(int R, int rounds)
+{
+    return R <= kSmallTabR ? (size_t)R * 32 * rounds : 0;
+}
+
 __host__ __device__ inline size_t small_smem_bytes(int E, int R, int rounds)
 {
-    return 2 * (size_t)E * 32 * rounds +
-           sizeof(int32_t) * ((size_t)E + E + 1 + 32 + 2 * (size_t)R + (size_t)kSmallThreads * rounds);
+    return 2 * ((size_t)E * 32 * rounds + small_ttab_halves(R, rounds)) +
+           sizeof(int32_t) * ((size_t)E + 2 * ((size_t)E + 1) + 64 + R + (size_t)kSmallThreads * rounds);
 }
 
 bool small_fits(int64_t T, int k, int E, int R)
@@ -539,36 +551,36 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
                     int32_t* __restrict__ recv_src, int32_t* err, FusedDispatch fd)
 {
     extern __shared__ __align__(16) unsigned char small_smem[];
-    pdl_wait();
-    pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool leader = blockIdx.x == 0;
     const int nent = T * k;
     const int rounds = small_rounds(nent);
     const int nv = 32 * rounds;
+    const bool tok_in_warp = (32 % k) == 0;
+    const bool use_ttab = tok_in_warp && R <= kSmallTabR;
     uint16_t* vtab = reinterpret_cast<uint16_t*>(small_smem);  // [E][nv]
-    int32_t* cnt = reinterpret_cast<int32_t*>(small_smem + 2 * (size_t)E * nv);
+    uint16_t* ttab = vtab + (size_t)E * nv;                     // [R][nv] when use_ttab
+    int32_t* cnt = reinterpret_cast<int32_t*>(ttab + small_ttab_halves(R, rounds));
     int32_t* off = cnt + E;
-    int32_t* wsum = off + E + 1;
-    int32_t* rhist = wsum + 32;
-    int32_t* rrows = rhist + R;
-    int32_t* erank = rrows + R;  // entry ranks, then (fused) positions
+    int32_t* uoff = off + E + 1;
+    int32_t* wsum = uoff + E + 1;  // [2][32]: padded, plain
+    int32_t* rhist = wsum + 64;
+    int32_t* erank = rhist + R;    // entry ranks, then (fused) positions
 
-    // 1: loads first; zeroing while they are in flight
+    // 1: shared tables zeroed before the wait (no global memory touched)
+    {
+        int4* z = reinterpret_cast<int4*>(vtab);
+        const int n16 = (int)(((size_t)E * nv + small_ttab_halves(R, rounds)) / 8);
+        for (int i = tid; i < n16; i += kSmallThreads) z[i] = make_int4(0, 0, 0, 0);
+    }
+    for (int r = tid; r < R; r += kSmallThreads) rhist[r] = 0;
+    pdl_wait();
+    pdl_trigger();
     int64_t raw[kSmallRounds];
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
         const int f = q * kSmallThreads + tid;
         raw[q] = (q < rounds && f < nent) ? topk_idx[f] : -1;
-    }
-    {
-        int4* z = reinterpret_cast<int4*>(vtab);
-        const int n16 = (int)(((size_t)E * nv) / 8);  // E nv halfwords, a multiple of 32
-        for (int i = tid; i < n16; i += kSmallThreads) z[i] = make_int4(0, 0, 0, 0);
-    }
-    for (int r = tid; r < R; r += kSmallThreads) {
-        rhist[r] = 0;
-        rrows[r] = 0;
     }
     if (leader) {
         const int64_t bytes = (int64_t)T * R;
@@ -588,33 +600,29 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     if (__syncthreads_or(bad) && tid == 0 && leader)
         atomicOr(err, kErrBadIndex);
 
-    // 2: equal experts inside each warp.  When k divides 32 a token's slots
-    // share a warp, and tokens per rank are counted here from the rank groups
-    // (an entry counts when no lower slot of its token is in its group).
+    // 2: equal experts (and ranks) inside each warp
     const unsigned lt = lanemask_lt();
     const int ebits = bit_width((unsigned)E), rbits = bit_width((unsigned)R);
-    const bool tok_in_warp = (32 % k) == 0;
     int rin[kSmallRounds];
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
         rin[q] = 0;
         if (q < rounds) {
             const int f = q * kSmallThreads + tid;
+            const int v = q * 32 + warp;
             const int e = e_r[q];
             const unsigned peers = match_key(e, ebits);
             rin[q] = __popc(peers & lt);
             const int rk = e >= 0 ? (int)(((uint64_t)e * rank_magic) >> 32) : -1;
             if (e >= 0 && rin[q] == 0)
-                vtab[(size_t)e * nv + q * 32 + warp] = (uint16_t)__popc(peers);
-            const unsigned rpeers = match_key(rk, rbits);
-            if (rk >= 0 && (rpeers & lt) == 0)
-                atomicAdd(&rrows[rk], __popc(rpeers));
-            if (leader && tok_in_warp) {
+                vtab[(size_t)e * nv + v] = (uint16_t)__popc(peers);
+            if (leader && use_ttab) {
+                const unsigned rpeers = match_key(rk, rbits);
                 const int j = lane % k;
                 const bool first = rk >= 0 && (rpeers & (((1u << j) - 1u) << (lane - j))) == 0;
                 const unsigned grp = rpeers & __ballot_sync(kFull, first);
                 if (first && (grp & lt) == 0)
-                    atomicAdd(&rhist[rk], __popc(grp));
+                    ttab[(size_t)rk * nv + v] = (uint16_t)__popc(grp);
             }
             if (f < nent) {
                 erank[f] = rk;
@@ -630,7 +638,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     while (2 * tpe * E <= kSmallThreads && (nv / (2 * tpe)) % 8 == 0) tpe *= 2;
     const int x = tid / tpe, p = tid - x * tpe;
     const int chunk = nv / tpe;  // a multiple of 8 halfwords: whole int4s
-    int32_t padded = 0;
+    int32_t padded = 0, plain = 0;
     {
         int4* row = reinterpret_cast<int4*>(vtab + (size_t)x * nv + p * chunk);
         int32_t part = 0;
@@ -651,19 +659,32 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             }
             if (p == tpe - 1) {
                 cnt[x] = incl;
+                plain = incl;
                 padded = pad_up(incl, block_m);
             }
         }
     }
-    int32_t pincl = padded;
+    int32_t pincl = padded, uincl = plain;
     for (int o = 1; o < 32; o <<= 1) {
         const int32_t u = __shfl_up_sync(kFull, pincl, o);
-        if (lane >= o)
+        const int32_t w2 = __shfl_up_sync(kFull, uincl, o);
+        if (lane >= o) {
             pincl += u;
+            uincl += w2;
+        }
     }
-    if (lane == 31)
+    if (lane == 31) {
         wsum[warp] = pincl;
-    if (leader && !tok_in_warp) {
+        wsum[32 + warp] = uincl;
+    }
+    if (leader && use_ttab) {
+        for (int r = tid; r < R; r += kSmallThreads) {
+            const int4* trow = reinterpret_cast<const int4*>(ttab + (size_t)r * nv);
+            int32_t sum = 0;
+            for (int i = 0; i < nv / 8; ++i) sum += sum_u16x8(trow[i]);
+            rhist[r] = sum;
+        }
+    } else if (leader) {
 #pragma unroll
         for (int q = 0; q < kSmallRounds; ++q) {
             const int f = q * kSmallThreads + tid;
@@ -679,20 +700,27 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     }
     __syncthreads();
 
-    // 4: expert offsets
+    // 4: expert offsets, padded and plain
     {
-        const int32_t v = wsum[lane];
-        int32_t inc = v;
+        const int32_t v = wsum[lane], v2 = wsum[32 + lane];
+        int32_t inc = v, inc2 = v2;
         for (int o = 1; o < 32; o <<= 1) {
             const int32_t u = __shfl_up_sync(kFull, inc, o);
-            if (lane >= o)
+            const int32_t u2 = __shfl_up_sync(kFull, inc2, o);
+            if (lane >= o) {
                 inc += u;
+                inc2 += u2;
+            }
         }
         const int32_t base = __shfl_sync(kFull, inc - v, warp);
+        const int32_t base2 = __shfl_sync(kFull, inc2 - v2, warp);
         if (x < E && p == tpe - 1) {
             off[x] = base + pincl - padded;
-            if (x == E - 1)
+            uoff[x] = base2 + uincl - plain;
+            if (x == E - 1) {
                 off[E] = base + pincl;
+                uoff[E] = base2 + uincl;
+            }
         }
     }
     __syncthreads();
@@ -703,7 +731,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
         for (int e = tid; e <= E; e += kSmallThreads) expert_off_g[e] = off[e];
         for (int r = tid; r <= R; r += kSmallThreads) rank_off_g[r] = off[r * epr];
         for (int r = tid; r < R; r += kSmallThreads) {
-            rows_per_rank_g[r] = rrows[r];
+            rows_per_rank_g[r] = uoff[(r + 1) * epr] - uoff[r * epr];
             tokens_per_rank_g[r] = rhist[r];
         }
         if (tid == 0)
