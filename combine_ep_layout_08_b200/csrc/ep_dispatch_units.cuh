@@ -65,6 +65,18 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d)
 
 // BF16: the lane's 32-byte vector of the unit is read once and written to
 // each of the k destination rows; consecutive lanes write consecutive bytes.
+// bf16_store takes the vector already loaded (v = the lane's vector index in
+// the row).
+__device__ __forceinline__ void bf16_store(const Vec32& val, int64_t v, int64_t vpr, int d, int k,
+                                           Vec32* __restrict__ recv)
+{
+    for (int j = 0; j < k; ++j) {
+        const int dj = __shfl_sync(kFull, d, j);
+        if (dj >= 0 && v < vpr)
+            st32(recv + (int64_t)dj * vpr + v, val);
+    }
+}
+
 __device__ __forceinline__ void bf16_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
                                           int d, int k, Vec32* __restrict__ recv)
 {
@@ -73,11 +85,7 @@ __device__ __forceinline__ void bf16_unit(const Vec32* __restrict__ xs, int64_t 
     Vec32 val;
     if (v < vpr)
         val = ld32_once(xs + v);
-    for (int j = 0; j < k; ++j) {
-        const int dj = __shfl_sync(kFull, d, j);
-        if (dj >= 0 && v < vpr)
-            st32(recv + (int64_t)dj * vpr + v, val);
-    }
+    bf16_store(val, v, vpr, d, k, recv);
 }
 
 // FP8: lane vector i of the unit covers channels 16 v .. 16 v + 15 with
@@ -87,15 +95,13 @@ __device__ __forceinline__ void bf16_unit(const Vec32* __restrict__ xs, int64_t 
 // store; the unit's 4 kU scales are gathered into lanes 0 .. 4 kU - 1 and
 // written as one run per destination row (row-major scales).  xs: the token
 // row in 32-byte vectors, vpr = H / 16.
-template <int kU = kU32Fp8>
-__device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
-                                         int d, int k, int H, uint8_t* __restrict__ recv_q,
-                                         float* __restrict__ recv_scales, int64_t scales_ld)
+// The lane's kU vectors of the unit, zero past the end of the row.
+template <int kU>
+__device__ __forceinline__ void fp8_load(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
+                                         Vec32 (&a)[kU])
 {
     const int lane = threadIdx.x & 31;
-    const int nblk = H / 128;
     const int64_t v0 = unit * (32 * kU) + lane;
-    Vec32 a[kU];
 #pragma unroll
     for (int i = 0; i < kU; ++i) {
         if (v0 + 32 * i < vpr) {
@@ -105,6 +111,17 @@ __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t v
             for (int c = 0; c < 8; ++c) a[i].w[c] = 0u;
         }
     }
+}
+
+// Quantise the loaded vectors and write codes and scales to the k rows.
+template <int kU>
+__device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int64_t unit, int d,
+                                          int k, int H, uint8_t* __restrict__ recv_q,
+                                          float* __restrict__ recv_scales, int64_t scales_ld)
+{
+    const int lane = threadIdx.x & 31;
+    const int nblk = H / 128;
+    const int64_t v0 = unit * (32 * kU) + lane;
     uint4 q[kU];
     float sc[kU];
 #pragma unroll
@@ -163,6 +180,16 @@ __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t v
         if (sc_ok)
             recv_scales[scale_index(dj, blk, nblk, scales_ld)] = my_scale;
     }
+}
+
+template <int kU = kU32Fp8>
+__device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
+                                         int d, int k, int H, uint8_t* __restrict__ recv_q,
+                                         float* __restrict__ recv_scales, int64_t scales_ld)
+{
+    Vec32 a[kU];
+    fp8_load<kU>(xs, vpr, unit, a);
+    fp8_store<kU>(a, vpr, unit, d, k, H, recv_q, recv_scales, scales_ld);
 }
 
 }  // namespace units

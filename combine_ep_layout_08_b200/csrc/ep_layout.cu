@@ -457,7 +457,6 @@ constexpr int kSmallRounds = 4;
 constexpr int kSmallEntries = kSmallThreads * kSmallRounds;
 constexpr int kSmallMaxE = 1024;
 constexpr int64_t kSmallMaxRankBytes = 65536;  // T x R bytes of is_token_in_rank
-constexpr int kFusedU32Fp8 = 1;                // fused FP8 pieces: 512 channels
 constexpr int kSmallTabR = 128;                // largest R with a tokens-per-rank table
 
 __host__ __device__ inline int small_rounds(int64_t nent)
@@ -481,6 +480,50 @@ bool small_fits(int64_t T, int k, int E, int R)
     const int64_t nent = T * k;
     return nent <= kSmallEntries && E <= kSmallMaxE && T * R <= kSmallMaxRankBytes &&
            small_smem_bytes(E, R, small_rounds(nent)) <= kSmemBudget;
+}
+
+// Per-launch constants of the small kernel, computed on the host so that the
+// kernel's 1024 threads shift instead of dividing (k and block_m are powers
+// of two in practice; other values take the division).
+struct SmallPlan {
+    int rounds;   // rounds of 1024 entries
+    int nv;       // virtual warps, 32 rounds
+    int tpe_log;  // log2 of the threads per expert in the count scan
+    int ebits;    // bit width of E: match keys e + 1 in [0, E]
+    int rbits;    // bit width of R
+    int k_log;    // log2 k when k is a power of two, else -1
+    int bm_log;   // log2 block_m when a power of two, else -1
+};
+
+int log2_if_pow2(int v)
+{
+    if (v <= 0 || (v & (v - 1)) != 0)
+        return -1;
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+}
+
+int bits_of(unsigned v)
+{
+    int n = 0;
+    while (n < 32 && (v >> n) != 0u) ++n;
+    return n;
+}
+
+SmallPlan make_small_plan(int T, int k, int E, int R, int block_m)
+{
+    SmallPlan pl;
+    pl.rounds = small_rounds((int64_t)T * k);
+    pl.nv = 32 * pl.rounds;
+    int tpe = 1;  // a power of two with tpe E <= 1024 and nv / tpe a multiple of 8
+    while (2 * tpe * E <= kSmallThreads && (pl.nv / (2 * tpe)) % 8 == 0) tpe *= 2;
+    pl.tpe_log = log2_if_pow2(tpe);
+    pl.ebits = bits_of((unsigned)E);
+    pl.rbits = bits_of((unsigned)R);
+    pl.k_log = log2_if_pow2(k);
+    pl.bm_log = log2_if_pow2(block_m);
+    return pl;
 }
 
 // The dispatch half of the fused small-batch kernel (layout + dispatch in
@@ -535,8 +578,6 @@ __device__ __forceinline__ unsigned match_key(int key, int nbits)
     return m;
 }
 
-__host__ __device__ inline int bit_width(unsigned v) { int n = 0; while (v >> n) ++n; return n; }
-
 // kFused = false: the layout alone.  kFused = true: then every warp of the
 // grid dispatches (token, unit) pieces with the positions in its own shared
 // memory -- no grid-wide wait.
@@ -548,15 +589,16 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
                     int32_t* __restrict__ tokens_per_rank_g,
                     int32_t* __restrict__ rows_per_rank_g, int32_t* __restrict__ total_rows_g,
                     uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
-                    int32_t* __restrict__ recv_src, int32_t* err, FusedDispatch fd)
+                    int32_t* __restrict__ recv_src, int32_t* err, FusedDispatch fd,
+                    SmallPlan pl)
 {
     extern __shared__ __align__(16) unsigned char small_smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool leader = blockIdx.x == 0;
     const int nent = T * k;
-    const int rounds = small_rounds(nent);
-    const int nv = 32 * rounds;
+    const int rounds = pl.rounds, nv = pl.nv;
     const bool tok_in_warp = (32 % k) == 0;
+    auto token_of = [&](int f) { return pl.k_log >= 0 ? f >> pl.k_log : f / k; };
     const bool use_ttab = tok_in_warp && R <= kSmallTabR;
     uint16_t* vtab = reinterpret_cast<uint16_t*>(small_smem);  // [E][nv]
     uint16_t* ttab = vtab + (size_t)E * nv;                     // [R][nv] when use_ttab
@@ -576,6 +618,23 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     for (int r = tid; r < R; r += kSmallThreads) rhist[r] = 0;
     pdl_wait();
     pdl_trigger();
+    // fused: this warp's first dispatch piece is loaded now, so that its
+    // latency hides behind the layout (x does not depend on it)
+    const int64_t G = gridDim.x;
+    const int64_t vpr = kFused ? fd.H / 16 : 0;
+    const int64_t upr = kFused ? (vpr + 31) / 32 : 1;  // 512-channel pieces, BF16 and FP8
+    const int64_t npieces = kFused ? (int64_t)T * upr : 0;
+    const bool narrow = npieces < (int64_t(1) << 31);  // 32-bit division suffices
+    auto token_of_piece = [&](int64_t u) {
+        return narrow ? (int64_t)((uint32_t)u / (uint32_t)upr) : u / upr;
+    };
+    const int64_t u0 = (int64_t)warp * G + blockIdx.x;
+    const units::Vec32* xv = static_cast<const units::Vec32*>(fd.x);
+    units::Vec32 cur[1];
+    if (kFused && u0 < npieces) {
+        const int64_t t = token_of_piece(u0);
+        units::fp8_load<1>(xv + t * vpr, vpr, u0 - t * upr, cur);
+    }
     int64_t raw[kSmallRounds];
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
@@ -602,7 +661,6 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
 
     // 2: equal experts (and ranks) inside each warp
     const unsigned lt = lanemask_lt();
-    const int ebits = bit_width((unsigned)E), rbits = bit_width((unsigned)R);
     int rin[kSmallRounds];
 #pragma unroll
     for (int q = 0; q < kSmallRounds; ++q) {
@@ -611,14 +669,14 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             const int f = q * kSmallThreads + tid;
             const int v = q * 32 + warp;
             const int e = e_r[q];
-            const unsigned peers = match_key(e, ebits);
+            const unsigned peers = match_key(e, pl.ebits);
             rin[q] = __popc(peers & lt);
             const int rk = e >= 0 ? (int)(((uint64_t)e * rank_magic) >> 32) : -1;
             if (e >= 0 && rin[q] == 0)
                 vtab[(size_t)e * nv + v] = (uint16_t)__popc(peers);
             if (leader && use_ttab) {
-                const unsigned rpeers = match_key(rk, rbits);
-                const int j = lane % k;
+                const unsigned rpeers = match_key(rk, pl.rbits);
+                const int j = lane & (k - 1);  // k divides 32: a power of two
                 const bool first = rk >= 0 && (rpeers & (((1u << j) - 1u) << (lane - j))) == 0;
                 const unsigned grp = rpeers & __ballot_sync(kFull, first);
                 if (first && (grp & lt) == 0)
@@ -627,17 +685,16 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             if (f < nent) {
                 erank[f] = rk;
                 if (leader && rk >= 0)
-                    is_token_in_rank[(int64_t)(f / k) * R + rk] = 1;
+                    is_token_in_rank[(int64_t)token_of(f) * R + rk] = 1;
             }
         }
     }
     __syncthreads();
 
     // 3: per expert, tpe consecutive threads over nv / tpe virtual warps each
-    int tpe = 1;
-    while (2 * tpe * E <= kSmallThreads && (nv / (2 * tpe)) % 8 == 0) tpe *= 2;
-    const int x = tid / tpe, p = tid - x * tpe;
-    const int chunk = nv / tpe;  // a multiple of 8 halfwords: whole int4s
+    const int tpe = 1 << pl.tpe_log;
+    const int x = tid >> pl.tpe_log, p = tid & (tpe - 1);
+    const int chunk = nv >> pl.tpe_log;  // a multiple of 8 halfwords: whole int4s
     int32_t padded = 0, plain = 0;
     {
         int4* row = reinterpret_cast<int4*>(vtab + (size_t)x * nv + p * chunk);
@@ -660,7 +717,8 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             if (p == tpe - 1) {
                 cnt[x] = incl;
                 plain = incl;
-                padded = pad_up(incl, block_m);
+                padded = pl.bm_log >= 0 ? ((incl + block_m - 1) >> pl.bm_log) << pl.bm_log
+                                        : pad_up(incl, block_m);
             }
         }
     }
@@ -690,7 +748,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             const int f = q * kSmallThreads + tid;
             if (q < rounds && f < nent && e_r[q] >= 0) {
                 const int rk = erank[f];
-                const int t = f / k, j = f - t * k;
+                const int t = token_of(f), j = f - t * k;
                 bool first = true;
                 for (int jj = 0; jj < j; ++jj) first &= (erank[t * k + jj] != rk);
                 if (first)
@@ -754,35 +812,36 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             if (leader) {
                 dst_row[f] = pos;
                 if (pos >= 0)
-                    recv_src[pos] = f / k;
+                    recv_src[pos] = token_of(f);
             }
         }
     }
     if (!kFused)
         return;
 
-    // dispatch: (token, unit) pieces dealt to the CTAs in turn, so that the
-    // row stores spread over every SM
+    // dispatch: (token, 512-channel piece) pairs dealt to the CTAs in turn,
+    // so that the row stores spread over every SM; each warp loads its next
+    // piece after storing the current one
     __syncthreads();
-    const int64_t G = gridDim.x;
-    const int64_t vpr = fd.H / 16;
-    const int64_t uvec = fd.fp8 ? 32 * kFusedU32Fp8 : units::kUnitVec32;
-    const int64_t upr = (vpr + uvec - 1) / uvec;
-    const units::Vec32* xv = static_cast<const units::Vec32*>(fd.x);
-    for (int64_t u = (int64_t)warp * G + blockIdx.x; u < (int64_t)T * upr;
-         u += G * (kSmallThreads / 32)) {
-        const int64_t t = u / upr;
+    const int64_t stride = G * (kSmallThreads / 32);
+    for (int64_t u = u0; u < npieces; u += stride) {
+        const int64_t t = token_of_piece(u);
         int d = lane < k ? erank[t * k + lane] : -1;
         if (d >= fd.cap_rows) {
             atomicOr(err, kErrDispatchCap);
             d = -1;
         }
         if (fd.fp8)
-            units::fp8_unit<kFusedU32Fp8>(xv + t * vpr, vpr, u - t * upr, d, k, fd.H,
-                            static_cast<uint8_t*>(fd.recv_x), fd.recv_scales, fd.scales_ld);
+            units::fp8_store<1>(cur, vpr, u - t * upr, d, k, fd.H,
+                                static_cast<uint8_t*>(fd.recv_x), fd.recv_scales, fd.scales_ld);
         else
-            units::bf16_unit(xv + t * vpr, vpr, u - t * upr, d, k,
-                             static_cast<units::Vec32*>(fd.recv_x));
+            units::bf16_store(cur[0], (u - t * upr) * 32 + lane, vpr, d, k,
+                              static_cast<units::Vec32*>(fd.recv_x));
+        const int64_t un = u + stride;
+        if (un < npieces) {
+            const int64_t tn = token_of_piece(un);
+            units::fp8_load<1>(xv + tn * vpr, vpr, un - tn * upr, cur);
+        }
     }
 }
 
@@ -1145,7 +1204,8 @@ cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaS
         return launch_pdl(layout_small_kernel<false>, grid, kSmallThreads, smem, s, topk_idx, T,
                           k, E, R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off,
                           h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
-                          h.is_token_in_rank, h.dst_row, h.recv_src, h.err, FusedDispatch{});
+                          h.is_token_in_rank, h.dst_row, h.recv_src, h.err, FusedDispatch{},
+                          make_small_plan(T, k, E, R, h.block_m));
     }
 
     if (allow_fused && nchunks > 0) {
@@ -1210,7 +1270,7 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
     return launch_pdl(layout_small_kernel<true>, grid, kSmallThreads, smem, s, topk_idx, T, k, E,
                       R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off, h.rank_off,
                       h.tokens_per_rank, h.rows_per_rank, h.total_rows, h.is_token_in_rank,
-                      h.dst_row, h.recv_src, h.err, fd);
+                      h.dst_row, h.recv_src, h.err, fd, make_small_plan(T, k, E, R, h.block_m));
 }
 
 }  // namespace ep
