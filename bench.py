@@ -115,13 +115,27 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
             os.close(fd)
             cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                   "-lms", "50"]
+                   "-lms", "25"]
             if bus_id:
                 cmd += ["-i", bus_id]
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
                                          stderr=subprocess.DEVNULL)
+            # nvidia-smi needs a moment to start: wait for its first sample so
+            # that the timed region is covered
+            deadline = time.time() + 15.0
+            while time.time() < deadline and self.proc.poll() is None:
+                if self._count_rows() > 0:
+                    break
+                time.sleep(0.05)
         except Exception:
             self.proc = None
+
+    def _count_rows(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for line in f if line.count(",") >= 8)
+        except OSError:
+            return 0
 
     def mark(self):
         return time.time()
@@ -129,7 +143,11 @@ class ClockSampler:
     def stop(self, t0, t1):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.12)
+        # let at least one sample land after the timed region
+        n0 = self._count_rows()
+        deadline = time.time() + 2.0
+        while time.time() < deadline and self._count_rows() < n0 + 2:
+            time.sleep(0.02)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -148,9 +166,9 @@ class ClockSampler:
             except Exception:
                 continue
         os.unlink(self.path)
-        inwin = [r for r in rows if t0 - 0.06 <= r[0] <= t1 + 0.06]
+        inwin = [r for r in rows if t0 - 0.03 <= r[0] <= t1 + 0.03]
         window = "timed"
-        if len(inwin) < 3:
+        if len(inwin) < 2:
             inwin, window = rows, "whole run (timed region shorter than the sampling period)"
         if not inwin:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
@@ -328,8 +346,12 @@ def fused_step(s):
     ep.ep_combine(s["h"], s["y"], s["wt"], out=s["out"])
 
 
-def graph_latency_us(s, reps=200, step=None):
-    """Decode-style latency: one CUDA graph holding layout+dispatch+combine."""
+def graph_latency_us(s, reps=200, step=None, inner=1):
+    """Decode-style latency: a CUDA graph holding `inner` back-to-back steps
+    (layout + dispatch + combine each), replayed `reps` times; returns the
+    device time per step.  With inner = 1 the replay rate of the host bounds
+    the figure; inner = 20 is a decode pass with many MoE layers in one
+    graph."""
     import torch
 
     step = step or gpu_step
@@ -341,8 +363,9 @@ def graph_latency_us(s, reps=200, step=None):
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        step(s)
-    for _ in range(20):
+        for _ in range(inner):
+            step(s)
+    for _ in range(10):
         g.replay()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
@@ -352,7 +375,7 @@ def graph_latency_us(s, reps=200, step=None):
         g.replay()
     b.record()
     b.synchronize()
-    us = a.elapsed_time(b) * 1000.0 / reps
+    us = a.elapsed_time(b) * 1000.0 / (reps * inner)
     del g
     return us
 
@@ -505,6 +528,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--secondary", default="all",
+                    help="comma-separated secondary workloads (skewed, dsv3, decode, backward) or all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args()
@@ -576,7 +601,9 @@ def main():
     if not args.no_secondary:
         del s
         torch.cuda.empty_cache()
-        for name in SECONDARY:
+        chosen = SECONDARY if args.secondary == "all" else \
+            [n for n in SECONDARY if n in args.secondary.split(",")]
+        for name in chosen:
             s2 = gpu_setup(name, args.seed + rank, dev)
             w2 = s2["w"]
             n = max(3, min(args.steps, 100))
@@ -591,13 +618,20 @@ def main():
                    "combine_GBps": round(cb / (statistics.mean(t2["combine"]) / 1e3) / 1e9, 1),
                    "value_GBps": round((db + cb) / (statistics.mean(t2["step"]) / 1e3) / 1e9, 1)}
             if name == "decode":
-                ent["graph_step_us"] = round(graph_latency_us(s2), 2)
-                ent["graph_fused_step_us"] = round(graph_latency_us(s2, step=fused_step), 2)
+                # per step inside a graph of 20 steps; one-step graphs as well
+                ent["graph_step_us"] = round(graph_latency_us(s2, reps=50, inner=20), 2)
+                ent["graph_fused_step_us"] = round(
+                    graph_latency_us(s2, reps=50, step=fused_step, inner=20), 2)
+                ent["graph1_step_us"] = round(graph_latency_us(s2), 2)
+                ent["graph1_fused_step_us"] = round(graph_latency_us(s2, step=fused_step), 2)
+                ent["graph_note"] = ("graph_*: device time per step in a CUDA graph of 20 "
+                                     "back-to-back steps; graph1_*: a one-step graph replayed "
+                                     "from the host (bounded by the replay rate)")
             secondary[name] = ent
             del s2
             torch.cuda.empty_cache()
 
-    if not args.no_secondary:
+    if not args.no_secondary and (args.secondary == "all" or "backward" in args.secondary.split(",")):
         secondary["8k_backward"] = time_backward(dev, flush, args.seed + rank,
                                                  max(3, min(args.steps, 50)))
         torch.cuda.empty_cache()
