@@ -61,15 +61,15 @@ def _load():
             lib.oracle_recv_rows_bound.restype = i64
             lib.oracle_dispatch_bf16.argtypes = [P, i64, i32, i64, P, P, i64]
             lib.oracle_dispatch_bf16.restype = i32
-            lib.oracle_dispatch_fp8.argtypes = [P, i64, i32, i64, P, P, P, i64]
+            lib.oracle_dispatch_fp8.argtypes = [P, i64, i32, i64, i32, P, P, P, i64]
             lib.oracle_dispatch_fp8.restype = i32
-            lib.oracle_quantize_token_fp8.argtypes = [P, i64, P, P]
+            lib.oracle_quantize_token_fp8.argtypes = [P, i64, i32, P, P]
             lib.oracle_quantize_token_fp8.restype = None
             lib.oracle_expert_scale_bf16.argtypes = [P, P, P, i32, i64, P, P]
             lib.oracle_expert_scale_bf16.restype = None
             lib.oracle_expert_scale_fp8.argtypes = [P, P, P, P, i32, i64, P, P]
             lib.oracle_expert_scale_fp8.restype = None
-            lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, P]
+            lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, i32, P]
             lib.oracle_combine.restype = i32
             lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, P]
             lib.oracle_dispatch_backward.restype = i32
@@ -79,10 +79,11 @@ def _load():
             lib.oracle_dispatch_weights.restype = i32
             lib.oracle_zero_pad_rows.argtypes = [P, i64, P, i64]
             lib.oracle_zero_pad_rows.restype = None
-            lib.oracle_dispatch_fp8_mn.argtypes = [P, i64, i32, i64, P, P, P, i64, i64]
+            lib.oracle_dispatch_fp8_mn.argtypes = [P, i64, i32, i64, i32, P, P, P, i64, i64]
             lib.oracle_dispatch_fp8_mn.restype = i32
             for name in ("oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
-                         "oracle_f32_to_bf16_array"):
+                         "oracle_f32_to_bf16_array", "oracle_fp16_to_f32_array",
+                         "oracle_f32_to_fp16_array"):
                 getattr(lib, name).argtypes = [P, P, i64]
                 getattr(lib, name).restype = None
             _lib = lib
@@ -129,6 +130,30 @@ def bf16_to_f32(b: np.ndarray) -> np.ndarray:
     """Exact widening of bf16 bits (a shift into the upper half of binary32)."""
     b = np.ascontiguousarray(b, dtype=np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def fp16_round(v: np.ndarray) -> np.ndarray:
+    """fp32 -> IEEE binary16 bits, round-to-nearest-even, overflow to infinity."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    h = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_f32_to_fp16_array(_p(v), _p(h), v.size)
+    return h
+
+
+def fp16_to_f32(h: np.ndarray) -> np.ndarray:
+    """Exact widening of binary16 bits to fp32."""
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    v = np.empty(h.shape, dtype=np.float32)
+    _load().oracle_fp16_to_f32_array(_p(h), _p(v), h.size)
+    return v
+
+
+DTYPES = {"bf16": 0, "fp16": 1}
+
+
+def to_f32(bits: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    """16-bit values of the given type (bf16 or fp16) widened to fp32."""
+    return fp16_to_f32(bits) if dtype == "fp16" else bf16_to_f32(bits)
 
 
 # ---------------------------------------------------------------- layout
@@ -191,24 +216,27 @@ def dispatch_bf16(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int) -> np
     return recv[:recv_rows]
 
 
-def quantize_token_fp8(x_bits_row: np.ndarray):
+def quantize_token_fp8(x_bits_row: np.ndarray, dtype: str = "bf16"):
+    """One token row of bf16 or fp16 bits -> (e4m3 codes [H], scales [H/128])."""
     x_bits_row = np.ascontiguousarray(x_bits_row, dtype=np.uint16)
     H = x_bits_row.shape[0]
     q = np.empty(H, np.uint8)
     s = np.empty(max(H // 128, 1), np.float32)
-    _load().oracle_quantize_token_fp8(_p(x_bits_row), H, _p(q), _p(s))
+    _load().oracle_quantize_token_fp8(_p(x_bits_row), H, DTYPES[dtype], _p(q), _p(s))
     return q, s[: H // 128]
 
 
-def dispatch_fp8(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int):
-    """FP8 e4m3 1x128 dispatch: returns (recv_q uint8 [P, H], recv_scales f32 [P, H/128])."""
+def dispatch_fp8(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int, dtype: str = "bf16"):
+    """FP8 e4m3 1x128 dispatch of bf16 or fp16 rows: returns (recv_q uint8 [P, H],
+    recv_scales f32 [P, H/128])."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
     T, H = x_bits.shape
     k = dst_row.shape[1]
     q = np.zeros((max(recv_rows, 1), H), np.uint8)
     s = np.zeros((max(recv_rows, 1), H // 128), np.float32)
-    rc = _load().oracle_dispatch_fp8(_p(x_bits), T, k, H, _p(dst_row), _p(q), _p(s), recv_rows)
+    rc = _load().oracle_dispatch_fp8(_p(x_bits), T, k, H, DTYPES[dtype], _p(dst_row), _p(q),
+                                     _p(s), recv_rows)
     if rc != OK:
         raise OracleError(rc, "oracle_dispatch_fp8")
     return q[:recv_rows], s[:recv_rows]
@@ -243,8 +271,10 @@ def expert_scale_fp8(recv_q: np.ndarray, recv_scales: np.ndarray, lay: Layout,
 
 # ---------------------------------------------------------------- combine
 
-def combine(y_bits: np.ndarray, topk_weights: np.ndarray, dst_row: np.ndarray) -> np.ndarray:
-    """out[t] = bf16(sum_j w[t, j] * y[dst_row[t, j]]), fp32 fma chain in slot order."""
+def combine(y_bits: np.ndarray, topk_weights: np.ndarray, dst_row: np.ndarray,
+            dtype: str = "bf16") -> np.ndarray:
+    """out[t] = rn(sum_j w[t, j] * y[dst_row[t, j]]), fp32 fma chain in slot order; y and
+    out are bf16 or fp16 bits."""
     y_bits = np.ascontiguousarray(y_bits, dtype=np.uint16)
     w = np.ascontiguousarray(topk_weights, dtype=np.float32)
     dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
@@ -253,7 +283,8 @@ def combine(y_bits: np.ndarray, topk_weights: np.ndarray, dst_row: np.ndarray) -
     out = np.zeros((T, H), np.uint16)
     if P == 0:
         y_bits = np.zeros((1, H), np.uint16)
-    rc = _load().oracle_combine(_p(y_bits), P, _p(w), _p(dst_row), T, k, H, _p(out))
+    rc = _load().oracle_combine(_p(y_bits), P, _p(w), _p(dst_row), T, k, H, DTYPES[dtype],
+                                _p(out))
     if rc != OK:
         raise OracleError(rc, "oracle_combine")
     return out
@@ -322,7 +353,8 @@ def zero_pad_rows(recv_src: np.ndarray, rows: np.ndarray) -> np.ndarray:
     return out
 
 
-def dispatch_fp8_mn(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int, ld: int):
+def dispatch_fp8_mn(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int, ld: int,
+                    dtype: str = "bf16"):
     """FP8 dispatch with MN-major scales: (recv_q [P, H], scales_mn [H/128, ld])."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
@@ -330,8 +362,8 @@ def dispatch_fp8_mn(x_bits: np.ndarray, dst_row: np.ndarray, recv_rows: int, ld:
     k = dst_row.shape[1]
     q = np.zeros((max(recv_rows, 1), H), np.uint8)
     s = np.zeros((H // 128, max(ld, 1)), np.float32)
-    rc = _load().oracle_dispatch_fp8_mn(_p(x_bits), T, k, H, _p(dst_row), _p(q), _p(s), ld,
-                                        recv_rows)
+    rc = _load().oracle_dispatch_fp8_mn(_p(x_bits), T, k, H, DTYPES[dtype], _p(dst_row), _p(q),
+                                        _p(s), ld, recv_rows)
     if rc != OK:
         raise OracleError(rc, "oracle_dispatch_fp8_mn")
     return q[:recv_rows], s[:, :ld]

@@ -77,6 +77,86 @@ uint16_t oracle_f32_to_bf16_rn(float f)
     return (uint16_t)kept;
 }
 
+/* IEEE-754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
+ * bits; exponent field 0 holds zero and the subnormals m * 2^-24; field 31
+ * holds the infinities (fraction 0) and NaNs.  Widening is exact. */
+float oracle_fp16_to_f32(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int ex = (h >> 10) & 0x1f;
+    int man = h & 0x3ff;
+    double v;
+    if (ex == 0x1f)
+        v = man ? NAN : INFINITY;
+    else if (ex == 0)
+        v = ldexp((double)man, -24);
+    else
+        v = ldexp(1.0 + man / 1024.0, ex - 15);
+    return (float)(sign ? -v : v);
+}
+
+/* binary32 -> binary16, round to nearest, ties to even.  Magnitudes are
+ * rounded on the binary16 grid: spacing 2^-24 below 2^-14 (subnormals) and
+ * 2^(floor(log2 a) - 10) above; a result of 2^16 or more (any a >= 65520,
+ * the midpoint between 65504 and 2^16) overflows to infinity.  NaN stays NaN
+ * (quiet, sign kept). */
+uint16_t oracle_f32_to_fp16_rn(float f)
+{
+    uint16_t sign = signbit(f) ? 0x8000 : 0x0000;
+    if (isnan(f))
+        return (uint16_t)(sign | 0x7e00);
+    double a = fabs((double)f);
+    if (isinf(f))
+        return (uint16_t)(sign | 0x7c00);
+    double step;
+    int e2 = 0;
+    if (a < ldexp(1.0, -14)) {
+        step = ldexp(1.0, -24);
+    } else {
+        (void)frexp(a, &e2);                /* a = f * 2^e2, f in [0.5, 1) */
+        step = ldexp(1.0, (e2 - 1) - 10);   /* binade [2^(e2-1), 2^e2) */
+    }
+    double q = a / step;                    /* exact */
+    double n = floor(q);
+    double rem = q - n;
+    if (rem > 0.5 || (rem == 0.5 && fmod(n, 2.0) != 0.0))
+        n += 1.0;
+    double r = n * step;
+    if (r >= 65536.0)
+        return (uint16_t)(sign | 0x7c00);
+    if (r < ldexp(1.0, -14))                /* zero or subnormal */
+        return (uint16_t)(sign | (uint16_t)(r / ldexp(1.0, -24)));
+    int er = 0;
+    double fr = frexp(r, &er);              /* r = fr * 2^er, fr in [0.5, 1) */
+    int ex = (er - 1) + 15;
+    int man = (int)((fr * 2.0 - 1.0) * 1024.0);
+    return (uint16_t)(sign | (ex << 10) | man);
+}
+
+void oracle_fp16_to_f32_array(const uint16_t* h, float* v, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        v[i] = oracle_fp16_to_f32(h[i]);
+}
+
+void oracle_f32_to_fp16_array(const float* v, uint16_t* h, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        h[i] = oracle_f32_to_fp16_rn(v[i]);
+}
+
+/* A 16-bit input value of the given type (0 = bfloat16, 1 = binary16) as
+ * binary32, and binary32 rounded to it. */
+static float in16_to_f32(uint16_t v, int dtype)
+{
+    return dtype == 1 ? oracle_fp16_to_f32(v) : oracle_bf16_to_f32(v);
+}
+
+static uint16_t f32_to_out16(float f, int dtype)
+{
+    return dtype == 1 ? oracle_f32_to_fp16_rn(f) : oracle_f32_to_bf16_rn(f);
+}
+
 /* OCP 8-bit floating point, E4M3 ("fn" variant): 1 sign bit, 4 exponent
  * bits with bias 7, 3 mantissa bits; no infinities; S.1111.111 is NaN, so
  * the largest finite magnitude is 1.75 * 2^8 = 448.  Exponent field 0
@@ -306,13 +386,15 @@ int oracle_dispatch_bf16(const uint16_t* x, int64_t T, int k, int64_t H,
 /* FP8 quantisation of one token: H/128 blocks of 128 channels; per block
  * amax = max |x|, s = amax / 448 (fp32 division), q = e4m3(x / s) (fp32
  * division, then round-to-nearest-even with saturation); amax == 0 gives
- * s = 0 and q = +0 for the whole block. */
-void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, uint8_t* q, float* scales)
+ * s = 0 and q = +0 for the whole block.  x holds bfloat16 (dtype 0) or
+ * binary16 (dtype 1) values, widened exactly to binary32. */
+void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, int dtype, uint8_t* q,
+                               float* scales)
 {
     for (int64_t b = 0; b < H / 128; ++b) {
         float amax = 0.0f;
         for (int i = 0; i < 128; ++i) {
-            float v = fabsf(oracle_bf16_to_f32(x[b * 128 + i]));
+            float v = fabsf(in16_to_f32(x[b * 128 + i], dtype));
             if (v > amax)
                 amax = v;
         }
@@ -325,7 +407,7 @@ void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, uint8_t* q, float* 
         float s = amax / 448.0f;
         scales[b] = s;
         for (int i = 0; i < 128; ++i) {
-            float v = oracle_bf16_to_f32(x[b * 128 + i]) / s;
+            float v = in16_to_f32(x[b * 128 + i], dtype) / s;
             q[b * 128 + i] = oracle_f32_to_e4m3_rn_sat(v);
         }
     }
@@ -333,7 +415,7 @@ void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, uint8_t* q, float* 
 
 /* FP8 dispatch: every used slot (t, j) receives the e4m3 row of x[t] and
  * its H/128 fp32 scales (row-major [rows][H/128]). */
-int oracle_dispatch_fp8(const uint16_t* x, int64_t T, int k, int64_t H,
+int oracle_dispatch_fp8(const uint16_t* x, int64_t T, int k, int64_t H, int dtype,
                         const int32_t* dst_row, uint8_t* recv_q, float* recv_scales,
                         int64_t recv_cap)
 {
@@ -349,7 +431,7 @@ int oracle_dispatch_fp8(const uint16_t* x, int64_t T, int k, int64_t H,
     }
     int rc = OR_OK;
     for (int64_t t = 0; t < T && rc == OR_OK; ++t) {
-        oracle_quantize_token_fp8(x + t * H, H, q, s);
+        oracle_quantize_token_fp8(x + t * H, H, dtype, q, s);
         for (int j = 0; j < k; ++j) {
             int64_t d = dst_row[t * k + j];
             if (d < 0)
@@ -409,12 +491,14 @@ void oracle_expert_scale_fp8(const uint8_t* recv_q, const float* recv_scales,
 /* Combine.                                                             */
 /* ------------------------------------------------------------------ */
 
-/* out[t][h] = bf16_rn(acc), acc = 0; for j = 0..k-1 over used slots:
- * acc = fmaf(w[t][j], float(y[dst_row[t][j]][h]), acc).  The slot loop is
+/* out[t][h] = rn16(acc), acc = 0; for j = 0..k-1 over used slots:
+ * acc = fmaf(w[t][j], float(y[dst_row[t][j]][h]), acc); y and out are
+ * bfloat16 (dtype 0) or binary16 (dtype 1), rn16 the round-to-nearest-even
+ * into that type.  The slot loop is
  * the outer loop over a row of accumulators; each element still sees its
  * terms in slot order. */
 int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* dst_row,
-                   int64_t T, int k, int64_t H, uint16_t* out)
+                   int64_t T, int k, int64_t H, int dtype, uint16_t* out)
 {
     float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
     if (!acc)
@@ -432,10 +516,10 @@ int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int3
             }
             const float wj = w[t * k + j];
             for (int64_t h = 0; h < H; ++h)
-                acc[h] = fmaf(wj, oracle_bf16_to_f32(y[d * H + h]), acc[h]);
+                acc[h] = fmaf(wj, in16_to_f32(y[d * H + h], dtype), acc[h]);
         }
         for (int64_t h = 0; h < H; ++h)
-            out[t * H + h] = oracle_f32_to_bf16_rn(acc[h]);
+            out[t * H + h] = f32_to_out16(acc[h], dtype);
     }
     free(acc);
     return OR_OK;
@@ -543,7 +627,7 @@ void oracle_zero_pad_rows(const int32_t* recv_src, int64_t P, uint8_t* rows, int
 
 /* MN-major FP8 scales: the same scales as oracle_dispatch_fp8, stored as
  * scales_mn[b][row] with leading dimension ld (b = 128-channel block). */
-int oracle_dispatch_fp8_mn(const uint16_t* x, int64_t T, int k, int64_t H,
+int oracle_dispatch_fp8_mn(const uint16_t* x, int64_t T, int k, int64_t H, int dtype,
                            const int32_t* dst_row, uint8_t* recv_q, float* scales_mn,
                            int64_t ld, int64_t recv_cap)
 {
@@ -559,7 +643,7 @@ int oracle_dispatch_fp8_mn(const uint16_t* x, int64_t T, int k, int64_t H,
     }
     int rc = OR_OK;
     for (int64_t t = 0; t < T && rc == OR_OK; ++t) {
-        oracle_quantize_token_fp8(x + t * H, H, q, s);
+        oracle_quantize_token_fp8(x + t * H, H, dtype, q, s);
         for (int j = 0; j < k; ++j) {
             int64_t d = dst_row[t * k + j];
             if (d < 0)

@@ -20,8 +20,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-__all__ = ["CONFIGS", "Workload", "make_workload", "make_x", "route", "expert_scale_table",
-           "random_topk"]
+__all__ = ["CONFIGS", "Workload", "make_workload", "make_x", "make_x_fp16", "route",
+           "expert_scale_table", "random_topk"]
 
 # name -> shape and recipe.  fmt is the dispatch format; combine is BF16 always.
 CONFIGS = {
@@ -73,6 +73,12 @@ def _bf16_bits_rn(a: np.ndarray) -> np.ndarray:
 def make_x(T: int, H: int, rng: np.random.Generator) -> np.ndarray:
     """Hidden states: N(0,1) in fp32, rounded to bf16 (RN-even); returned as bits."""
     return _bf16_bits_rn(rng.standard_normal((T, H), dtype=np.float32))
+
+
+def make_x_fp16(T: int, H: int, rng: np.random.Generator) -> np.ndarray:
+    """Hidden states for FP16 inputs: N(0,1) in fp32, cast to IEEE binary16 by NumPy;
+    returned as bits."""
+    return rng.standard_normal((T, H), dtype=np.float32).astype(np.float16).view(np.uint16)
 
 
 def expert_scale_table(E: int, identity: bool = False) -> np.ndarray:
