@@ -49,7 +49,24 @@ EP_ERR_TIMEOUT = 9
 EP_FMT_BF16 = 0
 EP_FMT_FP8_E4M3_1X128 = 1
 EP_FMT_FP8_E4M3_1X128_MN = 2
-_FMTS = {"bf16": EP_FMT_BF16, "fp8": EP_FMT_FP8_E4M3_1X128, "fp8_mn": EP_FMT_FP8_E4M3_1X128_MN}
+EP_FMT_FP16 = 3
+_FMTS = {"bf16": EP_FMT_BF16, "fp8": EP_FMT_FP8_E4M3_1X128, "fp8_mn": EP_FMT_FP8_E4M3_1X128_MN,
+         "fp16": EP_FMT_FP16}
+EP_DTYPE_BF16 = 0
+EP_DTYPE_FP16 = 1
+_DTYPES = {torch.bfloat16: EP_DTYPE_BF16, torch.float16: EP_DTYPE_FP16}
+_COPY_FMT = {torch.bfloat16: EP_FMT_BF16, torch.float16: EP_FMT_FP16}
+
+
+def _fmt_code(fmt: Optional[str], dtype: torch.dtype) -> int:
+    """Format code; None or "copy" means the rows in the input's own 16-bit type."""
+    if fmt is None or fmt == "copy":
+        return _COPY_FMT[dtype]
+    return _FMTS[fmt]
+
+
+def _is_copy(f: int) -> bool:
+    return f in (EP_FMT_BF16, EP_FMT_FP16)
 
 VIEWS = {
     "num_tokens_per_expert": (0, torch.int32),
@@ -98,6 +115,8 @@ def load_library():
             "ep_handle_read_counts": ([P, P, P, P, P, P], I),
             "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
             "ep_combine": ([P, P, I64, P, I, P, P], I),
+            "ep_dispatch_ex": ([P, P, I, I, I, P, P, I64, P], I),
+            "ep_combine_ex": ([P, P, I64, P, I, I, P, P], I),
             "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
             "ep_dispatch_backward": ([P, P, I64, I, P, P], I),
             "ep_dispatch_weights": ([P, P, P, I64, P], I),
@@ -259,14 +278,13 @@ def _recv_buffers(h: EPHandle, T: int, H: int, f: int, device, recv_x, recv_scal
             ep_recv_rows_upper_bound(T, h.k, h.E, h.block_m)
         if f == EP_FMT_FP8_E4M3_1X128_MN:
             cap = (cap + 3) // 4 * 4
-        dt = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
-        recv_x = torch.empty((cap, H), dtype=dt, device=device)
+        recv_x = torch.empty((cap, H), dtype=_recv_dtype(f), device=device)
     cap = recv_x.shape[0]
     if f == EP_FMT_FP8_E4M3_1X128 and recv_scales is None:
         recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=device)
     if f == EP_FMT_FP8_E4M3_1X128_MN and recv_scales is None:
         recv_scales = torch.empty((H // 128, cap), dtype=torch.float32, device=device)
-    want = torch.bfloat16 if f == EP_FMT_BF16 else torch.float8_e4m3fn
+    want = _recv_dtype(f)
     if recv_x.dtype != want or recv_x.shape[1] != H or not recv_x.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "recv_x must be contiguous %s [*, %d]" % (want, H))
     if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128:
@@ -277,44 +295,62 @@ def _recv_buffers(h: EPHandle, T: int, H: int, f: int, device, recv_x, recv_scal
         if (recv_scales.dtype != torch.float32 or tuple(recv_scales.shape) != (H // 128, cap)
                 or not recv_scales.is_contiguous()):
             raise EPError(EP_ERR_INVALID_ARG, "recv_scales must be f32 [H/128, cap]")
-    return recv_x, (recv_scales if f != EP_FMT_BF16 else None)
+    return recv_x, (recv_scales if not _is_copy(f) else None)
 
 
-def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: str = "bf16",
+def _recv_dtype(f: int) -> torch.dtype:
+    return {EP_FMT_BF16: torch.bfloat16, EP_FMT_FP16: torch.float16}.get(f, torch.float8_e4m3fn)
+
+
+def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: Optional[str] = None,
                 recv_x: Optional[torch.Tensor] = None, recv_scales: Optional[torch.Tensor] = None,
                 capacity_rows: Optional[int] = None):
-    """Scatter bf16 x [T, H] into the receive layout.  Returns (recv_x, recv_scales);
-    recv_scales is None for BF16.  Buffers not given are allocated with
-    capacity_rows rows (default: the no-sync upper bound).  fmt: "bf16", "fp8"
+    """Scatter x [T, H] (bf16 or fp16) into the receive layout.  Returns
+    (recv_x, recv_scales); recv_scales is None for the row copies.  Buffers not
+    given are allocated with capacity_rows rows (default: the no-sync upper
+    bound).  fmt: None / "copy" (rows in x's type), "bf16", "fp16", "fp8"
     (row-major scales [cap, H/128]) or "fp8_mn" (MN-major scales [H/128, cap])."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_dispatch")
-    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != h.T or not x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: x must be contiguous bf16 [T, H]")
+    if (x.dtype not in _DTYPES or x.dim() != 2 or x.shape[0] != h.T
+            or not x.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: x must be contiguous bf16/fp16 [T, H]")
     T, H = x.shape
-    f = _FMTS[fmt]
+    f = _fmt_code(fmt, x.dtype)
+    if _is_copy(f) and f != _COPY_FMT[x.dtype]:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: a row copy keeps x's type")
     recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
+    lib = load_library()
     with _on(h):
-        _check(load_library().ep_dispatch(h.handle, _ptr(x), H, f, _ptr(recv_x),
-                                          _ptr(recv_scales), recv_x.shape[0],
-                                          _stream(h.device)), "ep_dispatch")
+        if x.dtype == torch.bfloat16:
+            _check(lib.ep_dispatch(h.handle, _ptr(x), H, f, _ptr(recv_x), _ptr(recv_scales),
+                                   recv_x.shape[0], _stream(h.device)), "ep_dispatch")
+        else:
+            _check(lib.ep_dispatch_ex(h.handle, _ptr(x), _DTYPES[x.dtype], H, f, _ptr(recv_x),
+                                      _ptr(recv_scales), recv_x.shape[0], _stream(h.device)),
+                   "ep_dispatch_ex")
     return recv_x, recv_scales
 
 
-def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor, fmt: str = "bf16",
+def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor,
+                       fmt: Optional[str] = None,
                        recv_x: Optional[torch.Tensor] = None,
                        recv_scales: Optional[torch.Tensor] = None,
                        capacity_rows: Optional[int] = None):
-    """ep_layout then ep_dispatch, in one launch for decode-sized batches."""
+    """ep_layout then ep_dispatch, in one launch for decode-sized batches (x bf16,
+    or fp16 copied as rows)."""
     if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or topk_idx.shape[1] != h.k:
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be int64 [T, %d]" % h.k)
     if not topk_idx.is_cuda or not topk_idx.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be contiguous CUDA")
     T = topk_idx.shape[0]
-    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != T or not x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: x must be contiguous bf16 [T, H]")
+    if x.dtype not in _DTYPES or x.dim() != 2 or x.shape[0] != T or not x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: x must be contiguous [T, H]")
     H = x.shape[1]
-    f = _FMTS[fmt]
+    f = _fmt_code(fmt, x.dtype)
+    if x.dtype == torch.float16 and f != EP_FMT_FP16:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: fp16 x takes the fp16 copy only; "
+                      "for FP8 of fp16 rows call ep_layout then ep_dispatch")
     recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
     with _on(h):
         _check(load_library().ep_layout_dispatch(
@@ -326,22 +362,29 @@ def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor, fmt
 
 def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,
                out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Weighted gather-reduce of bf16 y [rows, H] (receive layout) into bf16 [T, H]."""
+    """Weighted gather-reduce of y [rows, H] (receive layout; bf16 or fp16) into
+    out [T, H] of the same type."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_combine")
-    if y.dtype != torch.bfloat16 or y.dim() != 2 or not y.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: y must be contiguous bf16 [rows, H]")
+    if y.dtype not in _DTYPES or y.dim() != 2 or not y.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: y must be contiguous bf16/fp16 [rows, H]")
     if (topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (h.T, h.k)
             or not topk_weights.is_contiguous()):
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine: topk_weights must be f32 [T, k]")
     H = y.shape[1]
     if out is None:
-        out = torch.empty((h.T, H), dtype=torch.bfloat16, device=y.device)
-    if out.dtype != torch.bfloat16 or tuple(out.shape) != (h.T, H) or not out.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: out must be contiguous bf16 [T, H]")
+        out = torch.empty((h.T, H), dtype=y.dtype, device=y.device)
+    if out.dtype != y.dtype or tuple(out.shape) != (h.T, H) or not out.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine: out must be contiguous [T, H], y's type")
+    lib = load_library()
     with _on(h):
-        _check(load_library().ep_combine(h.handle, _ptr(y), y.shape[0], _ptr(topk_weights), H,
-                                         _ptr(out), _stream(h.device)), "ep_combine")
+        if y.dtype == torch.bfloat16:
+            _check(lib.ep_combine(h.handle, _ptr(y), y.shape[0], _ptr(topk_weights), H,
+                                  _ptr(out), _stream(h.device)), "ep_combine")
+        else:
+            _check(lib.ep_combine_ex(h.handle, _ptr(y), y.shape[0], _ptr(topk_weights), H,
+                                     _DTYPES[y.dtype], _ptr(out), _stream(h.device)),
+                   "ep_combine_ex")
     return out
 
 
@@ -352,16 +395,20 @@ def ep_dispatch_range(h: EPHandle, t_begin: int, x_rows: torch.Tensor, fmt: str,
     those tokens)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_dispatch_range")
-    if x_rows.dtype != torch.bfloat16 or x_rows.dim() != 2 or not x_rows.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: x_rows must be contiguous bf16 [n, H]")
-    f = _FMTS[fmt]
+    if x_rows.dtype not in _DTYPES or x_rows.dim() != 2 or not x_rows.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: x_rows must be contiguous [n, H]")
+    f = _fmt_code(fmt, x_rows.dtype)
+    if _is_copy(f) and f != _COPY_FMT[x_rows.dtype] or not _is_copy(f) and \
+            x_rows.dtype != torch.bfloat16:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: x_rows type and format disagree")
     n, H = x_rows.shape
     if recv_x.shape[1] != H or not recv_x.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: recv_x must be contiguous [*, H]")
     with _on(h):
         _check(load_library().ep_dispatch_range(
             h.handle, t_begin, n, _ptr(x_rows), H, f, _ptr(recv_x),
-            _ptr(recv_scales) if f else ctypes.c_void_p(0), recv_x.shape[0], _stream(h.device)),
+            _ptr(recv_scales) if not _is_copy(f) else ctypes.c_void_p(0), recv_x.shape[0],
+            _stream(h.device)),
             "ep_dispatch_range")
 
 

@@ -142,15 +142,21 @@ namespace {
 // layout: the kernels see a shallow copy of the handle whose token count and
 // dst_row start at the range.
 // Argument checks of a dispatch of t_count tokens (no launch).
-ep_status_t dispatch_check(int t_count, const void* x, int H, ep_fmt_t fmt, const void* recv_x,
-                           const float* recv_scales, int64_t recv_capacity_rows)
+ep_status_t dispatch_check(int t_count, const void* x, ep_dtype_t x_dtype, int H, ep_fmt_t fmt,
+                           const void* recv_x, const float* recv_scales,
+                           int64_t recv_capacity_rows)
 {
     if (H <= 0 || recv_capacity_rows < 0)
         return EP_ERR_INVALID_ARG;
-    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
-    if (fmt != EP_FMT_BF16 && !fp8)
+    if (x_dtype != EP_DTYPE_BF16 && x_dtype != EP_DTYPE_FP16)
         return EP_ERR_INVALID_ARG;
-    if (fmt == EP_FMT_BF16 && H % 8 != 0)
+    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
+    const bool copy = fmt == EP_FMT_BF16 || fmt == EP_FMT_FP16;
+    if (!copy && !fp8)
+        return EP_ERR_INVALID_ARG;
+    if (copy && (fmt == EP_FMT_FP16) != (x_dtype == EP_DTYPE_FP16))
+        return EP_ERR_INVALID_ARG;
+    if (copy && H % 8 != 0)
         return EP_ERR_INVALID_ARG;
     if (fp8 && H % 128 != 0)
         return EP_ERR_INVALID_ARG;
@@ -165,11 +171,17 @@ ep_status_t dispatch_check(int t_count, const void* x, int H, ep_fmt_t fmt, cons
     return EP_OK;
 }
 
+// The input type the formats of ep_dispatch imply: fp16 for the fp16 copy.
+ep_dtype_t implied_dtype(ep_fmt_t fmt)
+{
+    return fmt == EP_FMT_FP16 ? EP_DTYPE_FP16 : EP_DTYPE_BF16;
+}
+
 // Dispatch / combine of the tokens [t_begin, t_begin + t_count) of the last
 // layout: the kernels see a shallow copy of the handle whose token count and
 // dst_row start at the range.
-ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, int H,
-                          ep_fmt_t fmt, void* recv_x, float* recv_scales,
+ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, ep_dtype_t x_dtype,
+                          int H, ep_fmt_t fmt, void* recv_x, float* recv_scales,
                           int64_t recv_capacity_rows, void* stream, const char* what)
 {
     if (!h)
@@ -179,19 +191,20 @@ ep_status_t dispatch_impl(Handle* h, int t_begin, int t_count, const void* x, in
     if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
         return EP_ERR_INVALID_ARG;
     const ep_status_t st =
-        dispatch_check(t_count, x, H, fmt, recv_x, recv_scales, recv_capacity_rows);
+        dispatch_check(t_count, x, x_dtype, H, fmt, recv_x, recv_scales, recv_capacity_rows);
     if (st != EP_OK)
         return st;
     Handle sub = *h;
     sub.T = t_count;
     sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = (fmt == EP_FMT_BF16)
+    const bool copy = fmt == EP_FMT_BF16 || fmt == EP_FMT_FP16;
+    cudaError_t rc = copy  // a 2-byte row copy, whatever the 16-bit type
                          ? ep::launch_dispatch_bf16(sub, x, H, recv_x, recv_capacity_rows, s)
                          : ep::launch_dispatch_fp8(
                                sub, x, H, recv_x, recv_scales,
                                fmt == EP_FMT_FP8_E4M3_1X128_MN ? recv_capacity_rows : 0,
-                               recv_capacity_rows, s);
+                               recv_capacity_rows, x_dtype == EP_DTYPE_FP16, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
 }
 
@@ -218,10 +231,12 @@ ep_status_t clear_error_words_once(Handle* h, cudaStream_t s)
 }
 
 ep_status_t combine_impl(Handle* h, int t_begin, int t_count, const void* y, int64_t y_rows,
-                         const float* topk_weights, int H, void* out, void* stream,
-                         const char* what)
+                         const float* topk_weights, int H, ep_dtype_t dtype, void* out,
+                         void* stream, const char* what)
 {
     if (!h || H <= 0 || H % 8 != 0 || y_rows < 0)
+        return EP_ERR_INVALID_ARG;
+    if (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16)
         return EP_ERR_INVALID_ARG;
     if (!h->has_layout)
         return EP_ERR_STATE;
@@ -235,7 +250,8 @@ ep_status_t combine_impl(Handle* h, int t_begin, int t_count, const void* y, int
     sub.T = t_count;
     sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = ep::launch_combine(sub, y, y_rows, topk_weights, H, out, s);
+    cudaError_t rc = ep::launch_combine(sub, y, y_rows, topk_weights, H, out,
+                                        dtype == EP_DTYPE_FP16, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, what);
 }
 
@@ -342,10 +358,12 @@ ep_status_t ep_layout_dispatch(ep_handle_t hh, const int64_t* topk_idx, int T, c
     ep_status_t st = layout_check(h, topk_idx, T);
     if (st != EP_OK)
         return st;
-    if ((st = dispatch_check(T, x, H, fmt, recv_x, recv_scales, recv_capacity_rows)) != EP_OK)
+    const ep_dtype_t x_dtype = implied_dtype(fmt);
+    if ((st = dispatch_check(T, x, x_dtype, H, fmt, recv_x, recv_scales, recv_capacity_rows)) !=
+        EP_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool fp8 = fmt != EP_FMT_BF16;
+    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128 || fmt == EP_FMT_FP8_E4M3_1X128_MN;
     const bool v32 = H % 16 == 0 && ep::aligned(x, 32) && (fp8 || ep::aligned(recv_x, 32));
     if (T > 0 && v32 && ep::fused_layout_dispatch_fits(*h, T)) {
         if ((st = clear_error_words_once(h, s)) != EP_OK)
@@ -363,8 +381,8 @@ ep_status_t ep_layout_dispatch(ep_handle_t hh, const int64_t* topk_idx, int T, c
     }
     if ((st = ep_layout(hh, topk_idx, T, stream)) != EP_OK)
         return st;
-    return dispatch_impl(h, 0, T, x, H, fmt, recv_x, recv_scales, recv_capacity_rows, stream,
-                         "ep_layout_dispatch");
+    return dispatch_impl(h, 0, T, x, x_dtype, H, fmt, recv_x, recv_scales, recv_capacity_rows,
+                         stream, "ep_layout_dispatch");
 }
 
 const void* ep_handle_view(ep_handle_t hh, ep_view_t what, int64_t* count)
@@ -427,24 +445,41 @@ ep_status_t ep_dispatch(ep_handle_t hh, const void* x, int H, ep_fmt_t fmt, void
                         float* recv_scales, int64_t recv_capacity_rows, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    return dispatch_impl(h, 0, h ? std::max(h->T, 0) : 0, x, H, fmt, recv_x, recv_scales,
-                         recv_capacity_rows, stream, "ep_dispatch");
+    return dispatch_impl(h, 0, h ? std::max(h->T, 0) : 0, x, implied_dtype(fmt), H, fmt, recv_x,
+                         recv_scales, recv_capacity_rows, stream, "ep_dispatch");
+}
+
+ep_status_t ep_dispatch_ex(ep_handle_t hh, const void* x, ep_dtype_t x_dtype, int H, ep_fmt_t fmt,
+                           void* recv_x, float* recv_scales, int64_t recv_capacity_rows,
+                           void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    return dispatch_impl(h, 0, h ? std::max(h->T, 0) : 0, x, x_dtype, H, fmt, recv_x,
+                         recv_scales, recv_capacity_rows, stream, "ep_dispatch_ex");
 }
 
 ep_status_t ep_dispatch_range(ep_handle_t hh, int t_begin, int t_count, const void* x_rows,
                               int H, ep_fmt_t fmt, void* recv_x, float* recv_scales,
                               int64_t recv_capacity_rows, void* stream)
 {
-    return dispatch_impl(ep::as_handle(hh), t_begin, t_count, x_rows, H, fmt, recv_x,
-                         recv_scales, recv_capacity_rows, stream, "ep_dispatch_range");
+    return dispatch_impl(ep::as_handle(hh), t_begin, t_count, x_rows, implied_dtype(fmt), H, fmt,
+                         recv_x, recv_scales, recv_capacity_rows, stream, "ep_dispatch_range");
 }
 
 ep_status_t ep_combine(ep_handle_t hh, const void* y, int64_t y_rows, const float* topk_weights,
                        int H, void* out, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    return combine_impl(h, 0, h ? std::max(h->T, 0) : 0, y, y_rows, topk_weights, H, out, stream,
-                        "ep_combine");
+    return combine_impl(h, 0, h ? std::max(h->T, 0) : 0, y, y_rows, topk_weights, H,
+                        EP_DTYPE_BF16, out, stream, "ep_combine");
+}
+
+ep_status_t ep_combine_ex(ep_handle_t hh, const void* y, int64_t y_rows, const float* topk_weights,
+                          int H, ep_dtype_t dtype, void* out, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    return combine_impl(h, 0, h ? std::max(h->T, 0) : 0, y, y_rows, topk_weights, H, dtype, out,
+                        stream, "ep_combine_ex");
 }
 
 ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const void* y,
@@ -452,7 +487,7 @@ ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const voi
                              void* out_rows, void* stream)
 {
     return combine_impl(ep::as_handle(hh), t_begin, t_count, y, y_rows, topk_weights_rows, H,
-                        out_rows, stream, "ep_combine_range");
+                        EP_DTYPE_BF16, out_rows, stream, "ep_combine_range");
 }
 
 ep_status_t ep_dispatch_weights(ep_handle_t hh, const float* topk_weights, float* recv_weights,
@@ -501,7 +536,7 @@ ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t 
     if (!ep::aligned(grad_recv, 16) || !ep::aligned(grad_x, 16))
         return EP_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = ep::launch_combine(*h, grad_recv, grad_rows, nullptr, H, grad_x, s);
+    cudaError_t rc = ep::launch_combine(*h, grad_recv, grad_rows, nullptr, H, grad_x, false, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_backward");
 }
 

@@ -8,7 +8,8 @@
 // batch x top_k x hidden x sizeof(dtype) bytes as dispatch ("DeepEP 编址服务
 // 深度对抗分析", section 五.2).  Reduction semantics (stated in ep.h): fp32
 // accumulator, one fused multiply-add per used slot in slot order
-// j = 0..k-1, round-to-nearest-even to bf16 at the end.
+// j = 0..k-1, round-to-nearest-even to bf16 (or, for FP16 expert outputs,
+// to binary16) at the end.
 //
 // With a null weight pointer every weight is 1 (fma(1, y, acc) rounds like
 // acc + y): that is the backward of dispatch, grad_x[t] = sum of the k rows.
@@ -18,8 +19,6 @@
 // slot of the token is used and in range (the common case), all k x U loads
 // of a lane are issued before the first multiply-add; the chain itself is
 // still evaluated in slot order.
-#include <cuda_bf16.h>
-
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -29,29 +28,20 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 256;
 constexpr int kU = 2;  // 16-byte vectors per lane per unit
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
+template <bool kHalf>
 __device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4& v)
 {
-    acc[0] = __fmaf_rn(w, bf16_lo(v.x), acc[0]);
-    acc[1] = __fmaf_rn(w, bf16_hi(v.x), acc[1]);
-    acc[2] = __fmaf_rn(w, bf16_lo(v.y), acc[2]);
-    acc[3] = __fmaf_rn(w, bf16_hi(v.y), acc[3]);
-    acc[4] = __fmaf_rn(w, bf16_lo(v.z), acc[4]);
-    acc[5] = __fmaf_rn(w, bf16_hi(v.z), acc[5]);
-    acc[6] = __fmaf_rn(w, bf16_lo(v.w), acc[6]);
-    acc[7] = __fmaf_rn(w, bf16_hi(v.w), acc[7]);
+    acc[0] = __fmaf_rn(w, lo16<kHalf>(v.x), acc[0]);
+    acc[1] = __fmaf_rn(w, hi16<kHalf>(v.x), acc[1]);
+    acc[2] = __fmaf_rn(w, lo16<kHalf>(v.y), acc[2]);
+    acc[3] = __fmaf_rn(w, hi16<kHalf>(v.y), acc[3]);
+    acc[4] = __fmaf_rn(w, lo16<kHalf>(v.z), acc[4]);
+    acc[5] = __fmaf_rn(w, hi16<kHalf>(v.z), acc[5]);
+    acc[6] = __fmaf_rn(w, lo16<kHalf>(v.w), acc[6]);
+    acc[7] = __fmaf_rn(w, hi16<kHalf>(v.w), acc[7]);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    return a | (b << 16);
-}
-
-template <int KMAX>
+template <int KMAX, bool kHalf>
 __device__ __forceinline__ void combine_unit_all_valid(const uint4* __restrict__ y, int64_t vpr,
                                                        int k, int d, float w, int64_t v0,
                                                        float (&acc)[kU][8])
@@ -76,11 +66,12 @@ __device__ __forceinline__ void combine_unit_all_valid(const uint4* __restrict__
 #pragma unroll
             for (int i = 0; i < kU; ++i)
                 if (v0 + 32 * i < vpr)
-                    fma8(acc[i], wj, v[j][i]);
+                    fma8<kHalf>(acc[i], wj, v[j][i]);
         }
     }
 }
 
+template <bool kHalf>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restrict__ weights,
                int T, int k, int64_t vpr, const int32_t* __restrict__ dst_row,
@@ -117,7 +108,7 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
             for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
 
         if (all_valid && k <= 8) {
-            combine_unit_all_valid<8>(y, vpr, k, d, w, v0, acc);
+            combine_unit_all_valid<8, kHalf>(y, vpr, k, d, w, v0, acc);
         } else {
             for (int j = 0; j < k; ++j) {
                 const int dj = __shfl_sync(kFull, d, j);
@@ -133,7 +124,7 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
 #pragma unroll
                 for (int i = 0; i < kU; ++i)
                     if (v0 + 32 * i < vpr)
-                        fma8(acc[i], wj, v[i]);
+                        fma8<kHalf>(acc[i], wj, v[i]);
             }
         }
 
@@ -142,10 +133,10 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
         for (int i = 0; i < kU; ++i)
             if (v0 + 32 * i < vpr) {
                 uint4 r;
-                r.x = pack_bf16x2(acc[i][0], acc[i][1]);
-                r.y = pack_bf16x2(acc[i][2], acc[i][3]);
-                r.z = pack_bf16x2(acc[i][4], acc[i][5]);
-                r.w = pack_bf16x2(acc[i][6], acc[i][7]);
+                r.x = pack16x2<kHalf>(acc[i][0], acc[i][1]);
+                r.y = pack16x2<kHalf>(acc[i][2], acc[i][3]);
+                r.z = pack16x2<kHalf>(acc[i][4], acc[i][5]);
+                r.w = pack16x2<kHalf>(acc[i][6], acc[i][7]);
                 o[v0 + 32 * i] = r;
             }
     }
@@ -154,16 +145,17 @@ combine_kernel(const uint4* __restrict__ y, int64_t y_rows, const float* __restr
 }  // namespace
 
 cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
-                           int H, void* out, cudaStream_t s)
+                           int H, void* out, bool half, cudaStream_t s)
 {
     if (h.T == 0)
         return cudaSuccess;
+    auto kern = half ? combine_kernel<true> : combine_kernel<false>;
     int grid = 0;
-    cudaError_t rc = persistent_grid((const void*)combine_kernel, kThreads, 0, 8, &grid);
+    cudaError_t rc = persistent_grid((const void*)kern, kThreads, 0, 8, &grid);
     if (rc != cudaSuccess)
         return rc;
-    return launch_pdl(combine_kernel, grid, kThreads, 0, s, static_cast<const uint4*>(y), y_rows, w,
-                      h.T, h.k, (int64_t)H / 8, h.dst_row, static_cast<uint4*>(out), h.err);
+    return launch_pdl(kern, grid, kThreads, 0, s, static_cast<const uint4*>(y), y_rows, w, h.T,
+                      h.k, (int64_t)H / 8, h.dst_row, static_cast<uint4*>(out), h.err);
 }
 
 }  // namespace ep

@@ -1,6 +1,6 @@
 // ep_dispatch.cu -- dispatch on sm_100a: scatter of token rows into the
-// expert-major receive buffer, as a BF16 copy or with fused FP8 e4m3 1x128
-// quantisation.
+// expert-major receive buffer, as a copy of the 16-bit rows (BF16 or FP16)
+// or with fused FP8 e4m3 1x128 quantisation of BF16 or FP16 rows.
 //
 // Dispatch sends every token to its top-k experts ("DeepEP是什麼？MoE
 // Dispatch、Combine、All-to-all與V2架構", stage table of section
@@ -111,8 +111,6 @@ dispatch_bf16_kernel(const uint4* __restrict__ x, int T, int k, int64_t vpr,
     }
 }
 
-using units::bf16_hi;
-using units::bf16_lo;
 using units::e4m3x4;
 using units::scale_index;
 
@@ -121,6 +119,7 @@ using units::scale_index;
 // lanes 16-31 block 2i + 1; the block amax is a 16-lane xor reduction.  The
 // 8 scales of a unit are gathered into lanes 0-7 and written as one 32-byte
 // run per destination row.
+template <bool kHalf>
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
                     const int32_t* __restrict__ dst_row, uint8_t* __restrict__ recv_q,
@@ -156,8 +155,9 @@ dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
         float sc[kU];
 #pragma unroll
         for (int i = 0; i < kU; ++i) {
-            float f[8] = {bf16_lo(a[i].x), bf16_hi(a[i].x), bf16_lo(a[i].y), bf16_hi(a[i].y),
-                          bf16_lo(a[i].z), bf16_hi(a[i].z), bf16_lo(a[i].w), bf16_hi(a[i].w)};
+            float f[8] = {lo16<kHalf>(a[i].x), hi16<kHalf>(a[i].x), lo16<kHalf>(a[i].y),
+                          hi16<kHalf>(a[i].y), lo16<kHalf>(a[i].z), hi16<kHalf>(a[i].z),
+                          lo16<kHalf>(a[i].w), hi16<kHalf>(a[i].w)};
             float m = 0.0f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) m = fmaxf(m, fabsf(f[c]));
@@ -208,6 +208,7 @@ dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
 
 
 // FP8 with 32-byte input vectors (units::fp8_unit); vpr = H / 16.
+template <bool kHalf>
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                         const int32_t* __restrict__ dst_row, uint8_t* __restrict__ recv_q,
@@ -229,7 +230,8 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
             atomicOr(err, kErrDispatchCap);
             d = -1;
         }
-        units::fp8_unit(x + t * vpr, vpr, u - t * upr, d, k, H, recv_q, recv_scales, scales_ld);
+        units::fp8_unit<units::kU32Fp8, kHalf>(x + t * vpr, vpr, u - t * upr, d, k, H, recv_q,
+                                               recv_scales, scales_ld);
     }
 }
 
@@ -261,16 +263,19 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
 
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
                                 float* recv_scales, int64_t scales_ld, int64_t cap_rows,
-                                cudaStream_t s)
+                                bool half, cudaStream_t s)
 {
     if (h.T == 0)
         return cudaSuccess;
-    if (aligned32(x))
-        return launch_pdl(dispatch_fp8_v32_kernel, unit_grid(h.T, H / 16, kUnitVec32Fp8),
-                          kThreads, 0, s, static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row,
+    if (aligned32(x)) {
+        auto kern = half ? dispatch_fp8_v32_kernel<true> : dispatch_fp8_v32_kernel<false>;
+        return launch_pdl(kern, unit_grid(h.T, H / 16, kUnitVec32Fp8), kThreads, 0, s,
+                          static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row,
                           static_cast<uint8_t*>(recv_q), recv_scales, scales_ld, cap_rows,
                           h.err);
-    return launch_pdl(dispatch_fp8_kernel, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
+    }
+    auto kern = half ? dispatch_fp8_kernel<true> : dispatch_fp8_kernel<false>;
+    return launch_pdl(kern, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
                       static_cast<const uint4*>(x), h.T, h.k, H, h.dst_row,
                       static_cast<uint8_t*>(recv_q), recv_scales, scales_ld, cap_rows, h.err);
 }

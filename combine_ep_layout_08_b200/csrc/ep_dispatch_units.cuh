@@ -113,8 +113,9 @@ __device__ __forceinline__ void fp8_load(const Vec32* __restrict__ xs, int64_t v
     }
 }
 
-// Quantise the loaded vectors and write codes and scales to the k rows.
-template <int kU>
+// Quantise the loaded vectors (bfloat16, or binary16 when kHalf) and write
+// codes and scales to the k rows.
+template <int kU, bool kHalf = false>
 __device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int64_t unit, int d,
                                           int k, int H, uint8_t* __restrict__ recv_q,
                                           float* __restrict__ recv_scales, int64_t scales_ld)
@@ -129,8 +130,8 @@ __device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int
         float f[16];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            f[2 * c] = bf16_lo(a[i].w[c]);
-            f[2 * c + 1] = bf16_hi(a[i].w[c]);
+            f[2 * c] = lo16<kHalf>(a[i].w[c]);
+            f[2 * c + 1] = hi16<kHalf>(a[i].w[c]);
         }
         float m = 0.0f;
 #pragma unroll
@@ -182,14 +183,14 @@ __device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int
     }
 }
 
-template <int kU = kU32Fp8>
+template <int kU = kU32Fp8, bool kHalf = false>
 __device__ __forceinline__ void fp8_unit(const Vec32* __restrict__ xs, int64_t vpr, int64_t unit,
                                          int d, int k, int H, uint8_t* __restrict__ recv_q,
                                          float* __restrict__ recv_scales, int64_t scales_ld)
 {
     Vec32 a[kU];
     fp8_load<kU>(xs, vpr, unit, a);
-    fp8_store<kU>(a, vpr, unit, d, k, H, recv_q, recv_scales, scales_ld);
+    fp8_store<kU, kHalf>(a, vpr, unit, d, k, H, recv_q, recv_scales, scales_ld);
 }
 
 }  // namespace units

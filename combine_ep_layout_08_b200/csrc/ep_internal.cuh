@@ -4,6 +4,8 @@
 // each kernel file exports to the C-ABI layer (ep_api.cu).
 #pragma once
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -63,6 +65,42 @@ bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c)
 // completed and its memory is visible -- and then pdl_trigger(), which lets
 // the next kernel's CTAs be scheduled while this one drains.  Nothing is
 // read or written before pdl_wait(), so a kernel may follow any other work.
+// 16-bit input values packed two to a 32-bit word: bfloat16 (kHalf = false,
+// the upper half of a binary32, widened by a shift) or IEEE binary16
+// (kHalf = true, widened exactly by the conversion instruction); and binary32
+// rounded to nearest even into that type.
+template <bool kHalf>
+__device__ __forceinline__ float lo16(uint32_t w)
+{
+    if constexpr (kHalf)
+        return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+    else
+        return __uint_as_float(w << 16);
+}
+
+template <bool kHalf>
+__device__ __forceinline__ float hi16(uint32_t w)
+{
+    if constexpr (kHalf)
+        return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    else
+        return __uint_as_float(w & 0xffff0000u);
+}
+
+template <bool kHalf>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi)
+{
+    uint32_t a, b;
+    if constexpr (kHalf) {
+        a = __half_as_ushort(__float2half_rn(lo));
+        b = __half_as_ushort(__float2half_rn(hi));
+    } else {
+        a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+        b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    }
+    return a | (b << 16);
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
 
@@ -98,13 +136,15 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
                                  int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* recv_q,
                                 float* recv_scales, int64_t scales_ld, int64_t cap_rows,
-                                cudaStream_t s);  // scales_ld 0: row-major scales
+                                bool half, cudaStream_t s);  // scales_ld 0: row-major scales;
+                                                             // half: x is binary16
 cudaError_t launch_dispatch_weights(const Handle& h, const float* w, float* recv_w,
                                     int64_t cap_rows, cudaStream_t s);
 cudaError_t launch_zero_pad_rows(const Handle& h, void* rows, int64_t row_bytes, int64_t cap_rows,
                                  cudaStream_t s);
 cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const float* w,
-                           int H, void* out, cudaStream_t s);  // w == nullptr: unit weights
+                           int H, void* out, bool half,
+                           cudaStream_t s);  // w == nullptr: unit weights; half: y, out binary16
 cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
                                     int64_t y_rows, const float* w, int H, void* grad_y,
                                     int64_t grad_y_rows, float* grad_w, cudaStream_t s);

@@ -80,14 +80,23 @@ typedef enum {
                                         resets the barrier. */
 } ep_status_t;
 
+/* Element type of 16-bit hidden rows (x, y, out).  The yololab page lists
+ * BF16, FP16 and FP8 as dispatch data types ("DeepEP是什麼？…", section
+ * FP8與低精度通訊). */
+typedef enum {
+    EP_DTYPE_BF16 = 0,            /* bfloat16 */
+    EP_DTYPE_FP16 = 1             /* IEEE-754 binary16 */
+} ep_dtype_t;
+
 typedef enum {
     EP_FMT_BF16 = 0,              /* receive rows are the bf16 input rows */
     EP_FMT_FP8_E4M3_1X128 = 1,    /* e4m3 rows + one fp32 scale per 128 channels,
                                      scales row-major [rows][H/128] */
-    EP_FMT_FP8_E4M3_1X128_MN = 2  /* the same codes and scales, scales MN-major
+    EP_FMT_FP8_E4M3_1X128_MN = 2, /* the same codes and scales, scales MN-major
                                      [H/128][recv_capacity_rows]: each block's scales
                                      contiguous over rows (recv_capacity_rows % 4 == 0,
                                      so every block's column starts 16-byte aligned) */
+    EP_FMT_FP16 = 3               /* receive rows are the fp16 input rows */
 } ep_fmt_t;
 
 /* Views of the layout held in the workspace (see ep_handle_view). */
@@ -151,7 +160,7 @@ ep_status_t ep_layout(ep_handle_t h, const int64_t* topk_idx, int T, void* strea
  * latency matters most: "DeepEP是什麼？…", section 高吞吐與低延遲工作負載).
  * Same arguments, results and errors as ep_layout(h, topk_idx, T, stream)
  * followed by ep_dispatch(h, x, H, fmt, recv_x, recv_scales,
- * recv_capacity_rows, stream).  When the batch is small (T*k <= 4096,
+ * recv_capacity_rows, stream) (so x is bf16, or fp16 with EP_FMT_FP16).  When the batch is small (T*k <= 4096,
  * E <= 1024, T*R <= 65536) and rows take 32-byte vectors (H % 16 == 0; x,
  * and for BF16 recv_x, 32-byte aligned), both run in ONE launch: every CTA
  * computes the same layout in its shared memory, CTA 0 publishes it, and all
@@ -193,6 +202,18 @@ ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
 ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void* recv_x,
                         float* recv_scales, int64_t recv_capacity_rows, void* stream);
 
+/* ep_dispatch with the type of x named.  x_dtype EP_DTYPE_BF16: as
+ * ep_dispatch.  x_dtype EP_DTYPE_FP16: x is device binary16 [T][H];
+ * fmt EP_FMT_FP16 copies the rows (recv_x binary16 [recv_capacity_rows][H]);
+ * the FP8 formats quantise the binary16 values, widened exactly to fp32, with
+ * the same amax, scale and rounding as above.  A copy format must match
+ * x_dtype (EP_FMT_BF16 with bf16, EP_FMT_FP16 with fp16), else
+ * EP_ERR_INVALID_ARG.  ep_dispatch itself takes fp16 rows only with
+ * EP_FMT_FP16. */
+ep_status_t ep_dispatch_ex(ep_handle_t h, const void* x, ep_dtype_t x_dtype, int H, ep_fmt_t fmt,
+                           void* recv_x, float* recv_scales, int64_t recv_capacity_rows,
+                           void* stream);
+
 /* Combine into token order for the T tokens of the last layout.
  * y: device bf16 [y_rows][H] in the receive layout, 16-byte aligned, H % 8 == 0.
  * topk_weights: device fp32 [T][k], 4-byte aligned.
@@ -204,12 +225,19 @@ ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void*
 ep_status_t ep_combine(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
                        int H, void* out, void* stream);
 
+/* ep_combine with the type of y and out named: EP_DTYPE_BF16 is ep_combine;
+ * EP_DTYPE_FP16 reads binary16 expert outputs (widened exactly), accumulates
+ * in fp32 in the same order and rounds the result to nearest even binary16
+ * (sums beyond the binary16 range become infinities). */
+ep_status_t ep_combine_ex(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
+                          int H, ep_dtype_t dtype, void* out, void* stream);
+
 /* Dispatch / combine a contiguous range of the last layout's tokens,
  * [t_begin, t_begin + t_count), 0 <= t_begin <= t_begin + t_count <= T.
  * Same semantics, formats and errors as ep_dispatch / ep_combine restricted
  * to those tokens; x_rows, topk_weights_rows and out_rows point at the rows
- * of token t_begin (x_rows: bf16 [t_count][H]; topk_weights_rows: fp32
- * [t_count][k]; out_rows: bf16 [t_count][H]).  recv_x, recv_scales and y are
+ * of token t_begin (x_rows: bf16 [t_count][H], or fp16 with EP_FMT_FP16;
+ * topk_weights_rows: fp32 [t_count][k]; out_rows: bf16 [t_count][H]).  recv_x, recv_scales and y are
  * the whole receive-layout buffers.  The ranges of one layout may run in any
  * order and on different streams: they write disjoint rows.  This lets a
  * caller overlap the transfer of token chunks (host copies, or an upstream
