@@ -262,12 +262,15 @@ def time_gpu(s, steps, warmup, flush, barrier):
     return dict(layout=lay, dispatch=dis, combine=com, step=tot, wall=(t0, t1))
 
 
-def time_gpu_e2e(s, steps, warmup, chunks=8):
-    """The same step through the public API with host buffers: pinned H2D of
-    topk_idx, weights and x, the three calls, D2H of out -- all inside the
-    events.  The batch moves in `chunks` token ranges on three streams so that
-    H2D of later chunks, the kernels of earlier ones and D2H of finished ones
-    overlap (PCIe is full duplex); the layout waits for all of topk_idx."""
+def time_gpu_e2e(s, steps, warmup):
+    """The same step through the public API with host buffers, as a stream of
+    batches: every step copies topk_idx, weights and x from pinned host memory,
+    runs ep_layout, ep_dispatch and ep_combine, and copies out back to pinned
+    host memory.  Device staging is double-buffered so that step i's
+    device->host copy runs while step i+1's inputs come in (PCIe is full
+    duplex); the kernels of one step run between the two.  The timed region
+    spans all steps, pipeline fill (the first inputs alone) and drain (the last
+    result alone) included; the time per step is the total over steps."""
     import torch
 
     import combine_ep_layout_08_b200 as ep
@@ -276,64 +279,67 @@ def time_gpu_e2e(s, steps, warmup, chunks=8):
     hx = s["x"].cpu().pin_memory()
     hidx = s["idx"].cpu().pin_memory()
     hwt = s["wt"].cpu().pin_memory()
-    hout = torch.empty(s["out"].shape, dtype=torch.bfloat16).pin_memory()
-    dx = torch.empty_like(s["x"])
-    didx = torch.empty_like(s["idx"])
-    dwt = torch.empty_like(s["wt"])
-    h, out, y = s["h"], s["out"], s["y"]
+    hout = [torch.empty(s["out"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dx = [torch.empty_like(s["x"]) for _ in range(2)]
+    didx = [torch.empty_like(s["idx"]) for _ in range(2)]
+    dwt = [torch.empty_like(s["wt"]) for _ in range(2)]
+    dout = [torch.empty_like(s["out"]) for _ in range(2)]
+    h, y = s["h"], s["y"]
     main = torch.cuda.current_stream()
-    s_h2d, s_cmp, s_d2h = (torch.cuda.Stream(device=dx.device) for _ in range(3))
-    cuts = [w.T * i // chunks for i in range(chunks + 1)]
+    s_h2d, s_cmp, s_d2h = (torch.cuda.Stream(device=s["x"].device) for _ in range(3))
 
-    def one(a_ev, b_ev):
+    def run(n):
+        """n pipelined steps; returns the device time in ms (events on main)."""
+        a_ev = torch.cuda.Event(enable_timing=True)
+        b_ev = torch.cuda.Event(enable_timing=True)
         a_ev.record(main)
-        s_h2d.wait_stream(main)
-        s_cmp.wait_stream(main)
-        s_d2h.wait_stream(main)
-        with torch.cuda.stream(s_h2d):
-            didx.copy_(hidx, non_blocking=True)
-            dwt.copy_(hwt, non_blocking=True)
-            meta = torch.cuda.Event()
-            meta.record(s_h2d)
-            x_ev = []
-            for lo, hi in zip(cuts[:-1], cuts[1:]):
-                dx[lo:hi].copy_(hx[lo:hi], non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(s_h2d)
-                x_ev.append(e)
-        with torch.cuda.stream(s_cmp):
-            s_cmp.wait_event(meta)
-            ep.ep_layout(h, didx)
-            c_ev = []
-            for (lo, hi), e in zip(zip(cuts[:-1], cuts[1:]), x_ev):
-                s_cmp.wait_event(e)
-                ep.ep_dispatch_range(h, lo, dx[lo:hi], w.fmt, s["recv"], s["scales"])
-                ep.ep_combine_range(h, lo, y, dwt[lo:hi], out[lo:hi])
+        for st in (s_h2d, s_cmp, s_d2h):
+            st.wait_stream(main)
+        cmp_done, d2h_done = [], []
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(cmp_done[i - 2])    # buffer b read by step i-2
+                didx[b].copy_(hidx, non_blocking=True)
+                dwt[b].copy_(hwt, non_blocking=True)
+                dx[b].copy_(hx, non_blocking=True)
+                in_ev = torch.cuda.Event()
+                in_ev.record(s_h2d)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_ev)
+                if i >= 2:
+                    s_cmp.wait_event(d2h_done[i - 2])   # dout[b] copied out by step i-2
+                ep.ep_layout(h, didx[b])
+                ep.ep_dispatch(h, dx[b], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+                ep.ep_combine(h, y, dwt[b], out=dout[b])
                 ce = torch.cuda.Event()
                 ce.record(s_cmp)
-                c_ev.append(ce)
-        with torch.cuda.stream(s_d2h):
-            for (lo, hi), ce in zip(zip(cuts[:-1], cuts[1:]), c_ev):
+                cmp_done.append(ce)
+            with torch.cuda.stream(s_d2h):
                 s_d2h.wait_event(ce)
-                hout[lo:hi].copy_(out[lo:hi], non_blocking=True)
+                hout[b].copy_(dout[b], non_blocking=True)
+                de = torch.cuda.Event()
+                de.record(s_d2h)
+                d2h_done.append(de)
         main.wait_stream(s_d2h)
         main.wait_stream(s_cmp)
         b_ev.record(main)
+        b_ev.synchronize()
+        return a_ev.elapsed_time(b_ev)
 
-    for _ in range(warmup):
-        one(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    run(max(warmup, 3))
     torch.cuda.synchronize()
-    ts = []
-    for _ in range(steps):
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        one(a, b)
-        b.synchronize()
-        ts.append(a.elapsed_time(b))
+    total_ms = run(steps)
     h2d = hx.numel() * 2 + hidx.numel() * 8 + hwt.numel() * 4
-    d2h = hout.numel() * 2
-    assert torch.equal(hout, out.cpu()), "host copy of out differs"
-    return statistics.mean(ts), h2d, d2h
+    d2h = hout[0].numel() * 2
+    # the result the device-resident step gives, for the check of both host buffers
+    ep.ep_layout(h, s["idx"])
+    ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+    ep.ep_combine(h, y, s["wt"], out=s["out"])
+    ref = s["out"].cpu()
+    assert torch.equal(hout[0], ref) and torch.equal(hout[1], ref), "host copy of out differs"
+    return total_ms / steps, h2d, d2h
 
 
 def fused_step(s):
@@ -594,8 +600,12 @@ def main():
         e2e = {"value": round(world * (d_bytes + c_bytes) / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_ms, 4),
-               "how": "pinned host buffers; 8 token chunks on 3 streams (H2D | layout, "
-                      "dispatch_range, combine_range | D2H), all inside the events"}
+               "steps": max(3, min(args.steps, 50)),
+               "how": "a stream of steps through the Python API: pinned host x, topk_idx, "
+                      "weights in and out back every step; double-buffered device staging on "
+                      "3 streams (H2D | ep_layout, ep_dispatch, ep_combine | D2H) so that a "
+                      "step's D2H overlaps the next step's H2D; events span all steps incl. "
+                      "pipeline fill and drain"}
 
     secondary = {}
     if not args.no_secondary:
