@@ -55,6 +55,22 @@ __device__ __forceinline__ unsigned lanemask_lt()
     return m;
 }
 
+// Lanes of the warp whose key equals this lane's, for keys in [-1, 2^nbits - 1)
+// (nbits uniform over the warp): the AND over the key bits of the matching
+// ballot -- nbits ballots, where __match_any_sync slows down with the number
+// of distinct keys (up to 32 here).
+__device__ __forceinline__ unsigned match_key(int key, int nbits)
+{
+    const unsigned v = (unsigned)(key + 1);
+    unsigned m = kFull;
+    for (int b = 0; b < nbits; ++b) {
+        const unsigned bit = (v >> b) & 1u;
+        const unsigned bal = __ballot_sync(kFull, bit);
+        m &= bit ? bal : ~bal;
+    }
+    return m;
+}
+
 __device__ __forceinline__ int32_t pad_up(int32_t c, int32_t b) { return ((c + b - 1) / b) * b; }
 
 // An expert in [0, E), or -1 for an unused slot; anything else is flagged.
@@ -183,15 +199,17 @@ __device__ __forceinline__ void fill_pad(int32_t* recv_src, int32_t a, int32_t b
 // One warp: replay a chunk's entries (ents in smem, -1 unused) in order and
 // give each its row.  runc[e] holds the next free row of expert e for this
 // chunk and is advanced here.
-__device__ __forceinline__ void chunk_assign(const int32_t* ents, int nent, int k, int64_t t0,
-                                             int32_t* runc, int32_t* dst_row, int32_t* recv_src)
+__device__ __forceinline__ void chunk_assign(const int32_t* ents, int nent, int k, int E,
+                                             int64_t t0, int32_t* runc, int32_t* dst_row,
+                                             int32_t* recv_src)
 {
     const int lane = threadIdx.x & 31;
     const unsigned lt = lanemask_lt();
+    const int ebits = 32 - __clz((unsigned)E);  // keys e + 1 in [0, E]
     for (int g = 0; g < nent; g += 32) {
         const int f = g + lane;
-        const int e = f < nent ? ents[f] : -2;  // -2: lanes past the chunk end
-        const unsigned peers = __match_any_sync(kFull, e);
+        const int e = f < nent ? ents[f] : -1;  // lanes past the chunk end: no expert
+        const unsigned peers = match_key(e, ebits);
         int pos = -1;
         if (e >= 0)
             pos = runc[e] + __popc(peers & lt);
@@ -421,7 +439,7 @@ __global__ void layout_assign_kernel(const int64_t* __restrict__ topk_idx, int T
         return;  // no block barrier follows
     for (int e = lane; e < E; e += 32) runc[e] += off[e];
     __syncwarp();
-    chunk_assign(ents, nent, k, t0, runc, dst_row, recv_src);
+    chunk_assign(ents, nent, k, E, t0, runc, dst_row, recv_src);
 }
 
 // Small batches (T k <= kSmallEntries, E <= kSmallMaxE): CTAs of 1024
@@ -560,22 +578,6 @@ __device__ __forceinline__ int32_t exscan_u16x8(int4& v, int32_t acc)
     }
     v = make_int4((int)w[0], (int)w[1], (int)w[2], (int)w[3]);
     return acc;
-}
-
-// Lanes of the warp whose key equals this lane's, for keys in [-1, 2^nbits - 1)
-// (nbits uniform over the warp): the AND over the key bits of the matching
-// ballot -- nbits ballots, where __match_any_sync slows down with the number
-// of distinct keys (up to 32 here).
-__device__ __forceinline__ unsigned match_key(int key, int nbits)
-{
-    const unsigned v = (unsigned)(key + 1);
-    unsigned m = kFull;
-    for (int b = 0; b < nbits; ++b) {
-        const unsigned bit = (v >> b) & 1u;
-        const unsigned bal = __ballot_sync(kFull, bit);
-        m &= bit ? bal : ~bal;
-    }
-    return m;
 }
 
 // kFused = false: the layout alone.  kFused = true: then every warp of the
@@ -1080,9 +1082,11 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
     int32_t* cnt = wsum + 32;
     int32_t* tpre = cnt + E;
     int64_t tile = blockIdx.x;
-    for (int e = threadIdx.x; e < E; e += nthr) {
-        cnt[e] = cnt_g[e];
-        tpre[e] = tile_counts[tile * E + e];  // tile < ntiles: G <= ntiles
+    {
+        for (int e = threadIdx.x; e < E; e += nthr) {
+            cnt[e] = cnt_g[e];
+            tpre[e] = tile_counts[tile * E + e];  // tile < ntiles: G <= ntiles
+        }
     }
     if (!resident)
         (void)load_tile(tile, nullptr);
@@ -1123,7 +1127,7 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
         const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
         const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
         if (ntok > 0)
-            chunk_assign(ents, ntok * k, k, t0, run, dst_row, recv_src);
+            chunk_assign(ents, ntok * k, k, E, t0, run, dst_row, recv_src);
     }
 }
 
