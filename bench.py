@@ -239,27 +239,39 @@ def gpu_step(s, ev=None):
 
 
 def time_gpu(s, steps, warmup, flush, barrier):
-    """Per-step event timing; returns dict of per-kernel and per-step ms lists."""
+    """Device timing of `steps` steps, L2 flushed before each (outside the
+    events).  Two passes: the step time from events at the two ends of each
+    step only (events between kernels keep a kernel from starting while its
+    predecessor drains: ~6 us per step at 8k), then the per-kernel split from
+    a pass with events between the three kernels.  Returns per-step lists in
+    ms and the wall-clock window of both passes."""
     import torch
 
     for _ in range(warmup):
         flush()
         gpu_step(s)
+    ends = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     torch.cuda.synchronize()
     barrier()
     t0 = time.time()
     for i in range(steps):
         flush()
+        ends[i][0].record()
+        gpu_step(s)
+        ends[i][1].record()
+    for i in range(steps):
+        flush()
         gpu_step(s, evs[i])
     torch.cuda.synchronize()
     t1 = time.time()
     barrier()
+    tot = [e[0].elapsed_time(e[1]) for e in ends]
     lay = [e[0].elapsed_time(e[1]) for e in evs]
     dis = [e[1].elapsed_time(e[2]) for e in evs]
     com = [e[2].elapsed_time(e[3]) for e in evs]
-    tot = [e[0].elapsed_time(e[3]) for e in evs]
-    return dict(layout=lay, dispatch=dis, combine=com, step=tot, wall=(t0, t1))
+    split = [e[0].elapsed_time(e[3]) for e in evs]
+    return dict(layout=lay, dispatch=dis, combine=com, step=tot, step_split=split, wall=(t0, t1))
 
 
 def time_gpu_e2e(s, steps, warmup):
@@ -679,7 +691,11 @@ def main():
                         "dispatch_p50_p95_p99_us": [round(np.percentile(tm["dispatch"], q) * 1e3, 2)
                                                     for q in (50, 95, 99)],
                         "combine_p50_p95_p99_us": [round(np.percentile(tm["combine"], q) * 1e3, 2)
-                                                   for q in (50, 95, 99)]},
+                                                   for q in (50, 95, 99)],
+                        "split_step_us": round(statistics.mean(tm["step_split"]) * 1e3, 2),
+                        "note": "per-kernel times from a second pass of the same steps with "
+                                "events between the kernels (split_step_us is that pass's step); "
+                                "value and ms_per_step come from events at the step's ends only"},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
