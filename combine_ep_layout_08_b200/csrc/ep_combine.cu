@@ -18,7 +18,8 @@
 // unit: one warp x (token, 32 x U 16-byte vectors of the row).  When every
 // slot of the token is used and in range (the common case), all k x U loads
 // of a lane are issued before the first multiply-add; the chain itself is
-// still evaluated in slot order.
+// still evaluated in slot order.  The persistent grid and 512-channel units
+// measured best (one unit per warp, or 256-channel units, were slower).
 #include "ep_internal.cuh"
 
 namespace ep {

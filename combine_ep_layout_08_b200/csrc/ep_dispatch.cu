@@ -12,10 +12,12 @@
 //
 // Both kernels are HBM-bound streams (read 2H bytes per token, write k rows),
 // and dispatch is write-dominated (k row writes per row read).  Work unit: one
-// warp x (token, 2 KiB of bf16 input = 1024 channels); each lane loads its
-// vectors of the unit up front (x is read once: no L1 allocation), then
-// writes them to the k destination rows; consecutive lanes write consecutive
-// bytes of a row, so every store instruction covers whole 32-byte sectors.
+// warp x (token, 512 channels for the copy, 1024 channels = 8 FP8 blocks for
+// FP8); each lane loads its vectors of the unit up front (x is read once: no
+// L1 allocation), then writes them to the k destination rows; consecutive
+// lanes write consecutive bytes of a row, so every store instruction covers
+// whole 32-byte sectors.  (Halving the FP8 unit measured slower at every
+// batch size tried, 4096 and 8192 tokens.)
 // The main kernels move 32-byte vectors (sm_100's 256-bit ld/st.global.v8),
 // halving the store instructions of 16-byte vectors; 16-byte kernels remain
 // for rows that are not 32-byte multiples.  The grid gives every warp one

@@ -20,7 +20,7 @@
 //              (in place), per-expert totals and per-rank token totals;
 //   K3 assign  every CTA scans the padded expert sizes into expert_off; each
 //              warp replays its chunk in order, ranking equal experts inside
-//              each group of 32 entries with __match_any_sync, to give
+//              each group of 32 entries by lane (a ballot per key bit), to give
 //              dst_row and recv_src; pad rows of recv_src are set to -1.
 // Large batches, one launch (the default): layout_tile_kernel runs the three
 // phases in one cooperative launch over 64-token tiles, its CTAs separated by
