@@ -74,12 +74,37 @@ KERNEL_FILES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and whitespace (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            if not text[i].isspace():
+                out.append(text[i])
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_hash(kernel: str = "dispatch_bf16_v32_kernel"):
-    """Hash of the source files that make up a kernel (first 16 hex digits)."""
+    """Hash of the code (comments and whitespace dropped) of the source files
+    that make up a kernel (first 16 hex digits)."""
     h = hashlib.sha256()
     for name in KERNEL_FILES[kernel]:
-        with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "combine_ep_layout_08_b200", "csrc", name),
+                  encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -66,3 +66,13 @@ def test_kernel_hash_is_stable():
     for k in ("dispatch_bf16_v32_kernel", "combine_kernel"):
         assert bench.kernel_source_hash(k) == bench.kernel_source_hash(k)
         assert len(bench.kernel_source_hash(k)) == 16
+
+
+def test_kernel_hash_ignores_comments_and_whitespace():
+    import bench
+
+    a = "int f(int x) { return x + 1; } // one\n/* block */"
+    b = "int f(int x)\n{\n    return x + 1;  /* other words */\n}\n"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only('s = "// kept";') == 's="// kept";'
+    assert bench._code_only("x = 1;") != bench._code_only("x = 2;")
