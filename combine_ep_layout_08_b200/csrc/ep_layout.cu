@@ -1007,18 +1007,18 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
     int32_t* run = run_all + (size_t)warp * E;
 
     // A barrier that timed out earlier leaves its words inconsistent until
-    // ep_handle_check resets them: refuse to run (every CTA reads the same
-    // word).  Every CTA reads the launch's barrier base here, before any
-    // CTA can finish the last barrier and store the next one.
+    // ep_handle_check resets them: refuse to take part in the barriers (every
+    // CTA reads the same word).  Every CTA reads the launch's barrier base
+    // before it arrives at the first barrier, so before any CTA can finish
+    // the last barrier and store the next one.  Both words are requested
+    // here and used after phase 1, so their latency hides behind its loads.
     __shared__ int stale;
     __shared__ int32_t bar_base;
+    int32_t err_word = 0, base_word = 0;
     if (threadIdx.x == 0) {
-        stale = (*(volatile int32_t*)err & kErrTimeout) != 0;
-        bar_base = *(volatile int32_t*)(bar + 1);
+        err_word = *(volatile int32_t*)err;
+        base_word = *(volatile int32_t*)(bar + 1);
     }
-    __syncthreads();
-    if (stale)
-        return;
     const int32_t G = (int32_t)gridDim.x;
 
     // a tile's entries into ents and each warp's histogram into its run row
@@ -1058,6 +1058,13 @@ layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, in
             __syncthreads();
         }
     }
+    if (threadIdx.x == 0) {
+        stale = (err_word & kErrTimeout) != 0;
+        bar_base = base_word;
+    }
+    __syncthreads();
+    if (stale)
+        return;
     if (!grid_barrier(bar, bar_base + G, false, err))
         return;
 
