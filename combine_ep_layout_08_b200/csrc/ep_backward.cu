@@ -12,7 +12,9 @@
 //                      grad_w[t][j] = sum_h grad_out[t][h] * y[dst_row[t][j]][h]
 //     (this file).
 //
-// combine_backward_kernel: one CTA per token.  Each thread takes 16-byte
+// combine_backward_v32_kernel (rows in 32-byte vectors, the common case) is
+// described where it is defined.  combine_backward_kernel (16-byte rows):
+// one CTA per token.  Each thread takes 16-byte
 // vectors of the row (8 channels), reads grad_out once and the k rows of y,
 // writes the k scaled rows of grad_y and keeps k fp32 partial dot products
 // (fused multiply-adds, its channels in order).  The partials are reduced
@@ -24,6 +26,7 @@
 
 #include <algorithm>
 
+#include "ep_dispatch_units.cuh"
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -124,6 +127,95 @@ combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restr
     }
 }
 
+// 32-byte vectors, one warp per token (rows 32-byte aligned, H % 16 == 0):
+// the token's row is walked in 512-channel units, one vector per lane.  Per
+// unit the lane loads grad_out's vector and the vectors of the (up to 8)
+// slots of the batch before using any, writes the scaled vectors of grad_y
+// (one fp32 product, bf16 round to nearest even: bit-exact) and adds its 16
+// products per slot to that slot's partial dot (units in order, channels in
+// order).  A fixed xor-shuffle tree then sums the 32 partials of each slot,
+// so grad_w is bitwise repeatable; no block barrier is needed.
+__global__ void __launch_bounds__(256)
+combine_backward_v32_kernel(const units::Vec32* __restrict__ grad_out,
+                            const units::Vec32* __restrict__ y, int64_t y_rows,
+                            const float* __restrict__ weights, int T, int k, int64_t vpr,
+                            const int32_t* __restrict__ dst_row, units::Vec32* __restrict__ grad_y,
+                            int64_t grad_y_rows, float* __restrict__ grad_w, int32_t* err)
+{
+    using units::Vec32;
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T)
+        return;
+    int d = -1;
+    float w = 0.0f;
+    if (lane < k) {
+        d = __ldg(dst_row + t * k + lane);
+        w = __ldg(weights + t * k + lane);
+        if (d >= y_rows || d >= grad_y_rows) {
+            atomicOr(err, kErrCombineCap);
+            d = -1;
+        }
+    }
+    const int64_t upr = (vpr + 31) / 32;
+    const Vec32* g_row = grad_out + t * vpr;
+    for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
+        const int nj = min(kSlotBatch, k - j0);
+        int dj[kSlotBatch];
+        float wj[kSlotBatch], part[kSlotBatch];
+#pragma unroll
+        for (int jj = 0; jj < kSlotBatch; ++jj) {
+            dj[jj] = __shfl_sync(kFull, d, (j0 + jj) & 31);
+            wj[jj] = __shfl_sync(kFull, w, (j0 + jj) & 31);
+            if (jj >= nj)
+                dj[jj] = -1;
+            part[jj] = 0.0f;
+        }
+        for (int64_t u = 0; u < upr; ++u) {
+            const int64_t v = u * 32 + lane;
+            if (v >= vpr)
+                continue;  // only the last unit is ragged; no shuffles below
+            const Vec32 gv = units::ld32_once(g_row + v);
+            Vec32 yv[kSlotBatch];
+#pragma unroll
+            for (int jj = 0; jj < kSlotBatch; ++jj)
+                if (dj[jj] >= 0)
+                    yv[jj] = units::ld32_once(y + (int64_t)dj[jj] * vpr + v);
+            float g[16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                g[2 * c] = bf16_lo(gv.w[c]);
+                g[2 * c + 1] = bf16_hi(gv.w[c]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < kSlotBatch; ++jj) {
+                if (dj[jj] < 0)
+                    continue;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    part[jj] = __fmaf_rn(g[2 * c], bf16_lo(yv[jj].w[c]), part[jj]);
+                    part[jj] = __fmaf_rn(g[2 * c + 1], bf16_hi(yv[jj].w[c]), part[jj]);
+                }
+                Vec32 o;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    o.w[c] = pack_bf16x2(__fmul_rn(wj[jj], g[2 * c]), __fmul_rn(wj[jj], g[2 * c + 1]));
+                units::st32(grad_y + (int64_t)dj[jj] * vpr + v, o);
+            }
+        }
+        // fixed-order reduction over the lanes
+#pragma unroll
+        for (int jj = 0; jj < kSlotBatch; ++jj)
+            for (int o = 16; o > 0; o >>= 1) part[jj] += __shfl_xor_sync(kFull, part[jj], o);
+#pragma unroll
+        for (int jj = 0; jj < kSlotBatch; ++jj)
+            if (lane == jj && jj < nj)
+                grad_w[t * k + j0 + jj] = dj[jj] >= 0 ? part[jj] : 0.0f;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
@@ -132,6 +224,15 @@ cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const
 {
     if (h.T == 0)
         return cudaSuccess;
+    if (H % 16 == 0 && ((uintptr_t)grad_out & 31u) == 0 && ((uintptr_t)y & 31u) == 0 &&
+        ((uintptr_t)grad_y & 31u) == 0) {
+        const unsigned grid = (unsigned)((h.T + 7) / 8);  // one warp per token
+        return launch_pdl(combine_backward_v32_kernel, grid, 256u, 0, s,
+                          static_cast<const units::Vec32*>(grad_out),
+                          static_cast<const units::Vec32*>(y), y_rows, w, h.T, h.k,
+                          (int64_t)H / 16, h.dst_row, static_cast<units::Vec32*>(grad_y),
+                          grad_y_rows, grad_w, h.err);
+    }
     const int64_t vpr = H / 8;
     const int threads = (int)std::min<int64_t>(kMaxThreads, 32 * ((vpr + 31) / 32));
     return launch_pdl(combine_backward_kernel, (unsigned)h.T, (unsigned)threads, 0, s,
