@@ -265,3 +265,40 @@ def test_non_default_stream(oracle):
     rows = lay.dst_row[lay.dst_row >= 0]
     assert np.array_equal(recv.view(torch.uint8).cpu().numpy()[rows], exp_q[rows])
     assert np.array_equal(sc.cpu().numpy()[rows].view(np.uint32), exp_s[rows].view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "fp8_mn"])
+def test_dispatch_fp8_receive_rows_16_byte_aligned(oracle, fmt):
+    """A receive buffer that is 16- but not 32-byte aligned (the API's
+    minimum): codes and scales bit-exact, nothing written outside it."""
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV, bits_to_bf16
+
+    rng = np.random.default_rng(29)
+    T, H, E, R, k = 90, 1024, 32, 8, 8
+    x_bits = make_x(T, H, rng)
+    idx, _ = random_topk(T, E, k, rng, p_unused=0.1)
+    lay = oracle.layout(idx, E, R)
+    P = lay.total_rows
+    cap = (P + 3) // 4 * 4
+    h = _handle(T, k, E, R)
+    ep.ep_layout(h, torch.from_numpy(idx).to(DEV))
+    raw = torch.full((cap * H + 32,), SENTINEL, dtype=torch.uint8, device=DEV)
+    recv = raw[16:16 + cap * H].view(cap, H).view(torch.float8_e4m3fn)
+    assert recv.data_ptr() % 32 == 16
+    rows = lay.dst_row[lay.dst_row >= 0]
+    if fmt == "fp8":
+        sc = torch.empty((cap, H // 128), dtype=torch.float32, device=DEV)
+        ep.ep_dispatch(h, bits_to_bf16(x_bits), "fp8", recv_x=recv, recv_scales=sc)
+        q_ref, s_ref = oracle.dispatch_fp8(x_bits, lay.dst_row, cap)
+        assert np.array_equal(sc.cpu().numpy()[rows].view(np.uint32), s_ref[rows].view(np.uint32))
+    else:
+        sc = torch.empty((H // 128, cap), dtype=torch.float32, device=DEV)
+        ep.ep_dispatch(h, bits_to_bf16(x_bits), "fp8_mn", recv_x=recv, recv_scales=sc)
+        q_ref, s_ref = oracle.dispatch_fp8_mn(x_bits, lay.dst_row, cap, cap)
+        assert np.array_equal(sc.cpu().numpy()[:, rows].view(np.uint32),
+                              s_ref[:, rows].view(np.uint32))
+    ep.ep_handle_check(h)
+    assert np.array_equal(recv.view(torch.uint8).cpu().numpy()[rows], q_ref[rows])
+    b = raw.cpu().numpy()
+    assert np.all(b[:16] == SENTINEL) and np.all(b[16 + cap * H:] == SENTINEL)
