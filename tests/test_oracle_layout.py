@@ -192,7 +192,7 @@ def test_recv_rows_bound(oracle):
     assert oracle.recv_rows_bound(4, 2, 8, 128) == 8 * 128
 
 
-def test_config_shapes_match_survey_sizes(oracle):
+def test_tiny_config_sizes(oracle):
     """The named configs give the sizes the design is built around."""
     from workloads import make_workload
 
