@@ -94,6 +94,8 @@ def library_path() -> str:
 def load_library():
     """Load libep.so (raises if it has not been built)."""
     global _lib
+    if _lib is not None:  # loaded: no lock on the per-call path
+        return _lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -154,17 +156,39 @@ def ep_strerror(status: int) -> str:
     return load_library().ep_strerror(status).decode()
 
 
+# PyTorch's raw current-stream getter (no Stream object per call), where this
+# build of PyTorch has it; the public API otherwise.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device):
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if _raw_stream is not None:
+        return _raw_stream(device.index)
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+class _NoSwitch:
+    """The handle's device is already current: nothing to switch."""
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NO_SWITCH = _NoSwitch()
 
 
 def _on(h: "EPHandle"):
     """Make the handle's device current for the duration of a library call."""
+    if torch.cuda.current_device() == h.device.index:
+        return _NO_SWITCH
     return torch.cuda.device(h.device)
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() > 0 else 0)
+    return t.data_ptr() if t is not None and t.numel() > 0 else None
 
 
 def ep_workspace_bytes(max_tokens: int, num_topk: int, num_experts: int, num_ranks: int,
