@@ -118,6 +118,8 @@ def load_library():
             "ep_dispatch": ([P, P, I, I, P, P, I64, P], I),
             "ep_combine": ([P, P, I64, P, I, P, P], I),
             "ep_dispatch_ex": ([P, P, I, I, I, P, P, I64, P], I),
+            "ep_dispatch_ranks": ([P, I, I, P, I, I, P, P, P, P], I),
+            "ep_combine_ranks": ([P, I, I, P, P, P, I, I, P, P], I),
             "ep_combine_ex": ([P, P, I64, P, I, I, P, P], I),
             "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
             "ep_dispatch_backward": ([P, P, I64, I, P, P], I),
@@ -452,6 +454,83 @@ def ep_combine_range(h: EPHandle, t_begin: int, y: torch.Tensor, topk_weights_ro
         _check(load_library().ep_combine_range(
             h.handle, t_begin, n, _ptr(y), y.shape[0], _ptr(topk_weights_rows), H, _ptr(out_rows),
             _stream(h.device)), "ep_combine_range")
+
+
+def _table(values, ctype):
+    return (ctype * len(values))(*values)
+
+
+def ep_dispatch_ranks(h: EPHandle, t_begin: int, x_rows: torch.Tensor, fmt: Optional[str],
+                      recv_x: list, recv_scales: Optional[list] = None) -> None:
+    """Expert-parallel dispatch of tokens [t_begin, t_begin + len(x_rows)) of
+    the last (global) layout into one receive buffer per rank: rank p gets
+    rows [rank_off[p], rank_off[p+1]) of the layout, renumbered from 0, in
+    recv_x[p] (and its FP8 scales in recv_scales[p]).  On several GPUs the
+    entries are peer views of the ranks' buffers."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch_ranks")
+    if x_rows.dtype not in _DTYPES or x_rows.dim() != 2 or not x_rows.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: x_rows must be contiguous [n, H]")
+    f = _fmt_code(fmt, x_rows.dtype)
+    if (_is_copy(f) and f != _COPY_FMT[x_rows.dtype]) or \
+            (not _is_copy(f) and (f != EP_FMT_FP8_E4M3_1X128 or x_rows.dtype != torch.bfloat16)):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: row copy or bf16 -> fp8 (row-major)")
+    n, H = x_rows.shape
+    if len(recv_x) != h.R or (not _is_copy(f) and (recv_scales is None or len(recv_scales) != h.R)):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: one buffer per rank")
+    for r in recv_x:
+        if r.shape[1] != H or not r.is_contiguous() or r.dtype != _recv_dtype(f):
+            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: recv_x[p] must be [*, H]")
+    ptrs = _table([_ptr(r) for r in recv_x], ctypes.c_void_p)
+    rows = _table([r.shape[0] for r in recv_x], ctypes.c_int64)
+    sptrs = _table([_ptr(sc) for sc in recv_scales], ctypes.c_void_p) if not _is_copy(f) else None
+    with _on(h):
+        _check(load_library().ep_dispatch_ranks(
+            h.handle, t_begin, n, _ptr(x_rows), H, f, ptrs, sptrs, rows, _stream(h.device)),
+            "ep_dispatch_ranks")
+
+
+def ep_combine_ranks(h: EPHandle, t_begin: int, y: list, topk_weights_rows: torch.Tensor,
+                     out_rows: torch.Tensor) -> None:
+    """Expert-parallel combine of tokens [t_begin, t_begin + len(out_rows)) of
+    the last (global) layout, reading each slot's expert output from its
+    rank's buffer y[p] (bf16 or fp16, the type of out_rows)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_combine_ranks")
+    n, H = out_rows.shape
+    if (out_rows.dtype not in _DTYPES or not out_rows.is_contiguous() or len(y) != h.R
+            or topk_weights_rows.dtype != torch.float32
+            or tuple(topk_weights_rows.shape) != (n, h.k) or not topk_weights_rows.is_contiguous()
+            or any(t.dtype != out_rows.dtype or t.shape[1] != H or not t.is_contiguous() for t in y)):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_ranks: bad tensor")
+    ptrs = _table([_ptr(t) for t in y], ctypes.c_void_p)
+    rows = _table([t.shape[0] for t in y], ctypes.c_int64)
+    with _on(h):
+        _check(load_library().ep_combine_ranks(
+            h.handle, t_begin, n, ptrs, rows, _ptr(topk_weights_rows), H, _DTYPES[out_rows.dtype],
+            _ptr(out_rows), _stream(h.device)), "ep_combine_ranks")
+
+
+def ep_allgather_topk(topk_idx: torch.Tensor, group=None):
+    """All ranks' top-k indices in rank order (the global token order of the
+    expert-parallel layout) and this rank's first global token: an all-gather
+    of the token counts, then of the index rows (padded to the largest
+    count).  Works with any torch.distributed backend the tensors suit."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    me = dist.get_rank(group)
+    n = torch.tensor([topk_idx.shape[0]], dtype=torch.int64, device=topk_idx.device)
+    counts = [torch.zeros_like(n) for _ in range(world)]
+    dist.all_gather(counts, n, group=group)
+    counts = [int(c.item()) for c in counts]
+    most = max(counts) if counts else 0
+    pad = torch.full((most, topk_idx.shape[1]), -1, dtype=topk_idx.dtype, device=topk_idx.device)
+    pad[:topk_idx.shape[0]] = topk_idx
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    glob = torch.cat([parts[r][:counts[r]] for r in range(world)], dim=0).contiguous()
+    return glob, sum(counts[:me])
 
 
 def ep_dispatch_backward(h: EPHandle, grad_recv: torch.Tensor,

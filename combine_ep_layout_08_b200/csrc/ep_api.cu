@@ -490,6 +490,81 @@ ep_status_t ep_combine_range(ep_handle_t hh, int t_begin, int t_count, const voi
                         EP_DTYPE_BF16, out_rows, stream, "ep_combine_range");
 }
 
+ep_status_t ep_dispatch_ranks(ep_handle_t hh, int t_begin, int t_count, const void* x_rows, int H,
+                              ep_fmt_t fmt, void* const* recv_x, float* const* recv_scales,
+                              const int64_t* recv_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 16 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    const bool fp8 = fmt == EP_FMT_FP8_E4M3_1X128;
+    if (!fp8 && fmt != EP_FMT_BF16 && fmt != EP_FMT_FP16)
+        return EP_ERR_INVALID_ARG;
+    if (fp8 && H % 128 != 0)
+        return EP_ERR_INVALID_ARG;
+    if (h->R > EP_MAX_RANK_TABLE || !recv_x || !recv_rows || (fp8 && !recv_scales))
+        return EP_ERR_INVALID_ARG;
+    if (t_count > 0 && !x_rows)
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(x_rows, 32))
+        return EP_ERR_ALIGNMENT;
+    ep::RankTable tab = {};
+    for (int p = 0; p < h->R; ++p) {
+        if (recv_rows[p] < 0 || (recv_rows[p] > 0 && !recv_x[p]) ||
+            (fp8 && recv_rows[p] > 0 && !recv_scales[p]))
+            return EP_ERR_INVALID_ARG;
+        if (!ep::aligned(recv_x[p], fp8 ? 16 : 32) || (fp8 && !ep::aligned(recv_scales[p], 4)))
+            return EP_ERR_ALIGNMENT;
+        tab.base[p] = recv_x[p];
+        tab.scales[p] = fp8 ? recv_scales[p] : nullptr;
+        tab.rows[p] = recv_rows[p];
+    }
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaError_t rc = ep::launch_dispatch_ranks(sub, x_rows, H, fp8, false, tab,
+                                               static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_ranks");
+}
+
+ep_status_t ep_combine_ranks(ep_handle_t hh, int t_begin, int t_count, const void* const* y,
+                             const int64_t* y_rows, const float* topk_weights_rows, int H,
+                             ep_dtype_t dtype, void* out_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 8 != 0 || (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16))
+        return EP_ERR_INVALID_ARG;
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    if (h->R > EP_MAX_RANK_TABLE || !y || !y_rows)
+        return EP_ERR_INVALID_ARG;
+    if (t_count > 0 && (!out_rows || !topk_weights_rows))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(out_rows, 16) || !ep::aligned(topk_weights_rows, 4))
+        return EP_ERR_ALIGNMENT;
+    ep::RankTable tab = {};
+    for (int p = 0; p < h->R; ++p) {
+        if (y_rows[p] < 0 || (y_rows[p] > 0 && !y[p]))
+            return EP_ERR_INVALID_ARG;
+        if (!ep::aligned(y[p], 16))
+            return EP_ERR_ALIGNMENT;
+        tab.base[p] = const_cast<void*>(y[p]);
+        tab.rows[p] = y_rows[p];
+    }
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaError_t rc = ep::launch_combine_ranks(sub, topk_weights_rows, H, dtype == EP_DTYPE_FP16,
+                                              tab, out_rows, static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine_ranks");
+}
+
 ep_status_t ep_dispatch_weights(ep_handle_t hh, const float* topk_weights, float* recv_weights,
                                 int64_t recv_capacity_rows, void* stream)
 {

@@ -113,17 +113,13 @@ __device__ __forceinline__ void fp8_load(const Vec32* __restrict__ xs, int64_t v
     }
 }
 
-// Quantise the loaded vectors (bfloat16, or binary16 when kHalf) and write
-// codes and scales to the k rows.
+// Quantise the loaded vectors (bfloat16, or binary16 when kHalf): the lane's
+// codes q and, in lanes 0 .. 4 kU - 1, the scale of the unit's block L.
 template <int kU, bool kHalf = false>
-__device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int64_t unit, int d,
-                                          int k, int H, uint8_t* __restrict__ recv_q,
-                                          float* __restrict__ recv_scales, int64_t scales_ld)
+__device__ __forceinline__ void fp8_quantize(const Vec32 (&a)[kU], uint4 (&q)[kU],
+                                             float& my_scale)
 {
     const int lane = threadIdx.x & 31;
-    const int nblk = H / 128;
-    const int64_t v0 = unit * (32 * kU) + lane;
-    uint4 q[kU];
     float sc[kU];
 #pragma unroll
     for (int i = 0; i < kU; ++i) {
@@ -157,7 +153,7 @@ __device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int
     }
     // lane L < 8 takes the scale of block L of the unit: vector L / 4, lane
     // group L % 4 (leader lane 8 (L % 4))
-    float my_scale = 0.0f;
+    my_scale = 0.0f;
 #pragma unroll
     for (int i = 0; i < kU; ++i) {
 #pragma unroll
@@ -167,6 +163,20 @@ __device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int
                 my_scale = sv;
         }
     }
+}
+
+// Quantise the loaded vectors and write codes and scales to the k rows.
+template <int kU, bool kHalf = false>
+__device__ __forceinline__ void fp8_store(const Vec32 (&a)[kU], int64_t vpr, int64_t unit, int d,
+                                          int k, int H, uint8_t* __restrict__ recv_q,
+                                          float* __restrict__ recv_scales, int64_t scales_ld)
+{
+    const int lane = threadIdx.x & 31;
+    const int nblk = H / 128;
+    const int64_t v0 = unit * (32 * kU) + lane;
+    uint4 q[kU];
+    float my_scale;
+    fp8_quantize<kU, kHalf>(a, q, my_scale);
     const int64_t blk = unit * (4 * kU) + lane;
     const bool sc_ok = lane < 4 * kU && blk < nblk;
     for (int j = 0; j < k; ++j) {

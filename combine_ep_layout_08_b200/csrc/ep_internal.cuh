@@ -149,6 +149,20 @@ cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const
                                     int64_t y_rows, const float* w, int H, void* grad_y,
                                     int64_t grad_y_rows, float* grad_w, cudaStream_t s);
 
+// Per-rank receive buffers of the expert-parallel entry points, passed by
+// value: base[p] (rows of the layout's rank-p block, renumbered from 0),
+// scales[p] (FP8 row-major scales, or null) and rows[p] (capacity in rows).
+struct RankTable {
+    void* base[EP_MAX_RANK_TABLE];
+    float* scales[EP_MAX_RANK_TABLE];
+    int64_t rows[EP_MAX_RANK_TABLE];
+};
+
+cudaError_t launch_dispatch_ranks(const Handle& h, const void* x, int H, bool fp8, bool half,
+                                  const RankTable& tab, cudaStream_t s);
+cudaError_t launch_combine_ranks(const Handle& h, const float* w, int H, bool half,
+                                 const RankTable& tab, void* out, cudaStream_t s);
+
 // Persistent-grid size: min(resident blocks per SM from the occupancy API,
 // max_per_sm) x the SM count of the current device, cached per kernel and
 // device.

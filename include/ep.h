@@ -99,6 +99,10 @@ typedef enum {
     EP_FMT_FP16 = 3               /* receive rows are the fp16 input rows */
 } ep_fmt_t;
 
+/* Most ranks a per-rank buffer table of ep_dispatch_ranks / ep_combine_ranks
+ * may have. */
+#define EP_MAX_RANK_TABLE 64
+
 /* Views of the layout held in the workspace (see ep_handle_view). */
 typedef enum {
     EP_VIEW_NUM_TOKENS_PER_EXPERT = 0, /* int32 [E]     slots routed to each expert */
@@ -248,6 +252,44 @@ ep_status_t ep_dispatch_range(ep_handle_t h, int t_begin, int t_count, const voi
 ep_status_t ep_combine_range(ep_handle_t h, int t_begin, int t_count, const void* y,
                              int64_t y_rows, const float* topk_weights_rows, int H,
                              void* out_rows, void* stream);
+
+/* Expert-parallel form: one receive buffer per rank.
+ *
+ * The pages describe dispatch as an all-to-all that sends each token's row
+ * to the GPUs holding its experts and combine as the reverse exchange plus
+ * the weighted reduction ("DeepEP是什麼？…", section MoE為什麼需要All-to-all);
+ * rank p holds experts [p E/R, (p+1) E/R).  With the top-k indices of all
+ * ranks gathered in rank order (T = the sum of the ranks' token counts), the
+ * layout of ep_layout over the concatenated tokens is the expert-parallel
+ * layout: rank p's receive buffer is rows [rank_off[p], rank_off[p+1]) of it,
+ * renumbered from 0, so row d of the layout is row d - rank_off[p] of rank
+ * p's buffer.  These calls take that global layout and a table of the R
+ * ranks' buffers -- on R GPUs each entry is a peer pointer (the writes and
+ * reads are plain stores and loads; no TMA, no multicast) -- and move the
+ * rows of the source's own tokens [t_begin, t_begin + t_count) of the global
+ * order.  Semantics, arithmetic and errors are those of ep_dispatch_range /
+ * ep_combine_range restricted to a rank's block and renumbered.
+ *
+ * ep_dispatch_ranks: x_rows device [t_count][H] (bf16, or fp16 with
+ *   EP_FMT_FP16), 32-byte aligned, H % 16 == 0.  fmt EP_FMT_BF16 /
+ *   EP_FMT_FP16 (row copy) or EP_FMT_FP8_E4M3_1X128 (bf16 rows; row-major
+ *   scales).  recv_x: HOST array of R device pointers, rank p's receive
+ *   buffer [recv_rows[p]][H] of the row type (copy: 32-byte aligned) or of
+ *   e4m3 bytes (FP8: 16-byte aligned); recv_scales (FP8 only): HOST array of
+ *   R device pointers to fp32 [recv_rows[p]][H/128], 4-byte aligned;
+ *   recv_rows: HOST array of R capacities.  R = the handle's rank count,
+ *   at most EP_MAX_RANK_TABLE.  A row past its rank's capacity is skipped and
+ *   sets EP_ERR_CAPACITY.
+ * ep_combine_ranks: y: HOST array of R device pointers, rank p's expert
+ *   outputs [y_rows[p]][H] (bf16 or fp16 as dtype), 16-byte aligned, H % 8 ==
+ *   0; topk_weights_rows device fp32 [t_count][k]; out_rows device [t_count][H]
+ *   of dtype.  out[t] = rn16(fma chain over the used slots, j = 0..k-1). */
+ep_status_t ep_dispatch_ranks(ep_handle_t h, int t_begin, int t_count, const void* x_rows, int H,
+                              ep_fmt_t fmt, void* const* recv_x, float* const* recv_scales,
+                              const int64_t* recv_rows, void* stream);
+ep_status_t ep_combine_ranks(ep_handle_t h, int t_begin, int t_count, const void* const* y,
+                             const int64_t* y_rows, const float* topk_weights_rows, int H,
+                             ep_dtype_t dtype, void* out_rows, void* stream);
 
 /* GEMM-ready receive layout.  The pages say the high-throughput and
  * low-latency kernels share one "GEMM layout" (DeepEP v2 release notes, "Có

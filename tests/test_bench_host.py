@@ -76,3 +76,48 @@ def test_kernel_hash_ignores_comments_and_whitespace():
     assert bench._code_only(a) == bench._code_only(b)
     assert bench._code_only('s = "// kept";') == 's="// kept";'
     assert bench._code_only("x = 1;") != bench._code_only("x = 2;")
+
+
+def _gather_worker(rank, world, port, q):
+    import os
+
+    import torch
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import combine_ep_layout_08_b200 as ep
+
+        n = [3, 5][rank]
+        idx = torch.arange(n * 2, dtype=torch.int64).view(n, 2) + 100 * rank
+        glob, t0 = ep.ep_allgather_topk(idx)
+        q.put((rank, glob.tolist(), t0))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_allgather_topk_gloo_world_2():
+    """The expert-parallel global token order: rank-major concatenation of
+    the ranks' top-k rows (unequal counts), and each rank's first token."""
+    import multiprocessing as mp
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict()
+    for _ in range(2):
+        r, glob, t0 = q.get(timeout=120)
+        res[r] = (glob, t0)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    exp = [[2 * i, 2 * i + 1] for i in range(3)] + [[100 + 2 * i, 101 + 2 * i] for i in range(5)]
+    assert res[0] == (exp, 0) and res[1] == (exp, 3)
