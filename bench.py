@@ -423,6 +423,60 @@ def graph_latency_us(s, reps=200, step=None, inner=1):
     return us
 
 
+def time_ranks(dev, flush, seed, steps):
+    """The expert-parallel entry points on one GPU: the 8k workload as R = 8
+    ranks, one separately allocated receive buffer per rank (the ranks' own
+    buffers, or peer views of them, on 8 GPUs).  Times ep_dispatch_ranks and
+    ep_combine_ranks as one launch over all 8192 tokens and as 8 launches of
+    1024 tokens (each source rank's own call).  Same bytes as the 8k step."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from workloads import make_workload
+
+    w = make_workload(MAIN_WORKLOAD, seed)
+    h = ep.ep_handle_create(w.T, w.k, w.E, w.R, w.block_m, device=dev)
+    x = torch.from_numpy(w.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.from_numpy(w.topk_idx).to(dev)
+    wt = torch.from_numpy(w.topk_weights).to(dev)
+    ep.ep_layout(h, idx)
+    roff = ep.ep_handle_view(h, "rank_off").cpu().tolist()
+    recv = [torch.empty((max(roff[p + 1] - roff[p], 1), w.H), dtype=torch.bfloat16, device=dev)
+            for p in range(w.R)]
+    ys = [torch.randn((r.shape[0], w.H), device=dev).to(torch.bfloat16) for r in recv]
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+    src = w.T // w.R
+    res = {}
+    for name, parts in (("one_launch", [(0, w.T)]),
+                        ("per_source_rank", [(s * src, src) for s in range(w.R)])):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(3 + steps):
+            flush()
+            e = ev[i - 3] if i >= 3 else None
+            if e:
+                e[0].record()
+            for t0, n in parts:
+                ep.ep_dispatch_ranks(h, t0, x[t0:t0 + n], "bf16", recv)
+            if e:
+                e[1].record()
+            for t0, n in parts:
+                ep.ep_combine_ranks(h, t0, ys, wt[t0:t0 + n], out[t0:t0 + n])
+            if e:
+                e[2].record()
+        torch.cuda.synchronize()
+        d_ms = statistics.mean(a[0].elapsed_time(a[1]) for a in ev)
+        c_ms = statistics.mean(a[1].elapsed_time(a[2]) for a in ev)
+        db, cb = algo_bytes(w.T, w.H, w.k, w.fmt)
+        res[name] = {"dispatch_us": round(d_ms * 1e3, 2),
+                     "dispatch_GBps": round(db / (d_ms / 1e3) / 1e9, 1),
+                     "combine_us": round(c_ms * 1e3, 2),
+                     "combine_GBps": round(cb / (c_ms / 1e3) / 1e9, 1)}
+    ep.ep_handle_check(h)
+    res["workload"] = ("8k routing as R = 8 ranks on one GPU, 8 separate receive buffers, BF16; "
+                       "dispatch_ranks / combine_ranks (no NVLink: the ranks' buffers are local)")
+    return res
+
+
 def time_backward(dev, flush, seed, steps):
     """Backward of the 8k step: ep_dispatch_backward (a k-row sum per token)
     and ep_combine_backward (k scaled rows written, k dot products), each
@@ -572,7 +626,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--secondary", default="all",
-                    help="comma-separated secondary workloads (skewed, dsv3, decode, backward) or all")
+                    help="comma-separated secondary workloads (skewed, dsv3, decode, ranks, backward) "
+                         "or all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args()
@@ -678,6 +733,9 @@ def main():
             del s2
             torch.cuda.empty_cache()
 
+    if not args.no_secondary and (args.secondary == "all" or "ranks" in args.secondary.split(",")):
+        secondary["8k_ranks"] = time_ranks(dev, flush, args.seed + rank, max(3, min(args.steps, 50)))
+        torch.cuda.empty_cache()
     if not args.no_secondary and (args.secondary == "all" or "backward" in args.secondary.split(",")):
         secondary["8k_backward"] = time_backward(dev, flush, args.seed + rank,
                                                  max(3, min(args.steps, 50)))

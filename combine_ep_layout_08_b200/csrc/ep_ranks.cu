@@ -31,6 +31,17 @@ constexpr int kThreads = 256;
 
 using units::Vec32;
 
+// A 16-byte read-only load that skips L1 (the expert outputs are read once
+// per slot and not written while the kernel runs).
+__device__ __forceinline__ uint4 ld16_once(const void* p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 // rank_off of the layout (R + 1 words) into shared memory.
 __device__ __forceinline__ void load_rank_off(const int32_t* rank_off, int R, int32_t* s_roff)
 {
@@ -181,32 +192,37 @@ combine_ranks_kernel(const float* __restrict__ weights, int T, int k, int64_t vp
     for (int64_t u = wg; u < (int64_t)T * upr; u += nw) {
         const int64_t t = u / upr;
         const int64_t v0 = (u - t * upr) * (32 * kU) + lane;
+        const float w = lane < k ? __ldg(weights + t * k + lane) : 0.0f;
         int64_t local;
         const int p = slot_rank(dst_row, t, k, s_roff, R, tab, kErrCombineCap, err, &local);
         const uint64_t rowp =
             p >= 0 ? (uint64_t)(static_cast<const uint4*>(tab.base[p]) + local * vpr) : 0ull;
-        const float w = lane < k ? __ldg(weights + t * k + lane) : 0.0f;
         float acc[kU][8];
 #pragma unroll
         for (int i = 0; i < kU; ++i)
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
         for (int j0 = 0; j0 < k; j0 += kBatch) {
-            uint4 val[kBatch][kU];
+            // all row pointers of the batch first, then all loads, then the
+            // multiply-adds in slot order
             uint64_t rj[kBatch];
+            float wj[kBatch];
 #pragma unroll
             for (int jj = 0; jj < kBatch; ++jj) {
                 rj[jj] = __shfl_sync(kFull, rowp, (j0 + jj) & 31);
+                wj[jj] = __shfl_sync(kFull, w, (j0 + jj) & 31);
                 if (j0 + jj >= k)
                     rj[jj] = 0ull;
+            }
+            uint4 val[kBatch][kU];
+#pragma unroll
+            for (int jj = 0; jj < kBatch; ++jj)
 #pragma unroll
                 for (int i = 0; i < kU; ++i)
                     if (rj[jj] != 0ull && v0 + 32 * i < vpr)
-                        val[jj][i] = __ldcs(reinterpret_cast<const uint4*>(rj[jj]) + v0 + 32 * i);
-            }
+                        val[jj][i] = ld16_once(reinterpret_cast<const uint4*>(rj[jj]) + v0 + 32 * i);
 #pragma unroll
             for (int jj = 0; jj < kBatch; ++jj) {
-                const float wj = __shfl_sync(kFull, w, (j0 + jj) & 31);
                 if (rj[jj] == 0ull)
                     continue;
 #pragma unroll
@@ -217,8 +233,9 @@ combine_ranks_kernel(const float* __restrict__ weights, int T, int k, int64_t vp
                     const uint32_t wd[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        acc[i][2 * c] = __fmaf_rn(wj, lo16<kHalf>(wd[c]), acc[i][2 * c]);
-                        acc[i][2 * c + 1] = __fmaf_rn(wj, hi16<kHalf>(wd[c]), acc[i][2 * c + 1]);
+                        acc[i][2 * c] = __fmaf_rn(wj[jj], lo16<kHalf>(wd[c]), acc[i][2 * c]);
+                        acc[i][2 * c + 1] =
+                            __fmaf_rn(wj[jj], hi16<kHalf>(wd[c]), acc[i][2 * c + 1]);
                     }
                 }
             }
