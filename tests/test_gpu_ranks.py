@@ -166,3 +166,57 @@ def test_rank_table_is_checked(oracle):
     with pytest.raises(ep.EPError):
         ep.ep_dispatch_ranks(h, 0, _bf16(x), "bf16", [off, recv[1]])      # 16-byte aligned only
     assert ep.ep_handle_check(h, raise_on_error=False) == 0
+
+
+def test_ranks_fp16_copy_and_cuda_graph_replay(oracle):
+    """fp16 rows through the rank table, captured once in a CUDA graph and
+    replayed with new inputs written into the same buffers (the table is
+    passed by value, so the graph keeps it)."""
+    import combine_ep_layout_08_b200 as ep
+
+    counts, E, R, k, H = [70, 58], 32, 2, 4, 512
+    rng = np.random.default_rng(31)
+    T = sum(counts)
+    idx, w = random_topk(T, E, k, rng)
+    lay = oracle.layout(idx, E, R)
+    blocks = _rank_rows(lay, R)
+    h = ep.ep_handle_create(T, k, E, R, device=DEV)
+    d_idx = torch.from_numpy(idx).to(DEV)
+    xd = torch.empty((T, H), dtype=torch.float16, device=DEV)
+    recv = [torch.zeros((b - a, H), dtype=torch.float16, device=DEV) for a, b in blocks]
+    ys = [torch.empty((b - a, H), dtype=torch.float16, device=DEV) for a, b in blocks]
+    wd = torch.from_numpy(w).to(DEV)
+    out = torch.empty((T, H), dtype=torch.float16, device=DEV)
+
+    def step():
+        ep.ep_layout(h, d_idx)
+        for s0, n in ((0, counts[0]), (counts[0], counts[1])):
+            ep.ep_dispatch_ranks(h, s0, xd[s0:s0 + n], "fp16", recv)
+        for s0, n in ((0, counts[0]), (counts[0], counts[1])):
+            ep.ep_combine_ranks(h, s0, ys, wd[s0:s0 + n], out[s0:s0 + n])
+
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        step()
+    torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    used = lay.dst_row[lay.dst_row >= 0]
+    for rep in range(2):
+        x = make_x_fp16(T, H, rng)
+        y = make_x_fp16(lay.total_rows, H, rng)
+        xd.copy_(torch.from_numpy(x.view(np.int16)).view(torch.float16))
+        for p, (a, b) in enumerate(blocks):
+            ys[p].copy_(torch.from_numpy(y[a:b].view(np.int16)).view(torch.float16))
+        g.replay()
+        torch.cuda.synchronize()
+        ep.ep_handle_check(h)
+        ref = oracle.dispatch_bf16(x, lay.dst_row, lay.total_rows)   # a 16-bit row copy
+        for p, (a, b) in enumerate(blocks):
+            rows = used[(used >= a) & (used < b)] - a
+            assert np.array_equal(_bits(recv[p])[rows], ref[a:b][rows]), (rep, p)
+        assert np.array_equal(_bits(out), oracle.combine(y, w, lay.dst_row, dtype="fp16")), rep
+    del g
