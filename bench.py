@@ -567,7 +567,22 @@ def cpu_baseline(w, budget_s=15.0):
     return {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": "first %d of %d tokens of the same workload, %d repetitions, "
                       "single-threaded C oracle (gcc -O2), layout+dispatch+combine" % (
-                          tokens, w.T, reps)}
+                          tokens, w.T, reps),
+            "host": host_cpu()}
+
+
+def host_cpu() -> dict:
+    """The host the CPU numbers come from: logical cores and CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"logical_cores": os.cpu_count(), "cpu_model": model}
 
 
 def run_reference(args, rank, world):
@@ -596,7 +611,8 @@ def run_reference(args, rank, world):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens_per_step": tokens},
             "cpu_baseline": {"value": round(val, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": "first %d of %d tokens per step" % (tokens, w.T)},
+                             "sample": "first %d of %d tokens per step" % (tokens, w.T),
+                             "host": host_cpu()},
             "e2e": {"value": round(val, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
