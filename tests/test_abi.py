@@ -152,3 +152,34 @@ def test_strerror(lib):
     assert ep_strerror(0) == "EP_OK"
     assert "BAD_INDEX" in ep_strerror(5)
     assert ep_strerror(1234) == "unknown ep_status_t"
+
+
+def test_newer_entry_points_rejected_before_any_launch(lib):
+    """The FP16, expert-parallel, backward and GEMM-layout calls check their
+    arguments (and that a layout exists) on the host, before any launch."""
+    from combine_ep_layout_08_b200 import (EP_ERR_INVALID_ARG, EP_ERR_STATE,
+                                           ep_workspace_bytes)
+
+    need = ep_workspace_bytes(64, 2, 16, 4)
+    st, h = _create(lib, 0x7f0000000000, need, 64, 2, 16, 4, 128)
+    assert st == 0
+    P = ctypes.c_void_p
+    tab = (ctypes.c_void_p * 4)(0x1000, 0x2000, 0x3000, 0x4000)
+    rows = (ctypes.c_int64 * 4)(8, 8, 8, 8)
+    # no layout yet: every data call reports the state error
+    assert lib.ep_dispatch_ex(h, P(0x1000), 1, 256, 3, P(0x2000), None, 8, None) == EP_ERR_STATE
+    assert lib.ep_combine_ex(h, P(0x1000), 8, P(0x2000), 256, 1, P(0x3000), None) == EP_ERR_STATE
+    assert lib.ep_dispatch_ranks(h, 0, 0, P(0x1000), 256, 0, tab, None, rows, None) == EP_ERR_STATE
+    assert lib.ep_combine_ranks(h, 0, 0, tab, rows, P(0x2000), 256, 0, P(0x3000), None) \
+        == EP_ERR_STATE
+    assert lib.ep_dispatch_backward(h, P(0x1000), 8, 256, P(0x2000), None) == EP_ERR_STATE
+    # bad sizes and types are rejected before the state is looked at
+    assert lib.ep_dispatch_ranks(h, 0, 0, P(0x1000), 200, 0, tab, None, rows, None) \
+        == EP_ERR_INVALID_ARG                                   # H % 16 != 0
+    assert lib.ep_combine_ranks(h, 0, 0, tab, rows, P(0x2000), 256, 7, P(0x3000), None) \
+        == EP_ERR_INVALID_ARG                                   # unknown dtype
+    assert lib.ep_combine_ex(h, P(0x1000), 8, P(0x2000), 250, 0, P(0x3000), None) \
+        == EP_ERR_INVALID_ARG                                   # H % 8 != 0
+    assert lib.ep_layout_dispatch(h, P(0x1000), 65, P(0x2000), 256, 0, P(0x3000), None, 8, None) \
+        == EP_ERR_INVALID_ARG                                   # T > max_tokens
+    lib.ep_handle_destroy(h)
