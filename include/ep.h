@@ -14,6 +14,15 @@
  *   ep_combine   gather of the k expert outputs of each token, reduced with
  *                the routing weights in fp32, back into token order.
  *
+ * Around them: ep_layout_dispatch (layout and dispatch in one launch for
+ * decode-sized batches), token-range forms (ep_dispatch_range /
+ * ep_combine_range), FP16 rows (EP_FMT_FP16, ep_dispatch_ex, ep_combine_ex),
+ * the expert-parallel form with one receive buffer per rank
+ * (ep_dispatch_ranks / ep_combine_ranks), GEMM-ready helpers (MN-major FP8
+ * scales, ep_dispatch_weights, ep_zero_pad_rows), the backward of dispatch
+ * and combine, and a layout entry point that needs no workspace
+ * (ep_layout_static_scratch).
+ *
  * Source of the operations.  "DeepEP是什麼？MoE Dispatch、Combine、
  * All-to-all與V2架構" (yololab.net), stage table of the section
  * "MoE為什麼需要All-to-all": dispatch takes tokens, top-k indices and weights
@@ -164,9 +173,11 @@ ep_status_t ep_layout(ep_handle_t h, const int64_t* topk_idx, int T, void* strea
  * latency matters most: "DeepEP是什麼？…", section 高吞吐與低延遲工作負載).
  * Same arguments, results and errors as ep_layout(h, topk_idx, T, stream)
  * followed by ep_dispatch(h, x, H, fmt, recv_x, recv_scales,
- * recv_capacity_rows, stream) (so x is bf16, or fp16 with EP_FMT_FP16).  When the batch is small (T*k <= 4096,
- * E <= 1024, T*R <= 65536) and rows take 32-byte vectors (H % 16 == 0; x,
- * and for BF16 recv_x, 32-byte aligned), both run in ONE launch: every CTA
+ * recv_capacity_rows, stream) (so x is bf16, or fp16 with EP_FMT_FP16).
+ * When the batch is small (T*k <= 4096, E <= 1024, T*R <= 65536, and the
+ * per-CTA count tables fit 200 KB of shared memory) and rows take 32-byte
+ * vectors (H % 16 == 0; x, and for a row copy recv_x, 32-byte aligned),
+ * both run in ONE launch: every CTA
  * computes the same layout in its shared memory, CTA 0 publishes it, and all
  * CTAs dispatch from their own copy -- no grid-wide wait.  Otherwise the two
  * launches of the separate calls run.  All arguments are checked before
@@ -190,9 +201,10 @@ ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
                                   int32_t* total_recv_rows, void* stream);
 
 /* Dispatch the T tokens of the last layout.
- * x: device bf16 [T][H], 16-byte aligned.
- * EP_FMT_BF16: H % 8 == 0; recv_x: device bf16 [recv_capacity_rows][H],
- *   16-byte aligned; recv_scales ignored.  recv_x[dst_row[t][j]] = x[t].
+ * x: device bf16 [T][H] (fp16 with EP_FMT_FP16), 16-byte aligned.
+ * EP_FMT_BF16 / EP_FMT_FP16: H % 8 == 0; recv_x: device rows of x's type
+ *   [recv_capacity_rows][H], 16-byte aligned; recv_scales ignored.
+ *   recv_x[dst_row[t][j]] = x[t].
  * EP_FMT_FP8_E4M3_1X128: H % 128 == 0; recv_x: device e4m3 bytes
  *   [recv_capacity_rows][H], 16-byte aligned; recv_scales: device fp32
  *   [recv_capacity_rows][H/128], 16-byte aligned.  For every token and every
@@ -201,6 +213,9 @@ ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
  *   +-448); amax == 0 gives s = 0 and q = 0.  Written to every dst row.
  *   This is the reading taken of the FP8 section of the yololab page, which
  *   asks to confirm scale granularity and format without fixing them.
+ * EP_FMT_FP8_E4M3_1X128_MN: the same codes and scales; recv_scales is
+ *   MN-major, fp32 [H/128][recv_capacity_rows] (scale of row r, block b at
+ *   b * recv_capacity_rows + r), recv_capacity_rows % 4 == 0.
  * Only the rows listed in dst_row are written; pad rows keep their contents.
  * A row >= recv_capacity_rows is skipped and sets EP_ERR_CAPACITY. */
 ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void* recv_x,
