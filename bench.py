@@ -703,12 +703,13 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = time_gpu_e2e(s, max(3, min(args.steps, 50)), 3)
+        e_steps = max(3, min(args.steps, 100))
+        e_ms, h2d, d2h = time_gpu_e2e(s, e_steps, 3)
         e_ms = aggregate_max(e_ms)
         e2e = {"value": round(world * (d_bytes + c_bytes) / (e_ms / 1e3) / 1e9, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_ms, 4),
-               "steps": max(3, min(args.steps, 50)),
+               "steps": e_steps,
                "how": "a stream of steps through the Python API: pinned host x, topk_idx, "
                       "weights in and out back every step; double-buffered device staging on "
                       "3 streams (H2D | ep_layout, ep_dispatch, ep_combine | D2H) so that a "
