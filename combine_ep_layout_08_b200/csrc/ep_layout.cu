@@ -580,10 +580,13 @@ __device__ __forceinline__ int32_t exscan_u16x8(int4& v, int32_t acc)
     return acc;
 }
 
+// kR: rounds the kernel is compiled for (kSmallRounds; the fused launch of a
+// one-round batch, every decode batch, takes kR = 1: measured 2 % faster in
+// CUDA graphs; the layout-only kernel was slower so, and keeps kSmallRounds).
 // kFused = false: the layout alone.  kFused = true: then every warp of the
 // grid dispatches (token, unit) pieces with the positions in its own shared
 // memory -- no grid-wide wait.
-template <bool kFused>
+template <bool kFused, int kR = kSmallRounds>
 __global__ void __launch_bounds__(kSmallThreads)
 layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
                     uint64_t rank_magic, int block_m, int32_t* __restrict__ cnt_g,
@@ -637,9 +640,9 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
         const int64_t t = token_of_piece(u0);
         units::fp8_load<1>(xv + t * vpr, vpr, u0 - t * upr, cur);
     }
-    int64_t raw[kSmallRounds];
+    int64_t raw[kR];
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
+    for (int q = 0; q < kR; ++q) {
         const int f = q * kSmallThreads + tid;
         raw[q] = (q < rounds && f < nent) ? topk_idx[f] : -1;
     }
@@ -654,18 +657,18 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             for (int64_t i = tid; i < bytes; i += kSmallThreads) itr[i] = 0;
         }
     }
-    int e_r[kSmallRounds];
+    int e_r[kR];
     int bad = 0;
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) e_r[q] = to_expert(raw[q], E, bad);
+    for (int q = 0; q < kR; ++q) e_r[q] = to_expert(raw[q], E, bad);
     if (__syncthreads_or(bad) && tid == 0 && leader)
         atomicOr(err, kErrBadIndex);
 
     // 2: equal experts (and ranks) inside each warp
     const unsigned lt = lanemask_lt();
-    int rin[kSmallRounds];
+    int rin[kR];
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
+    for (int q = 0; q < kR; ++q) {
         rin[q] = 0;
         if (q < rounds) {
             const int f = q * kSmallThreads + tid;
@@ -746,7 +749,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
         }
     } else if (leader) {
 #pragma unroll
-        for (int q = 0; q < kSmallRounds; ++q) {
+        for (int q = 0; q < kR; ++q) {
             const int f = q * kSmallThreads + tid;
             if (q < rounds && f < nent && e_r[q] >= 0) {
                 const int rk = erank[f];
@@ -804,7 +807,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
             fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
     }
 #pragma unroll
-    for (int q = 0; q < kSmallRounds; ++q) {
+    for (int q = 0; q < kR; ++q) {
         const int f = q * kSmallThreads + tid;
         if (q < rounds && f < nent) {
             const int e = e_r[q];
@@ -1268,7 +1271,9 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
     const size_t smem = small_smem_bytes(E, R, small_rounds((int64_t)T * k));
     cudaError_t rc;
-    if ((rc = set_smem((const void*)layout_small_kernel<true>, smem)) != cudaSuccess)
+    const bool one_round = small_rounds((int64_t)T * k) == 1;
+    auto kern = one_round ? layout_small_kernel<true, 1> : layout_small_kernel<true>;
+    if ((rc = set_smem((const void*)kern, smem)) != cudaSuccess)
         return rc;
     int dev = 0, sms = 0;
     if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
@@ -1278,7 +1283,7 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
     // the dispatch -- FP8 division and row stores -- spreads over the GPU
     const unsigned grid = (unsigned)std::max(1, sms);
     FusedDispatch fd{x, H, fp8 ? 1 : 0, recv_x, recv_scales, scales_ld, cap_rows};
-    return launch_pdl(layout_small_kernel<true>, grid, kSmallThreads, smem, s, topk_idx, T, k, E,
+    return launch_pdl(kern, grid, kSmallThreads, smem, s, topk_idx, T, k, E,
                       R, epr, rank_magic_for(epr), h.block_m, h.cnt, h.expert_off, h.rank_off,
                       h.tokens_per_rank, h.rows_per_rank, h.total_rows, h.is_token_in_rank,
                       h.dst_row, h.recv_src, h.err, fd, make_small_plan(T, k, E, R, h.block_m));
