@@ -14,6 +14,14 @@ Typical use::
     y = expert(recv_x, recv_scales)                # user code, receive layout
     out = ep_combine(h, y, topk_weights)           # bf16 [T, H]
     ep_handle_check(h)                             # raises on a device-side error
+
+Also: ``ep_layout_dispatch`` (layout and dispatch in one launch for decode-
+sized batches), fp16 rows (``fmt="fp16"`` / fp16 tensors), token ranges
+(``ep_dispatch_range`` / ``ep_combine_range``), one receive buffer per
+expert-parallel rank (``ep_allgather_topk``, ``ep_dispatch_ranks``,
+``ep_combine_ranks``), GEMM-ready helpers (``fmt="fp8_mn"``,
+``ep_dispatch_weights``, ``ep_zero_pad_rows``) and the backward
+(``ep_dispatch_backward``, ``ep_combine_backward``).
 """
 from __future__ import annotations
 
@@ -28,7 +36,8 @@ __all__ = [
     "EPError", "EPHandle", "ep_workspace_bytes", "ep_recv_rows_upper_bound", "ep_handle_create",
     "ep_layout", "ep_layout_dispatch", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
     "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
-    "ep_dispatch_weights", "ep_zero_pad_rows",
+    "ep_dispatch_weights", "ep_zero_pad_rows", "ep_dispatch_ranks", "ep_combine_ranks",
+    "ep_allgather_topk",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
