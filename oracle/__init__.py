@@ -71,9 +71,9 @@ def _load():
             lib.oracle_expert_scale_fp8.restype = None
             lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, i32, P]
             lib.oracle_combine.restype = i32
-            lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, P]
+            lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, i32, P]
             lib.oracle_dispatch_backward.restype = i32
-            lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
+            lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, i32, P, P]
             lib.oracle_combine_backward.restype = i32
             lib.oracle_dispatch_weights.argtypes = [P, P, i64, i32, P, i64]
             lib.oracle_dispatch_weights.restype = i32
@@ -292,8 +292,10 @@ def combine(y_bits: np.ndarray, topk_weights: np.ndarray, dst_row: np.ndarray,
 
 # ---------------------------------------------------------------- backward
 
-def dispatch_backward(grad_recv_bits: np.ndarray, dst_row: np.ndarray) -> np.ndarray:
-    """grad_x[t] = bf16(sum over used slots of grad_recv[dst_row[t, j]]), fp32 in slot order."""
+def dispatch_backward(grad_recv_bits: np.ndarray, dst_row: np.ndarray,
+                      dtype: str = "bf16") -> np.ndarray:
+    """grad_x[t] = rn16(sum over used slots of grad_recv[dst_row[t, j]]), fp32 in slot
+    order; bf16 or fp16 bits."""
     g = np.ascontiguousarray(grad_recv_bits, dtype=np.uint16)
     dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
     rows, H = g.shape
@@ -301,15 +303,16 @@ def dispatch_backward(grad_recv_bits: np.ndarray, dst_row: np.ndarray) -> np.nda
     out = np.zeros((T, H), np.uint16)
     if rows == 0:
         g = np.zeros((1, H), np.uint16)
-    rc = _load().oracle_dispatch_backward(_p(g), rows, _p(dst_row), T, k, H, _p(out))
+    rc = _load().oracle_dispatch_backward(_p(g), rows, _p(dst_row), T, k, H, DTYPES[dtype],
+                                          _p(out))
     if rc != OK:
         raise OracleError(rc, "oracle_dispatch_backward")
     return out
 
 
 def combine_backward(grad_out_bits: np.ndarray, y_bits: np.ndarray, topk_weights: np.ndarray,
-                     dst_row: np.ndarray):
-    """(grad_y bits [rows, H] with pad rows zero, grad_w f32 [T, k])."""
+                     dst_row: np.ndarray, dtype: str = "bf16"):
+    """(grad_y bits [rows, H] with pad rows zero, grad_w f32 [T, k]); bf16 or fp16 rows."""
     g = np.ascontiguousarray(grad_out_bits, dtype=np.uint16)
     y = np.ascontiguousarray(y_bits, dtype=np.uint16)
     w = np.ascontiguousarray(topk_weights, dtype=np.float32)
@@ -321,7 +324,7 @@ def combine_backward(grad_out_bits: np.ndarray, y_bits: np.ndarray, topk_weights
     if rows == 0:
         y = np.zeros((1, H), np.uint16)
     rc = _load().oracle_combine_backward(_p(g), _p(y), rows, _p(w), _p(dst_row), T, k, H,
-                                         _p(gy), _p(gw))
+                                         DTYPES[dtype], _p(gy), _p(gw))
     if rc != OK:
         raise OracleError(rc, "oracle_combine_backward")
     return gy[:rows], gw

@@ -535,9 +535,9 @@ int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int3
 /* Backward of dispatch: every used slot (t, j) copied x[t] to row
  * dst_row[t][j], so grad_x[t] = sum over used slots of grad_recv[row],
  * accumulated in fp32 in slot order j = 0..k-1 (plain additions), rounded to
- * bf16 at the end. */
+ * the 16-bit type (bfloat16, dtype 0, or binary16, dtype 1) at the end. */
 int oracle_dispatch_backward(const uint16_t* grad_recv, int64_t rows, const int32_t* dst_row,
-                             int64_t T, int k, int64_t H, uint16_t* grad_x)
+                             int64_t T, int k, int64_t H, int dtype, uint16_t* grad_x)
 {
     float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
     if (!acc)
@@ -554,22 +554,23 @@ int oracle_dispatch_backward(const uint16_t* grad_recv, int64_t rows, const int3
                 return OR_ERR_CAPACITY;
             }
             for (int64_t h = 0; h < H; ++h)
-                acc[h] = acc[h] + oracle_bf16_to_f32(grad_recv[d * H + h]);
+                acc[h] = acc[h] + in16_to_f32(grad_recv[d * H + h], dtype);
         }
         for (int64_t h = 0; h < H; ++h)
-            grad_x[t * H + h] = oracle_f32_to_bf16_rn(acc[h]);
+            grad_x[t * H + h] = f32_to_out16(acc[h], dtype);
     }
     free(acc);
     return OR_OK;
 }
 
 /* Backward of combine, out[t] = sum_j w[t][j] y[dst_row[t][j]]:
- *   grad_y[dst_row[t][j]][h] = bf16_rn(w[t][j] * grad_out[t][h])  (one fp32 product)
- *   grad_w[t][j] = sum_h grad_out[t][h] * y[dst_row[t][j]][h]      (fp64, rounded to fp32)
- * Unused slots get grad_w = 0 and write no row. */
+ *   grad_y[dst_row[t][j]][h] = rn16(w[t][j] * grad_out[t][h])  (one fp32 product)
+ *   grad_w[t][j] = sum_h grad_out[t][h] * y[dst_row[t][j]][h]   (fp64, rounded to fp32)
+ * Unused slots get grad_w = 0 and write no row.  The 16-bit rows are
+ * bfloat16 (dtype 0) or binary16 (dtype 1); rn16 rounds to that type. */
 int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_rows,
                             const float* w, const int32_t* dst_row, int64_t T, int k, int64_t H,
-                            uint16_t* grad_y, float* grad_w)
+                            int dtype, uint16_t* grad_y, float* grad_w)
 {
     for (int64_t t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {
@@ -582,9 +583,9 @@ int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t
                 return OR_ERR_CAPACITY;
             double dot = 0.0;
             for (int64_t h = 0; h < H; ++h) {
-                const float g = oracle_bf16_to_f32(grad_out[t * H + h]);
-                dot += (double)g * (double)oracle_bf16_to_f32(y[d * H + h]);
-                grad_y[d * H + h] = oracle_f32_to_bf16_rn(w[t * k + j] * g);
+                const float g = in16_to_f32(grad_out[t * H + h], dtype);
+                dot += (double)g * (double)in16_to_f32(y[d * H + h], dtype);
+                grad_y[d * H + h] = f32_to_out16(w[t * k + j] * g, dtype);
             }
             grad_w[t * k + j] = (float)dot;
         }

@@ -206,3 +206,54 @@ def test_combine_fp16_within_bound_of_exact_sum(oracle):
     # half a binary16 ulp of the result (normal range; subnormal step 2^-25)
     half_ulp = np.maximum(np.ldexp(1.0, np.frexp(np.abs(exact) + acc_err)[1] - 12), 2.0 ** -25)
     assert np.all(np.abs(out - exact) <= acc_err + half_ulp)
+
+
+# ------------------------------------------------------------------ backward, binary16
+
+def test_dispatch_backward_fp16_gather_and_bound(oracle):
+    rng = np.random.default_rng(131)
+    T, H, E, k = 40, 128, 16, 4
+    idx1, _ = random_topk(T, E, 1, rng)
+    lay1 = oracle.layout(idx1, E, 4, 8)
+    g1 = make_x_fp16(lay1.total_rows, H, rng)
+    assert np.array_equal(oracle.dispatch_backward(g1, lay1.dst_row, dtype="fp16"),
+                          g1[lay1.dst_row[:, 0]])                      # k = 1: a gather
+    idx, _ = random_topk(T, E, k, rng, p_unused=0.2)
+    lay = oracle.layout(idx, E, 4, 8)
+    g = make_x_fp16(lay.total_rows, H, rng)
+    gx = oracle.fp16_to_f32(oracle.dispatch_backward(g, lay.dst_row, dtype="fp16")).astype(np.float64)
+    gf = oracle.fp16_to_f32(g).astype(np.float64)
+    exact = np.zeros((T, H))
+    absum = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            d = lay.dst_row[t, j]
+            if d >= 0:
+                exact[t] += gf[d]
+                absum[t] += np.abs(gf[d])
+    acc_err = k * 2.0 ** -24 * absum * (1 + 1e-6)
+    half_ulp = np.maximum(np.ldexp(1.0, np.frexp(np.abs(exact) + acc_err)[1] - 12), 2.0 ** -25)
+    assert np.all(np.abs(gx - exact) <= acc_err + half_ulp)
+
+
+def test_combine_backward_fp16_scaling_and_dot(oracle):
+    rng = np.random.default_rng(137)
+    T, H, E, k = 30, 256, 8, 3
+    idx, _ = random_topk(T, E, k, rng)
+    lay = oracle.layout(idx, E, 2, 4)
+    y = make_x_fp16(lay.total_rows, H, rng)
+    g = make_x_fp16(T, H, rng)
+    # power-of-two weights scale grad_out exactly (within the binary16 range)
+    w = (2.0 ** rng.integers(-3, 3, size=(T, k))).astype(np.float32)
+    gy, gw = oracle.combine_backward(g, y, w, lay.dst_row, dtype="fp16")
+    gf = oracle.fp16_to_f32(g).astype(np.float64)
+    yf = oracle.fp16_to_f32(y).astype(np.float64)
+    for t in range(T):
+        for j in range(k):
+            d = lay.dst_row[t, j]
+            assert np.array_equal(oracle.fp16_to_f32(gy[d]).astype(np.float64), w[t, j] * gf[t])
+            ref = np.float32(np.dot(gf[t], yf[d]))
+            assert abs(gw[t, j] - ref) <= abs(ref) * 2.0 ** -23 + 1e-30
+    # the bf16 reading of the same bits differs: the type is honoured
+    _, gw_b = oracle.combine_backward(g, y, w, lay.dst_row, dtype="bf16")
+    assert not np.array_equal(gw, gw_b)
