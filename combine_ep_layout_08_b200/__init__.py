@@ -128,6 +128,8 @@ def load_library():
             "ep_combine": ([P, P, I64, P, I, P, P], I),
             "ep_dispatch_ex": ([P, P, I, I, I, P, P, I64, P], I),
             "ep_dispatch_ranks": ([P, I, I, P, I, I, P, P, P, P], I),
+            "ep_dispatch_backward_ex": ([P, P, I64, I, I, P, P], I),
+            "ep_combine_backward_ex": ([P, P, P, I64, P, I, I, P, I64, P, P], I),
             "ep_combine_ranks": ([P, I, I, P, P, P, I, I, P, P], I),
             "ep_combine_ex": ([P, P, I64, P, I, I, P, P], I),
             "ep_dispatch_range": ([P, I, I, P, I, I, P, P, I64, P], I),
@@ -544,40 +546,51 @@ def ep_allgather_topk(topk_idx: torch.Tensor, group=None):
 
 def ep_dispatch_backward(h: EPHandle, grad_recv: torch.Tensor,
                          grad_x: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """grad_x[t] = sum over the used slots of grad_recv[dst_row[t, j]] (bf16 [T, H])."""
+    """grad_x[t] = sum over the used slots of grad_recv[dst_row[t, j]] ([T, H], the type
+    of grad_recv: bf16 or fp16)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_dispatch_backward")
-    if grad_recv.dtype != torch.bfloat16 or grad_recv.dim() != 2 or not grad_recv.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_backward: grad_recv must be bf16 [rows, H]")
+    if grad_recv.dtype not in _DTYPES or grad_recv.dim() != 2 or not grad_recv.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG,
+                      "ep_dispatch_backward: grad_recv must be bf16/fp16 [rows, H]")
     H = grad_recv.shape[1]
     if grad_x is None:
-        grad_x = torch.empty((h.T, H), dtype=torch.bfloat16, device=grad_recv.device)
+        grad_x = torch.empty((h.T, H), dtype=grad_recv.dtype, device=grad_recv.device)
+    if grad_x.dtype != grad_recv.dtype or tuple(grad_x.shape) != (h.T, H) or \
+            not grad_x.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_backward: grad_x must be [T, H]")
     with _on(h):
-        _check(load_library().ep_dispatch_backward(h.handle, _ptr(grad_recv), grad_recv.shape[0],
-                                                   H, _ptr(grad_x), _stream(h.device)),
-               "ep_dispatch_backward")
+        _check(load_library().ep_dispatch_backward_ex(
+            h.handle, _ptr(grad_recv), grad_recv.shape[0], H, _DTYPES[grad_recv.dtype],
+            _ptr(grad_x), _stream(h.device)), "ep_dispatch_backward")
     return grad_x
 
 
 def ep_combine_backward(h: EPHandle, grad_out: torch.Tensor, y: torch.Tensor,
                         topk_weights: torch.Tensor, grad_y: Optional[torch.Tensor] = None):
-    """(grad_y bf16 in the receive layout, grad_weights f32 [T, k]) for ep_combine."""
+    """(grad_y in the receive layout, grad_weights f32 [T, k]) for ep_combine; the rows
+    are bf16 or fp16 (grad_out, y and grad_y of one type)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_combine_backward")
     for name, t in (("grad_out", grad_out), ("y", y)):
-        if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
-            raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: %s must be bf16 2-D" % name)
+        if t.dtype not in _DTYPES or t.dtype != y.dtype or t.dim() != 2 or not t.is_contiguous():
+            raise EPError(EP_ERR_INVALID_ARG,
+                          "ep_combine_backward: %s must be 2-D bf16/fp16 of y's type" % name)
     if (topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (h.T, h.k)
             or not topk_weights.is_contiguous()):
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: topk_weights must be f32 [T, k]")
     H = y.shape[1]
     if grad_y is None:
         grad_y = torch.empty_like(y)
+    if grad_y.dtype != y.dtype or grad_y.dim() != 2 or grad_y.shape[1] != H or \
+            not grad_y.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: grad_y must be [*, H], y's type")
     grad_w = torch.empty((h.T, h.k), dtype=torch.float32, device=y.device)
     with _on(h):
-        _check(load_library().ep_combine_backward(
-            h.handle, _ptr(grad_out), _ptr(y), y.shape[0], _ptr(topk_weights), H, _ptr(grad_y),
-            grad_y.shape[0], _ptr(grad_w), _stream(h.device)), "ep_combine_backward")
+        _check(load_library().ep_combine_backward_ex(
+            h.handle, _ptr(grad_out), _ptr(y), y.shape[0], _ptr(topk_weights), H,
+            _DTYPES[y.dtype], _ptr(grad_y), grad_y.shape[0], _ptr(grad_w), _stream(h.device)),
+            "ep_combine_backward")
     return grad_y, grad_w
 
 

@@ -598,11 +598,12 @@ ep_status_t ep_zero_pad_rows(ep_handle_t hh, void* rows, int64_t row_bytes, int6
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_zero_pad_rows");
 }
 
-ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t grad_rows, int H,
-                                 void* grad_x, void* stream)
+ep_status_t ep_dispatch_backward_ex(ep_handle_t hh, const void* grad_recv, int64_t grad_rows,
+                                    int H, ep_dtype_t dtype, void* grad_x, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    if (!h || H <= 0 || H % 8 != 0 || grad_rows < 0)
+    if (!h || H <= 0 || H % 8 != 0 || grad_rows < 0 ||
+        (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16))
         return EP_ERR_INVALID_ARG;
     if (!h->has_layout)
         return EP_ERR_STATE;
@@ -611,16 +612,25 @@ ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t 
     if (!ep::aligned(grad_recv, 16) || !ep::aligned(grad_x, 16))
         return EP_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t rc = ep::launch_combine(*h, grad_recv, grad_rows, nullptr, H, grad_x, false, s);
+    cudaError_t rc = ep::launch_combine(*h, grad_recv, grad_rows, nullptr, H, grad_x,
+                                        dtype == EP_DTYPE_FP16, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_backward");
 }
 
-ep_status_t ep_combine_backward(ep_handle_t hh, const void* grad_out, const void* y,
-                                int64_t y_rows, const float* topk_weights, int H, void* grad_y,
-                                int64_t grad_y_rows, float* grad_weights, void* stream)
+ep_status_t ep_dispatch_backward(ep_handle_t hh, const void* grad_recv, int64_t grad_rows, int H,
+                                 void* grad_x, void* stream)
+{
+    return ep_dispatch_backward_ex(hh, grad_recv, grad_rows, H, EP_DTYPE_BF16, grad_x, stream);
+}
+
+ep_status_t ep_combine_backward_ex(ep_handle_t hh, const void* grad_out, const void* y,
+                                   int64_t y_rows, const float* topk_weights, int H,
+                                   ep_dtype_t dtype, void* grad_y, int64_t grad_y_rows,
+                                   float* grad_weights, void* stream)
 {
     Handle* h = ep::as_handle(hh);
-    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0 || grad_y_rows < 0)
+    if (!h || H <= 0 || H % 8 != 0 || y_rows < 0 || grad_y_rows < 0 ||
+        (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16))
         return EP_ERR_INVALID_ARG;
     if (!h->has_layout)
         return EP_ERR_STATE;
@@ -632,8 +642,17 @@ ep_status_t ep_combine_backward(ep_handle_t hh, const void* grad_out, const void
         return EP_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t rc = ep::launch_combine_backward(*h, grad_out, y, y_rows, topk_weights, H, grad_y,
-                                                 grad_y_rows, grad_weights, s);
+                                                 grad_y_rows, grad_weights,
+                                                 dtype == EP_DTYPE_FP16, s);
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine_backward");
+}
+
+ep_status_t ep_combine_backward(ep_handle_t hh, const void* grad_out, const void* y,
+                                int64_t y_rows, const float* topk_weights, int H, void* grad_y,
+                                int64_t grad_y_rows, float* grad_weights, void* stream)
+{
+    return ep_combine_backward_ex(hh, grad_out, y, y_rows, topk_weights, H, EP_DTYPE_BF16,
+                                  grad_y, grad_y_rows, grad_weights, stream);
 }
 
 ep_status_t ep_handle_check(ep_handle_t hh, void* stream)

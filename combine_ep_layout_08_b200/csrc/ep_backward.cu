@@ -6,9 +6,9 @@
 // defining gradients.  These are the gradients of the forward definitions:
 //
 //   dispatch backward: grad_x[t] = sum over used slots of grad_recv[dst_row[t][j]],
-//     fp32 in slot order j = 0..k-1, bf16 out -- the combine kernel with unit
-//     weights (ep_combine.cu);
-//   combine backward:  grad_y[dst_row[t][j]] = bf16(w[t][j] * grad_out[t])
+//     fp32 in slot order j = 0..k-1, rounded to the 16-bit type (bf16 or
+//     fp16) -- the combine kernel with unit weights (ep_combine.cu);
+//   combine backward:  grad_y[dst_row[t][j]] = rn16(w[t][j] * grad_out[t])
 //                      grad_w[t][j] = sum_h grad_out[t][h] * y[dst_row[t][j]][h]
 //     (this file).
 //
@@ -36,16 +36,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxThreads = 256;
 constexpr int kSlotBatch = 8;
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-    return a | (b << 16);
-}
-
+template <bool kHalf>
 __global__ void __launch_bounds__(kMaxThreads)
 combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restrict__ y,
                         int64_t y_rows, const float* __restrict__ weights, int T, int k,
@@ -82,8 +73,8 @@ combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restr
         for (int jj = 0; jj < kSlotBatch; ++jj) part[jj] = 0.0f;
         for (int64_t v = threadIdx.x; v < vpr; v += blockDim.x) {
             const uint4 gv = g_row[v];
-            const float g[8] = {bf16_lo(gv.x), bf16_hi(gv.x), bf16_lo(gv.y), bf16_hi(gv.y),
-                                bf16_lo(gv.z), bf16_hi(gv.z), bf16_lo(gv.w), bf16_hi(gv.w)};
+            const float g[8] = {lo16<kHalf>(gv.x), hi16<kHalf>(gv.x), lo16<kHalf>(gv.y), hi16<kHalf>(gv.y),
+                                lo16<kHalf>(gv.z), hi16<kHalf>(gv.z), lo16<kHalf>(gv.w), hi16<kHalf>(gv.w)};
             uint4 yv[kSlotBatch];
 #pragma unroll
             for (int jj = 0; jj < kSlotBatch; ++jj) {
@@ -96,17 +87,17 @@ combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restr
                 const int d = jj < nj ? s_row[j0 + jj] : -1;
                 if (d < 0)
                     continue;
-                const float f[8] = {bf16_lo(yv[jj].x), bf16_hi(yv[jj].x), bf16_lo(yv[jj].y),
-                                    bf16_hi(yv[jj].y), bf16_lo(yv[jj].z), bf16_hi(yv[jj].z),
-                                    bf16_lo(yv[jj].w), bf16_hi(yv[jj].w)};
+                const float f[8] = {lo16<kHalf>(yv[jj].x), hi16<kHalf>(yv[jj].x), lo16<kHalf>(yv[jj].y),
+                                    hi16<kHalf>(yv[jj].y), lo16<kHalf>(yv[jj].z), hi16<kHalf>(yv[jj].z),
+                                    lo16<kHalf>(yv[jj].w), hi16<kHalf>(yv[jj].w)};
 #pragma unroll
                 for (int c = 0; c < 8; ++c) part[jj] = __fmaf_rn(g[c], f[c], part[jj]);
                 const float w = s_w[j0 + jj];
                 uint4 o;
-                o.x = pack_bf16x2(__fmul_rn(w, g[0]), __fmul_rn(w, g[1]));
-                o.y = pack_bf16x2(__fmul_rn(w, g[2]), __fmul_rn(w, g[3]));
-                o.z = pack_bf16x2(__fmul_rn(w, g[4]), __fmul_rn(w, g[5]));
-                o.w = pack_bf16x2(__fmul_rn(w, g[6]), __fmul_rn(w, g[7]));
+                o.x = pack16x2<kHalf>(__fmul_rn(w, g[0]), __fmul_rn(w, g[1]));
+                o.y = pack16x2<kHalf>(__fmul_rn(w, g[2]), __fmul_rn(w, g[3]));
+                o.z = pack16x2<kHalf>(__fmul_rn(w, g[4]), __fmul_rn(w, g[5]));
+                o.w = pack16x2<kHalf>(__fmul_rn(w, g[6]), __fmul_rn(w, g[7]));
                 grad_y[(int64_t)d * vpr + v] = o;
             }
         }
@@ -135,6 +126,7 @@ combine_backward_kernel(const uint4* __restrict__ grad_out, const uint4* __restr
 // products per slot to that slot's partial dot (units in order, channels in
 // order).  A fixed xor-shuffle tree then sums the 32 partials of each slot,
 // so grad_w is bitwise repeatable; no block barrier is needed.
+template <bool kHalf>
 __global__ void __launch_bounds__(256)
 combine_backward_v32_kernel(const units::Vec32* __restrict__ grad_out,
                             const units::Vec32* __restrict__ y, int64_t y_rows,
@@ -186,8 +178,8 @@ combine_backward_v32_kernel(const units::Vec32* __restrict__ grad_out,
             float g[16];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                g[2 * c] = bf16_lo(gv.w[c]);
-                g[2 * c + 1] = bf16_hi(gv.w[c]);
+                g[2 * c] = lo16<kHalf>(gv.w[c]);
+                g[2 * c + 1] = hi16<kHalf>(gv.w[c]);
             }
 #pragma unroll
             for (int jj = 0; jj < kSlotBatch; ++jj) {
@@ -195,13 +187,13 @@ combine_backward_v32_kernel(const units::Vec32* __restrict__ grad_out,
                     continue;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    part[jj] = __fmaf_rn(g[2 * c], bf16_lo(yv[jj].w[c]), part[jj]);
-                    part[jj] = __fmaf_rn(g[2 * c + 1], bf16_hi(yv[jj].w[c]), part[jj]);
+                    part[jj] = __fmaf_rn(g[2 * c], lo16<kHalf>(yv[jj].w[c]), part[jj]);
+                    part[jj] = __fmaf_rn(g[2 * c + 1], hi16<kHalf>(yv[jj].w[c]), part[jj]);
                 }
                 Vec32 o;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    o.w[c] = pack_bf16x2(__fmul_rn(wj[jj], g[2 * c]), __fmul_rn(wj[jj], g[2 * c + 1]));
+                    o.w[c] = pack16x2<kHalf>(__fmul_rn(wj[jj], g[2 * c]), __fmul_rn(wj[jj], g[2 * c + 1]));
                 units::st32(grad_y + (int64_t)dj[jj] * vpr + v, o);
             }
         }
@@ -220,22 +212,23 @@ combine_backward_v32_kernel(const units::Vec32* __restrict__ grad_out,
 
 cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
                                     int64_t y_rows, const float* w, int H, void* grad_y,
-                                    int64_t grad_y_rows, float* grad_w, cudaStream_t s)
+                                    int64_t grad_y_rows, float* grad_w, bool half, cudaStream_t s)
 {
     if (h.T == 0)
         return cudaSuccess;
     if (H % 16 == 0 && ((uintptr_t)grad_out & 31u) == 0 && ((uintptr_t)y & 31u) == 0 &&
         ((uintptr_t)grad_y & 31u) == 0) {
         const unsigned grid = (unsigned)((h.T + 7) / 8);  // one warp per token
-        return launch_pdl(combine_backward_v32_kernel, grid, 256u, 0, s,
-                          static_cast<const units::Vec32*>(grad_out),
+        auto kern = half ? combine_backward_v32_kernel<true> : combine_backward_v32_kernel<false>;
+        return launch_pdl(kern, grid, 256u, 0, s, static_cast<const units::Vec32*>(grad_out),
                           static_cast<const units::Vec32*>(y), y_rows, w, h.T, h.k,
                           (int64_t)H / 16, h.dst_row, static_cast<units::Vec32*>(grad_y),
                           grad_y_rows, grad_w, h.err);
     }
     const int64_t vpr = H / 8;
     const int threads = (int)std::min<int64_t>(kMaxThreads, 32 * ((vpr + 31) / 32));
-    return launch_pdl(combine_backward_kernel, (unsigned)h.T, (unsigned)threads, 0, s,
+    auto kern = half ? combine_backward_kernel<true> : combine_backward_kernel<false>;
+    return launch_pdl(kern, (unsigned)h.T, (unsigned)threads, 0, s,
                       static_cast<const uint4*>(grad_out), static_cast<const uint4*>(y), y_rows, w,
                       h.T, h.k, vpr, h.dst_row, static_cast<uint4*>(grad_y), grad_y_rows, grad_w,
                       h.err);

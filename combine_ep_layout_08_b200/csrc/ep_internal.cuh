@@ -147,7 +147,8 @@ cudaError_t launch_combine(const Handle& h, const void* y, int64_t y_rows, const
                            cudaStream_t s);  // w == nullptr: unit weights; half: y, out binary16
 cudaError_t launch_combine_backward(const Handle& h, const void* grad_out, const void* y,
                                     int64_t y_rows, const float* w, int H, void* grad_y,
-                                    int64_t grad_y_rows, float* grad_w, cudaStream_t s);
+                                    int64_t grad_y_rows, float* grad_w, bool half,
+                                    cudaStream_t s);  // half: the rows are binary16
 
 // Per-rank receive buffers of the expert-parallel entry points, passed by
 // value: base[p] (rows of the layout's rank-p block, renumbered from 0),

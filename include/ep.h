@@ -358,6 +358,18 @@ ep_status_t ep_combine_backward(ep_handle_t h, const void* grad_out, const void*
                                 int64_t y_rows, const float* topk_weights, int H, void* grad_y,
                                 int64_t grad_y_rows, float* grad_weights, void* stream);
 
+/* The two backward calls with the type of the 16-bit rows named:
+ * EP_DTYPE_BF16 is the calls above; EP_DTYPE_FP16 takes binary16 gradient and
+ * expert-output rows (widened exactly) and writes binary16 grad_x / grad_y
+ * (round to nearest even), with the same fp32 arithmetic and order; grad_w
+ * stays fp32. */
+ep_status_t ep_dispatch_backward_ex(ep_handle_t h, const void* grad_recv, int64_t grad_rows, int H,
+                                    ep_dtype_t dtype, void* grad_x, void* stream);
+ep_status_t ep_combine_backward_ex(ep_handle_t h, const void* grad_out, const void* y,
+                                   int64_t y_rows, const float* topk_weights, int H,
+                                   ep_dtype_t dtype, void* grad_y, int64_t grad_y_rows,
+                                   float* grad_weights, void* stream);
+
 /* Wait for the stream (SYNCHRONISING), read and clear the sticky device
  * error word.  Returns EP_ERR_TIMEOUT, EP_ERR_BAD_INDEX or EP_ERR_CAPACITY
  * (in that order of precedence when several are set) or EP_OK. */

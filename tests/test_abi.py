@@ -183,3 +183,18 @@ def test_newer_entry_points_rejected_before_any_launch(lib):
     assert lib.ep_layout_dispatch(h, P(0x1000), 65, P(0x2000), 256, 0, P(0x3000), None, 8, None) \
         == EP_ERR_INVALID_ARG                                   # T > max_tokens
     lib.ep_handle_destroy(h)
+
+
+def test_backward_ex_rejected_before_any_launch(lib):
+    from combine_ep_layout_08_b200 import EP_ERR_INVALID_ARG, EP_ERR_STATE, ep_workspace_bytes
+
+    need = ep_workspace_bytes(64, 2, 16, 4)
+    st, h = _create(lib, 0x7f0000000000, need, 64, 2, 16, 4, 128)
+    assert st == 0
+    P = ctypes.c_void_p
+    assert lib.ep_dispatch_backward_ex(h, P(0x1000), 8, 256, 1, P(0x2000), None) == EP_ERR_STATE
+    assert lib.ep_dispatch_backward_ex(h, P(0x1000), 8, 256, 3, P(0x2000), None) \
+        == EP_ERR_INVALID_ARG                                   # unknown dtype
+    assert lib.ep_combine_backward_ex(h, P(0x1000), P(0x2000), 8, P(0x3000), 256, 1, P(0x4000),
+                                      8, P(0x5000), None) == EP_ERR_STATE
+    lib.ep_handle_destroy(h)

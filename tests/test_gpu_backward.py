@@ -107,3 +107,57 @@ def test_combine_backward_full_dsv3_shape(oracle):
     # typical error is far inside the worst-case bound
     rel = np.abs(gw - ref) / np.maximum(np.abs(ref), 1e-6)
     assert np.median(rel) < 1e-5
+
+
+def _f16(bits):
+    from gpu_util import DEV
+
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.float16).to(DEV)
+
+
+def _f16_bits(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("T,H,E,R,k,p_unused", [
+    (200, 1032, 32, 8, 8, 0.1),     # 16-byte rows: the fallback kernels
+    (64, 7168, 256, 8, 8, 0.0),     # 32-byte rows
+    (40, 2048, 64, 8, 20, 0.2),     # k > 8: slots in batches of 8
+])
+def test_backward_fp16(oracle, T, H, E, R, k, p_unused):
+    """fp16 rows: dispatch backward bit-exact; combine backward grad_y
+    bit-exact, grad_w within the fp32 summation bound of the fp64 dot."""
+    import combine_ep_layout_08_b200 as ep
+    from workloads import make_x_fp16
+
+    rng = np.random.default_rng(5 * T + H + k)
+    idx, w = random_topk(T, E, k, rng, p_unused=p_unused)
+    lay = oracle.layout(idx, E, R)
+    P = max(lay.total_rows, 1)
+    h = _setup(idx, E, R)
+    g = make_x_fp16(P, H, rng)
+    gx = ep.ep_dispatch_backward(h, _f16(g))
+    ep.ep_handle_check(h)
+    assert gx.dtype == torch.float16
+    assert np.array_equal(_f16_bits(gx), oracle.dispatch_backward(g, lay.dst_row, dtype="fp16"))
+
+    y = make_x_fp16(P, H, rng)
+    go = make_x_fp16(T, H, rng)
+    from gpu_util import DEV
+
+    gy, gw = ep.ep_combine_backward(h, _f16(go), _f16(y), torch.from_numpy(w).to(DEV))
+    ep.ep_handle_check(h)
+    gy_ref, gw_ref = oracle.combine_backward(go, y, w, lay.dst_row, dtype="fp16")
+    rows = lay.dst_row[lay.dst_row >= 0]
+    assert np.array_equal(_f16_bits(gy)[rows], gy_ref[rows])
+    gwg = gw.cpu().numpy()
+    yf = oracle.fp16_to_f32(y).astype(np.float64)
+    gf = oracle.fp16_to_f32(go).astype(np.float64)
+    for t in range(T):
+        for j in range(k):
+            d = lay.dst_row[t, j]
+            if d < 0:
+                assert gwg[t, j] == 0.0
+                continue
+            bound = H * 2.0 ** -24 * float(np.abs(gf[t] * yf[d]).sum()) + 2.0 ** -24 * abs(gw_ref[t, j])
+            assert abs(float(gwg[t, j]) - float(gw_ref[t, j])) <= bound + 1e-30, (t, j)
