@@ -37,7 +37,7 @@ __all__ = [
     "ep_layout", "ep_layout_dispatch", "ep_handle_view", "ep_handle_read_counts", "ep_dispatch", "ep_combine",
     "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_weights", "ep_zero_pad_rows", "ep_dispatch_ranks", "ep_combine_ranks",
-    "ep_allgather_topk",
+    "ep_dispatch_ranks_backward", "ep_combine_ranks_backward", "ep_allgather_topk",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
@@ -129,6 +129,8 @@ def load_library():
             "ep_dispatch_ex": ([P, P, I, I, I, P, P, I64, P], I),
             "ep_dispatch_ranks": ([P, I, I, P, I, I, P, P, P, P], I),
             "ep_dispatch_backward_ex": ([P, P, I64, I, I, P, P], I),
+            "ep_dispatch_ranks_backward": ([P, I, I, P, P, I, I, P, P], I),
+            "ep_combine_ranks_backward": ([P, I, I, P, P, P, P, I, I, P, P, P, P], I),
             "ep_combine_backward_ex": ([P, P, P, I64, P, I, I, P, I64, P, P], I),
             "ep_combine_ranks": ([P, I, I, P, P, P, I, I, P, P], I),
             "ep_combine_ex": ([P, P, I64, P, I, I, P, P], I),
@@ -520,6 +522,53 @@ def ep_combine_ranks(h: EPHandle, t_begin: int, y: list, topk_weights_rows: torc
         _check(load_library().ep_combine_ranks(
             h.handle, t_begin, n, ptrs, rows, _ptr(topk_weights_rows), H, _DTYPES[out_rows.dtype],
             _ptr(out_rows), _stream(h.device)), "ep_combine_ranks")
+
+
+def ep_dispatch_ranks_backward(h: EPHandle, t_begin: int, grad_recv: list,
+                               grad_x_rows: torch.Tensor) -> None:
+    """Backward of ep_dispatch_ranks for tokens [t_begin, t_begin + len(grad_x_rows)):
+    the fp32 sum, in slot order, of each token's slot rows of the ranks' gradient
+    buffers grad_recv[p], rounded to grad_x_rows' type (bf16 or fp16)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_dispatch_ranks_backward")
+    n, H = grad_x_rows.shape
+    if (grad_x_rows.dtype not in _DTYPES or not grad_x_rows.is_contiguous() or
+            len(grad_recv) != h.R or any(t.dtype != grad_x_rows.dtype or t.shape[1] != H or
+                                         not t.is_contiguous() for t in grad_recv)):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks_backward: bad tensor")
+    ptrs = _table([_ptr(t) for t in grad_recv], ctypes.c_void_p)
+    rows = _table([t.shape[0] for t in grad_recv], ctypes.c_int64)
+    with _on(h):
+        _check(load_library().ep_dispatch_ranks_backward(
+            h.handle, t_begin, n, ptrs, rows, H, _DTYPES[grad_x_rows.dtype], _ptr(grad_x_rows),
+            _stream(h.device)), "ep_dispatch_ranks_backward")
+
+
+def ep_combine_ranks_backward(h: EPHandle, t_begin: int, grad_out_rows: torch.Tensor, y: list,
+                              topk_weights_rows: torch.Tensor, grad_y: list) -> torch.Tensor:
+    """Backward of ep_combine_ranks for tokens [t_begin, t_begin + len(grad_out_rows)):
+    writes each used slot's row of grad_y[p] (w * grad_out, rounded) and returns
+    grad_weights f32 [n, k] (dot products of grad_out with the slots' y rows)."""
+    if h.T is None:
+        raise EPError(EP_ERR_STATE, "ep_combine_ranks_backward")
+    n, H = grad_out_rows.shape
+    dt = grad_out_rows.dtype
+    if (dt not in _DTYPES or not grad_out_rows.is_contiguous() or len(y) != h.R
+            or len(grad_y) != h.R or topk_weights_rows.dtype != torch.float32
+            or tuple(topk_weights_rows.shape) != (n, h.k) or not topk_weights_rows.is_contiguous()
+            or any(t.dtype != dt or t.shape[1] != H or not t.is_contiguous()
+                   for t in list(y) + list(grad_y))):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_ranks_backward: bad tensor")
+    grad_w = torch.empty((n, h.k), dtype=torch.float32, device=grad_out_rows.device)
+    yp = _table([_ptr(t) for t in y], ctypes.c_void_p)
+    yr = _table([t.shape[0] for t in y], ctypes.c_int64)
+    gp = _table([_ptr(t) for t in grad_y], ctypes.c_void_p)
+    gr = _table([t.shape[0] for t in grad_y], ctypes.c_int64)
+    with _on(h):
+        _check(load_library().ep_combine_ranks_backward(
+            h.handle, t_begin, n, _ptr(grad_out_rows), yp, yr, _ptr(topk_weights_rows), H,
+            _DTYPES[dt], gp, gr, _ptr(grad_w), _stream(h.device)), "ep_combine_ranks_backward")
+    return grad_w
 
 
 def ep_allgather_topk(topk_idx: torch.Tensor, group=None):

@@ -565,6 +565,95 @@ ep_status_t ep_combine_ranks(ep_handle_t hh, int t_begin, int t_count, const voi
     return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine_ranks");
 }
 
+namespace {
+
+// A host table of R (pointer, rows) pairs into a RankTable; alignment of
+// every non-empty entry checked.
+ep_status_t fill_rank_table(const Handle* h, const void* const* ptrs, const int64_t* rows,
+                            int align, ep::RankTable* tab)
+{
+    if (h->R > EP_MAX_RANK_TABLE || !ptrs || !rows)
+        return EP_ERR_INVALID_ARG;
+    for (int p = 0; p < h->R; ++p) {
+        if (rows[p] < 0 || (rows[p] > 0 && !ptrs[p]))
+            return EP_ERR_INVALID_ARG;
+        if (!ep::aligned(ptrs[p], align))
+            return EP_ERR_ALIGNMENT;
+        tab->base[p] = const_cast<void*>(ptrs[p]);
+        tab->rows[p] = rows[p];
+    }
+    return EP_OK;
+}
+
+ep_status_t range_check(const Handle* h, int t_begin, int t_count)
+{
+    if (!h->has_layout)
+        return EP_ERR_STATE;
+    if (t_begin < 0 || t_count < 0 || (int64_t)t_begin + t_count > h->T)
+        return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+}  // namespace
+
+ep_status_t ep_dispatch_ranks_backward(ep_handle_t hh, int t_begin, int t_count,
+                                       const void* const* grad_recv, const int64_t* grad_rows,
+                                       int H, ep_dtype_t dtype, void* grad_x_rows, void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 8 != 0 || (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16))
+        return EP_ERR_INVALID_ARG;
+    ep_status_t st = range_check(h, t_begin, t_count);
+    if (st != EP_OK)
+        return st;
+    if (t_count > 0 && !grad_x_rows)
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(grad_x_rows, 16))
+        return EP_ERR_ALIGNMENT;
+    ep::RankTable tab = {};
+    if ((st = fill_rank_table(h, grad_recv, grad_rows, 16, &tab)) != EP_OK)
+        return st;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaError_t rc = ep::launch_combine_ranks(sub, nullptr, H, dtype == EP_DTYPE_FP16, tab,
+                                              grad_x_rows, static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_dispatch_ranks_backward");
+}
+
+ep_status_t ep_combine_ranks_backward(ep_handle_t hh, int t_begin, int t_count,
+                                      const void* grad_out_rows, const void* const* y,
+                                      const int64_t* y_rows, const float* topk_weights_rows, int H,
+                                      ep_dtype_t dtype, void* const* grad_y,
+                                      const int64_t* grad_y_rows, float* grad_weights_rows,
+                                      void* stream)
+{
+    Handle* h = ep::as_handle(hh);
+    if (!h || H <= 0 || H % 16 != 0 || (dtype != EP_DTYPE_BF16 && dtype != EP_DTYPE_FP16))
+        return EP_ERR_INVALID_ARG;
+    ep_status_t st = range_check(h, t_begin, t_count);
+    if (st != EP_OK)
+        return st;
+    if (t_count > 0 && (!grad_out_rows || !topk_weights_rows || !grad_weights_rows))
+        return EP_ERR_INVALID_ARG;
+    if (!ep::aligned(grad_out_rows, 32) || !ep::aligned(topk_weights_rows, 4) ||
+        !ep::aligned(grad_weights_rows, 4))
+        return EP_ERR_ALIGNMENT;
+    ep::RankTable ytab = {}, gytab = {};
+    if ((st = fill_rank_table(h, y, y_rows, 32, &ytab)) != EP_OK)
+        return st;
+    if ((st = fill_rank_table(h, const_cast<const void* const*>(grad_y), grad_y_rows, 32,
+                              &gytab)) != EP_OK)
+        return st;
+    Handle sub = *h;
+    sub.T = t_count;
+    sub.dst_row = h->dst_row + (int64_t)t_begin * h->k;
+    cudaError_t rc = ep::launch_combine_ranks_backward(
+        sub, grad_out_rows, topk_weights_rows, H, dtype == EP_DTYPE_FP16, ytab, gytab,
+        grad_weights_rows, static_cast<cudaStream_t>(stream));
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_combine_ranks_backward");
+}
+
 ep_status_t ep_dispatch_weights(ep_handle_t hh, const float* topk_weights, float* recv_weights,
                                 int64_t recv_capacity_rows, void* stream)
 {

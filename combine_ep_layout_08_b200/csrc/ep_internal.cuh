@@ -162,7 +162,11 @@ struct RankTable {
 cudaError_t launch_dispatch_ranks(const Handle& h, const void* x, int H, bool fp8, bool half,
                                   const RankTable& tab, cudaStream_t s);
 cudaError_t launch_combine_ranks(const Handle& h, const float* w, int H, bool half,
-                                 const RankTable& tab, void* out, cudaStream_t s);
+                                 const RankTable& tab, void* out,
+                                 cudaStream_t s);  // w == nullptr: unit weights
+cudaError_t launch_combine_ranks_backward(const Handle& h, const void* grad_out, const float* w,
+                                          int H, bool half, const RankTable& ytab,
+                                          const RankTable& gytab, float* grad_w, cudaStream_t s);
 
 // Persistent-grid size: min(resident blocks per SM from the occupancy API,
 // max_per_sm) x the SM count of the current device, cached per kernel and

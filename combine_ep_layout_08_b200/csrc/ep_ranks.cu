@@ -192,7 +192,8 @@ combine_ranks_kernel(const float* __restrict__ weights, int T, int k, int64_t vp
     for (int64_t u = wg; u < (int64_t)T * upr; u += nw) {
         const int64_t t = u / upr;
         const int64_t v0 = (u - t * upr) * (32 * kU) + lane;
-        const float w = lane < k ? __ldg(weights + t * k + lane) : 0.0f;
+        // null weights: unit weights (the backward of dispatch)
+        const float w = lane < k ? (weights ? __ldg(weights + t * k + lane) : 1.0f) : 0.0f;
         int64_t local;
         const int p = slot_rank(dst_row, t, k, s_roff, R, tab, kErrCombineCap, err, &local);
         const uint64_t rowp =
@@ -254,6 +255,103 @@ combine_ranks_kernel(const float* __restrict__ weights, int T, int k, int64_t vp
     }
 }
 
+// Backward of the per-rank combine, one warp per token (32-byte vectors):
+// grad_y of slot j, in its rank's grad_y buffer, = rn16(w[t][j] * grad_out[t])
+// (one fp32 product: bit-exact), and grad_w[t][j] = the fp32 dot product of
+// grad_out[t] with the slot's expert-output row, read from its rank's y
+// buffer -- units in order, channels in order within the lane, then a fixed
+// xor-shuffle tree over the lanes (bitwise repeatable).  ytab and gytab hold
+// the ranks' y and grad_y buffers.
+template <bool kHalf>
+__global__ void __launch_bounds__(kThreads)
+combine_ranks_backward_kernel(const Vec32* __restrict__ grad_out, const float* __restrict__ weights,
+                              int T, int k, int64_t vpr, const int32_t* __restrict__ dst_row,
+                              const int32_t* __restrict__ rank_off, int R, RankTable ytab,
+                              RankTable gytab, float* __restrict__ grad_w, int32_t* err)
+{
+    extern __shared__ int32_t s_roff[];
+    pdl_wait();
+    pdl_trigger();
+    load_rank_off(rank_off, R, s_roff);
+    constexpr int kBatch = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T)
+        return;
+    float w = 0.0f;
+    uint64_t yrow = 0ull, gyrow = 0ull;
+    if (lane < k) {
+        w = __ldg(weights + t * k + lane);
+        const int32_t d = __ldg(dst_row + t * k + lane);
+        if (d >= 0) {
+            const int p = rank_of_row(s_roff, R, d);
+            const int64_t local = (int64_t)d - s_roff[p];
+            if (local >= ytab.rows[p] || local >= gytab.rows[p]) {
+                atomicOr(err, kErrCombineCap);
+            } else {
+                yrow = (uint64_t)(static_cast<const Vec32*>(ytab.base[p]) + local * vpr);
+                gyrow = (uint64_t)(static_cast<Vec32*>(gytab.base[p]) + local * vpr);
+            }
+        }
+    }
+    const int64_t upr = (vpr + 31) / 32;
+    const Vec32* g_row = grad_out + t * vpr;
+    for (int j0 = 0; j0 < k; j0 += kBatch) {
+        const int nj = min(kBatch, k - j0);
+        uint64_t yj[kBatch], gj[kBatch];
+        float wj[kBatch], part[kBatch];
+#pragma unroll
+        for (int jj = 0; jj < kBatch; ++jj) {
+            yj[jj] = __shfl_sync(kFull, yrow, (j0 + jj) & 31);
+            gj[jj] = __shfl_sync(kFull, gyrow, (j0 + jj) & 31);
+            wj[jj] = __shfl_sync(kFull, w, (j0 + jj) & 31);
+            if (jj >= nj)
+                yj[jj] = 0ull;
+            part[jj] = 0.0f;
+        }
+        for (int64_t u = 0; u < upr; ++u) {
+            const int64_t v = u * 32 + lane;
+            if (v >= vpr)
+                continue;  // only the last unit is ragged; no shuffles below
+            const Vec32 gv = units::ld32_once(g_row + v);
+            Vec32 yv[kBatch];
+#pragma unroll
+            for (int jj = 0; jj < kBatch; ++jj)
+                if (yj[jj] != 0ull)
+                    yv[jj] = units::ld32_once(reinterpret_cast<const Vec32*>(yj[jj]) + v);
+            float g[16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                g[2 * c] = lo16<kHalf>(gv.w[c]);
+                g[2 * c + 1] = hi16<kHalf>(gv.w[c]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < kBatch; ++jj) {
+                if (yj[jj] == 0ull)
+                    continue;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    part[jj] = __fmaf_rn(g[2 * c], lo16<kHalf>(yv[jj].w[c]), part[jj]);
+                    part[jj] = __fmaf_rn(g[2 * c + 1], hi16<kHalf>(yv[jj].w[c]), part[jj]);
+                }
+                Vec32 o;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    o.w[c] = pack16x2<kHalf>(__fmul_rn(wj[jj], g[2 * c]),
+                                             __fmul_rn(wj[jj], g[2 * c + 1]));
+                units::st32(reinterpret_cast<Vec32*>(gj[jj]) + v, o);
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kBatch; ++jj)
+            for (int o = 16; o > 0; o >>= 1) part[jj] += __shfl_xor_sync(kFull, part[jj], o);
+#pragma unroll
+        for (int jj = 0; jj < kBatch; ++jj)
+            if (lane == jj && jj < nj)
+                grad_w[t * k + j0 + jj] = yj[jj] != 0ull ? part[jj] : 0.0f;
+    }
+}
+
 unsigned warp_grid(int64_t units)
 {
     const int64_t warps = kThreads / 32;
@@ -276,6 +374,20 @@ cudaError_t launch_dispatch_ranks(const Handle& h, const void* x, int H, bool fp
     auto kern = half ? dispatch_ranks_fp8_kernel<true> : dispatch_ranks_fp8_kernel<false>;
     return launch_pdl(kern, warp_grid(h.T * ((vpr + 31) / 32)), kThreads, smem, s,
                       static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row, h.rank_off, h.R, tab,
+                      h.err);
+}
+
+cudaError_t launch_combine_ranks_backward(const Handle& h, const void* grad_out, const float* w,
+                                          int H, bool half, const RankTable& ytab,
+                                          const RankTable& gytab, float* grad_w, cudaStream_t s)
+{
+    if (h.T == 0)
+        return cudaSuccess;
+    const size_t smem = sizeof(int32_t) * (size_t)(h.R + 1);
+    auto kern = half ? combine_ranks_backward_kernel<true> : combine_ranks_backward_kernel<false>;
+    const unsigned grid = (unsigned)((h.T + 7) / 8);  // one warp per token
+    return launch_pdl(kern, grid, kThreads, smem, s, static_cast<const Vec32*>(grad_out), w, h.T,
+                      h.k, (int64_t)H / 16, h.dst_row, h.rank_off, h.R, ytab, gytab, grad_w,
                       h.err);
 }
 

@@ -306,6 +306,29 @@ ep_status_t ep_combine_ranks(ep_handle_t h, int t_begin, int t_count, const void
                              const int64_t* y_rows, const float* topk_weights_rows, int H,
                              ep_dtype_t dtype, void* out_rows, void* stream);
 
+/* Backward of the two calls above, for the source's tokens [t_begin,
+ * t_begin + t_count) of the global layout (rows bf16 or fp16 as dtype).
+ * ep_dispatch_ranks_backward: grad_x_rows[t] = the fp32 sum, in slot order,
+ *   of the slot rows of the ranks' gradient buffers grad_recv[p] (HOST table
+ *   of R device pointers, 16-byte aligned, grad_rows[p] rows), rounded to
+ *   dtype -- ep_combine_ranks with unit weights.  H % 8 == 0.
+ * ep_combine_ranks_backward: for every used slot, rank p's grad_y[p] row =
+ *   rn16(w * grad_out[t]) (one fp32 product) and grad_weights[t][j] = the
+ *   fp32 dot product of grad_out[t] with the slot's row of y[p] (fixed
+ *   reduction order: bitwise repeatable).  y and grad_y: HOST tables of R
+ *   device pointers with y_rows / grad_y_rows rows, 32-byte aligned;
+ *   grad_out_rows device [t_count][H], 32-byte aligned; H % 16 == 0.
+ * Rows past a rank's capacity are skipped and set EP_ERR_CAPACITY. */
+ep_status_t ep_dispatch_ranks_backward(ep_handle_t h, int t_begin, int t_count,
+                                       const void* const* grad_recv, const int64_t* grad_rows,
+                                       int H, ep_dtype_t dtype, void* grad_x_rows, void* stream);
+ep_status_t ep_combine_ranks_backward(ep_handle_t h, int t_begin, int t_count,
+                                      const void* grad_out_rows, const void* const* y,
+                                      const int64_t* y_rows, const float* topk_weights_rows, int H,
+                                      ep_dtype_t dtype, void* const* grad_y,
+                                      const int64_t* grad_y_rows, float* grad_weights_rows,
+                                      void* stream);
+
 /* GEMM-ready receive layout.  The pages say the high-throughput and
  * low-latency kernels share one "GEMM layout" (DeepEP v2 release notes, "Có
  * gì mới trong v2") without defining it; these helpers complete the reading

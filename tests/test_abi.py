@@ -198,3 +198,21 @@ def test_backward_ex_rejected_before_any_launch(lib):
     assert lib.ep_combine_backward_ex(h, P(0x1000), P(0x2000), 8, P(0x3000), 256, 1, P(0x4000),
                                       8, P(0x5000), None) == EP_ERR_STATE
     lib.ep_handle_destroy(h)
+
+
+def test_ranks_backward_rejected_before_any_launch(lib):
+    from combine_ep_layout_08_b200 import EP_ERR_INVALID_ARG, EP_ERR_STATE, ep_workspace_bytes
+
+    need = ep_workspace_bytes(64, 2, 16, 4)
+    st, h = _create(lib, 0x7f0000000000, need, 64, 2, 16, 4, 128)
+    assert st == 0
+    P = ctypes.c_void_p
+    tab = (ctypes.c_void_p * 4)(0x1000, 0x2000, 0x3000, 0x4000)
+    rows = (ctypes.c_int64 * 4)(8, 8, 8, 8)
+    assert lib.ep_dispatch_ranks_backward(h, 0, 0, tab, rows, 256, 0, P(0x5000), None) \
+        == EP_ERR_STATE
+    assert lib.ep_combine_ranks_backward(h, 0, 0, P(0x5000), tab, rows, P(0x6000), 256, 0, tab,
+                                         rows, P(0x7000), None) == EP_ERR_STATE
+    assert lib.ep_combine_ranks_backward(h, 0, 0, P(0x5000), tab, rows, P(0x6000), 200, 0, tab,
+                                         rows, P(0x7000), None) == EP_ERR_INVALID_ARG  # H % 16
+    lib.ep_handle_destroy(h)

@@ -220,3 +220,60 @@ def test_ranks_fp16_copy_and_cuda_graph_replay(oracle):
             assert np.array_equal(_bits(recv[p])[rows], ref[a:b][rows]), (rep, p)
         assert np.array_equal(_bits(out), oracle.combine(y, w, lay.dst_row, dtype="fp16")), rep
     del g
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("counts,E,R,k,H", [
+    ([50, 0, 77, 31], 32, 4, 8, 1024),
+    ([30, 33], 16, 2, 12, 256),            # k > 8: two slot batches
+])
+def test_backward_ranks_matches_the_global_backward(oracle, dtype, counts, E, R, k, H):
+    """Per-rank backward: dispatch backward bit-exact; combine backward grad_y
+    bit-exact on every used row and grad_w within the fp32 summation bound of
+    the oracle's fp64 dot product."""
+    import combine_ep_layout_08_b200 as ep
+
+    h, lay, idx, w, _, rng, starts = _setup(oracle, counts, E, R, k, H, 9 * sum(counts) + k)
+    P = max(lay.total_rows, 1)
+    gen = make_x if dtype == "bf16" else make_x_fp16
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    to_dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt).to(DEV)
+    blocks = _rank_rows(lay, R)
+    T = sum(counts)
+    # dispatch backward
+    g = gen(P, H, rng)
+    gd = to_dev(g)
+    gr = [gd[a:b].clone() if b > a else torch.zeros((1, H), dtype=tdt, device=DEV) for a, b in blocks]
+    gx = torch.zeros((T, H), dtype=tdt, device=DEV)
+    for s, n in zip(starts, counts):
+        ep.ep_dispatch_ranks_backward(h, int(s), gr, gx[s:s + n])
+    ep.ep_handle_check(h)
+    assert np.array_equal(_bits(gx), oracle.dispatch_backward(g, lay.dst_row, dtype=dtype))
+    # combine backward
+    y = gen(P, H, rng)
+    go = gen(T, H, rng)
+    yd = to_dev(y)
+    ys = [yd[a:b].clone() if b > a else torch.zeros((1, H), dtype=tdt, device=DEV) for a, b in blocks]
+    gys = [torch.zeros_like(t) for t in ys]
+    god = to_dev(go)
+    wd = torch.from_numpy(w).to(DEV)
+    gw = torch.zeros((T, k), dtype=torch.float32, device=DEV)
+    for s, n in zip(starts, counts):
+        gw[s:s + n] = ep.ep_combine_ranks_backward(h, int(s), god[s:s + n].contiguous(), ys,
+                                                   wd[s:s + n].contiguous(), gys)
+    ep.ep_handle_check(h)
+    gy_ref, gw_ref = oracle.combine_backward(go, y, w, lay.dst_row, dtype=dtype)
+    used = lay.dst_row[lay.dst_row >= 0]
+    for p, (a, b) in enumerate(blocks):
+        rows = used[(used >= a) & (used < b)]
+        assert np.array_equal(_bits(gys[p])[rows - a], gy_ref[rows]), p
+    to32 = oracle.bf16_to_f32 if dtype == "bf16" else oracle.fp16_to_f32
+    yf, gf, gwg = to32(y).astype(np.float64), to32(go).astype(np.float64), gw.cpu().numpy()
+    for t in range(T):
+        for j in range(k):
+            d = lay.dst_row[t, j]
+            if d < 0:
+                assert gwg[t, j] == 0.0
+                continue
+            bound = H * 2.0 ** -24 * float(np.abs(gf[t] * yf[d]).sum()) + 2.0 ** -24 * abs(gw_ref[t, j])
+            assert abs(float(gwg[t, j]) - float(gw_ref[t, j])) <= bound + 1e-30, (t, j)
