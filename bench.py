@@ -471,9 +471,37 @@ def time_ranks(dev, flush, seed, steps):
                      "dispatch_GBps": round(db / (d_ms / 1e3) / 1e9, 1),
                      "combine_us": round(c_ms * 1e3, 2),
                      "combine_GBps": round(cb / (c_ms / 1e3) / 1e9, 1)}
+    # the backward of both, one launch over all tokens
+    gys = [torch.empty_like(t) for t in ys]
+    go = torch.randn((w.T, w.H), device=dev).to(torch.bfloat16)
+    gx = torch.empty_like(out)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(3 + steps):
+        flush()
+        e = ev[i - 3] if i >= 3 else None
+        if e:
+            e[0].record()
+        ep.ep_dispatch_ranks_backward(h, 0, recv, gx)
+        if e:
+            e[1].record()
+        ep.ep_combine_ranks_backward(h, 0, go, ys, wt, gys)
+        if e:
+            e[2].record()
+    torch.cuda.synchronize()
+    d_ms = statistics.mean(a[0].elapsed_time(a[1]) for a in ev)
+    c_ms = statistics.mean(a[1].elapsed_time(a[2]) for a in ev)
+    db, _ = algo_bytes(w.T, w.H, w.k, w.fmt)
+    # grad_out and k y rows read, k grad_y rows and grad_w written (as time_backward)
+    cbb = w.T * 2 * w.H + 2 * w.T * w.k * 2 * w.H + w.T * w.k * 4
+    res["backward_one_launch"] = {
+        "dispatch_backward_us": round(d_ms * 1e3, 2),
+        "dispatch_backward_GBps": round(db / (d_ms / 1e3) / 1e9, 1),
+        "combine_backward_us": round(c_ms * 1e3, 2),
+        "combine_backward_GBps": round(cbb / (c_ms / 1e3) / 1e9, 1)}
     ep.ep_handle_check(h)
     res["workload"] = ("8k routing as R = 8 ranks on one GPU, 8 separate receive buffers, BF16; "
-                       "dispatch_ranks / combine_ranks (no NVLink: the ranks' buffers are local)")
+                       "dispatch_ranks / combine_ranks and their backward (no NVLink: the ranks' "
+                       "buffers are local)")
     return res
 
 

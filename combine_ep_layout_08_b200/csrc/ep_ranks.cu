@@ -263,7 +263,7 @@ combine_ranks_kernel(const float* __restrict__ weights, int T, int k, int64_t vp
 // xor-shuffle tree over the lanes (bitwise repeatable).  ytab and gytab hold
 // the ranks' y and grad_y buffers.
 template <bool kHalf>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 combine_ranks_backward_kernel(const Vec32* __restrict__ grad_out, const float* __restrict__ weights,
                               int T, int k, int64_t vpr, const int32_t* __restrict__ dst_row,
                               const int32_t* __restrict__ rank_off, int R, RankTable ytab,
