@@ -243,7 +243,34 @@ def gpu_setup(name, seed, dev):
     else:
         y[:P] = (recv[:P].float() * scales[:P].repeat_interleave(128, 1) * c).to(torch.bfloat16)
     ep.ep_handle_check(h)
-    return dict(w=w, h=h, x=x, idx=idx, wt=wt, recv=recv, scales=scales, out=out, y=y, P=P)
+    return dict(w=w, h=h, x=x, idx=idx, wt=wt, recv=recv, scales=scales, out=out, y=y, P=P,
+                routing=routing_stats(ep.ep_handle_read_counts(h), w))
+
+
+def routing_stats(c: dict, w) -> dict:
+    """Load balance of the layout (read once, untimed): per-expert slot counts and
+    per-rank rows as max / mean, and the share of pad rows in the receive buffer."""
+    e = np.asarray(c["num_tokens_per_expert"], np.float64)
+    r = np.asarray(c["num_rows_per_rank"], np.float64)
+    P = max(int(c["total_recv_rows"]), 1)
+    return {"expert_slots_max": int(e.max()) if e.size else 0,
+            "expert_slots_max_over_mean": round(float(e.max() / max(e.mean(), 1e-9)), 3),
+            "rank_rows_max_over_mean": round(float(r.max() / max(r.mean(), 1e-9)), 3),
+            "receive_rows": P,
+            "pad_row_share": round(1.0 - float(e.sum()) / P, 4)}
+
+
+NVTX = False  # --nvtx: name the three calls for a profiler's timeline (off when timing)
+
+
+def _range(name):
+    import contextlib
+
+    import torch
+
+    if not NVTX:
+        return contextlib.nullcontext()
+    return torch.cuda.nvtx.range(name)
 
 
 def gpu_step(s, ev=None):
@@ -252,13 +279,16 @@ def gpu_step(s, ev=None):
     h, w = s["h"], s["w"]
     if ev is not None:
         ev[0].record()
-    ep.ep_layout(h, s["idx"])
+    with _range("ep_layout"):
+        ep.ep_layout(h, s["idx"])
     if ev is not None:
         ev[1].record()
-    ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+    with _range("ep_dispatch"):
+        ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
     if ev is not None:
         ev[2].record()
-    ep.ep_combine(h, s["y"], s["wt"], out=s["out"])
+    with _range("ep_combine"):
+        ep.ep_combine(h, s["y"], s["wt"], out=s["out"])
     if ev is not None:
         ev[3].record()
 
@@ -674,7 +704,11 @@ def main():
                          "or all")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--nvtx", action="store_true",
+                    help="NVTX ranges around the three calls (for a profiler's timeline)")
     args = ap.parse_args()
+    global NVTX
+    NVTX = args.nvtx
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -713,6 +747,7 @@ def main():
     peak, peak_src = load_peaks()
     s = gpu_setup(MAIN_WORKLOAD, args.seed + rank, dev)
     w = s["w"]
+    routing_main = s["routing"]
     bus = None
     try:
         bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
@@ -756,7 +791,7 @@ def main():
             n = max(3, min(args.steps, 100))
             t2 = time_gpu(s2, n, min(args.warmup, 10), flush, barrier)
             db, cb = algo_bytes(w2.T, w2.H, w2.k, w2.fmt)
-            ent = {"workload": WORKLOAD_TEXT[name],
+            ent = {"workload": WORKLOAD_TEXT[name], "routing": s2["routing"],
                    "step_us": round(statistics.mean(t2["step"]) * 1e3, 2),
                    "layout_us": round(statistics.mean(t2["layout"]) * 1e3, 2),
                    "dispatch_us": round(statistics.mean(t2["dispatch"]) * 1e3, 2),
@@ -809,7 +844,8 @@ def main():
                        "experts": w.E, "virtual_ranks": w.R, "topk": w.k, "fmt": w.fmt,
                        "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "flushed between steps (write of 2x L2), outside the events",
-                       "bytes_per_step": d_bytes + c_bytes},
+                       "bytes_per_step": d_bytes + c_bytes,
+                       "routing": routing_main},
             "pct_of_measured_hbm": round(value / world / peak, 4),
             "pct_of_hbm_spec_8TBps": round(value / world / 8000.0, 4),
             "kernels": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(dis_ms * 1e3, 2),

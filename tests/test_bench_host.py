@@ -121,3 +121,16 @@ def test_allgather_topk_gloo_world_2():
         assert p.exitcode == 0
     exp = [[2 * i, 2 * i + 1] for i in range(3)] + [[100 + 2 * i, 101 + 2 * i] for i in range(5)]
     assert res[0] == (exp, 0) and res[1] == (exp, 3)
+
+
+def test_routing_stats_closed_form():
+    import numpy as np
+
+    import bench
+
+    c = dict(num_tokens_per_expert=np.array([3, 1, 0, 4], np.int32),
+             num_tokens_per_rank=np.array([2, 2], np.int32),
+             num_rows_per_rank=np.array([4, 4], np.int32), total_recv_rows=16)
+    r = bench.routing_stats(c, None)
+    assert r["expert_slots_max"] == 4 and r["expert_slots_max_over_mean"] == 2.0
+    assert r["rank_rows_max_over_mean"] == 1.0 and r["pad_row_share"] == 0.5
