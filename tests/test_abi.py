@@ -216,3 +216,22 @@ def test_ranks_backward_rejected_before_any_launch(lib):
     assert lib.ep_combine_ranks_backward(h, 0, 0, P(0x5000), tab, rows, P(0x6000), 200, 0, tab,
                                          rows, P(0x7000), None) == EP_ERR_INVALID_ARG  # H % 16
     lib.ep_handle_destroy(h)
+
+
+def test_binding_constants_match_the_header():
+    """Status codes, formats, dtypes and limits the binding mirrors equal the
+    header's (parsed from the text)."""
+    import combine_ep_layout_08_b200 as ep
+
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    enums = dict((m.group(1), int(m.group(2)))
+                 for m in re.finditer(r"\b(EP_[A-Z0-9_]+)\s*=\s*(\d+)", src))
+    defines = dict((m.group(1), int(m.group(2)))
+                   for m in re.finditer(r"#define\s+(EP_[A-Z0-9_]+)\s+(\d+)", src))
+    for name in dir(ep):
+        if name.startswith(("EP_ERR_", "EP_FMT_", "EP_DTYPE_")) or name == "EP_OK":
+            assert name in enums, name
+            assert getattr(ep, name) == enums[name], name
+    assert enums["EP_FMT_FP16"] == ep._FMTS["fp16"]
+    assert defines["EP_MAX_RANK_TABLE"] >= 8
+    assert set(ep._DTYPES.values()) == {enums["EP_DTYPE_BF16"], enums["EP_DTYPE_FP16"]}
