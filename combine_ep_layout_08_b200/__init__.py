@@ -264,8 +264,9 @@ def ep_layout(h: EPHandle, topk_idx: torch.Tensor) -> None:
     """get_dispatch_layout of int64 [T, k] top-k indices (-1 = unused slot)."""
     if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or topk_idx.shape[1] != h.k:
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout: topk_idx must be int64 [T, %d]" % h.k)
-    if not topk_idx.is_cuda or not topk_idx.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_layout: topk_idx must be a contiguous CUDA tensor")
+    if not topk_idx.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout: topk_idx must be contiguous")
+    _same_device(h, "ep_layout", topk_idx)
     T = topk_idx.shape[0]
     with _on(h):
         _check(load_library().ep_layout(h.handle, _ptr(topk_idx), T, _stream(h.device)),
@@ -308,10 +309,47 @@ def ep_handle_read_counts(h: EPHandle) -> dict:
                 total_recv_rows=int(d[0]))
 
 
+def _same_device(h: EPHandle, where: str, *tensors) -> None:
+    """Every tensor given (None skipped) lives on the handle's device."""
+    for t in tensors:
+        if t is not None and t.device != h.device:
+            raise EPError(EP_ERR_INVALID_ARG, "%s: tensors must be on %s" % (where, h.device))
+
+
+def _rank_list(h: EPHandle, where: str, tensors) -> None:
+    """Per-rank buffers: 2-D, on a device of the handle's kind (CUDA; other
+    GPUs' buffers, seen as peers, are allowed)."""
+    for t in tensors:
+        if t.device.type != h.device.type or t.dim() != 2:
+            raise EPError(EP_ERR_INVALID_ARG, "%s: per-rank buffers must be 2-D %s tensors"
+                          % (where, h.device.type))
+
+
+def _check_recv(where: str, H: int, f: int, recv_x, recv_scales):
+    """Receive buffers of format f: recv_x [cap, H] of the format's type; FP8
+    scales f32 [>= cap, H/128] (row-major) or [H/128, cap] (MN-major)."""
+    want = _recv_dtype(f)
+    if (recv_x.dtype != want or recv_x.dim() != 2 or recv_x.shape[1] != H
+            or not recv_x.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "%s: recv_x must be contiguous %s [*, %d]"
+                      % (where, want, H))
+    cap = recv_x.shape[0]
+    if _is_copy(f):
+        return
+    if recv_scales is None or recv_scales.dtype != torch.float32 or recv_scales.dim() != 2 \
+            or not recv_scales.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "%s: FP8 needs contiguous f32 recv_scales" % where)
+    if f == EP_FMT_FP8_E4M3_1X128 and (recv_scales.shape[0] < cap
+                                       or recv_scales.shape[1] != H // 128):
+        raise EPError(EP_ERR_INVALID_ARG, "%s: recv_scales must be f32 [cap, H/128]" % where)
+    if f == EP_FMT_FP8_E4M3_1X128_MN and tuple(recv_scales.shape) != (H // 128, cap):
+        raise EPError(EP_ERR_INVALID_ARG, "%s: recv_scales must be f32 [H/128, cap]" % where)
+
+
 def _recv_buffers(h: EPHandle, T: int, H: int, f: int, device, recv_x, recv_scales,
-                  capacity_rows):
+                  capacity_rows, where: str):
     """Allocate missing receive buffers (default capacity: the no-sync bound)
-    and check the given ones."""
+    and check them."""
     if recv_x is None:
         cap = capacity_rows if capacity_rows is not None else \
             ep_recv_rows_upper_bound(T, h.k, h.E, h.block_m)
@@ -323,17 +361,8 @@ def _recv_buffers(h: EPHandle, T: int, H: int, f: int, device, recv_x, recv_scal
         recv_scales = torch.empty((cap, H // 128), dtype=torch.float32, device=device)
     if f == EP_FMT_FP8_E4M3_1X128_MN and recv_scales is None:
         recv_scales = torch.empty((H // 128, cap), dtype=torch.float32, device=device)
-    want = _recv_dtype(f)
-    if recv_x.dtype != want or recv_x.shape[1] != H or not recv_x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "recv_x must be contiguous %s [*, %d]" % (want, H))
-    if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128:
-        if (recv_scales.dtype != torch.float32 or recv_scales.shape[0] < cap
-                or recv_scales.shape[1] != H // 128 or not recv_scales.is_contiguous()):
-            raise EPError(EP_ERR_INVALID_ARG, "recv_scales must be f32 [cap, H/128]")
-    if recv_scales is not None and f == EP_FMT_FP8_E4M3_1X128_MN:
-        if (recv_scales.dtype != torch.float32 or tuple(recv_scales.shape) != (H // 128, cap)
-                or not recv_scales.is_contiguous()):
-            raise EPError(EP_ERR_INVALID_ARG, "recv_scales must be f32 [H/128, cap]")
+    _check_recv(where, H, f, recv_x, recv_scales)
+    _same_device(h, where, recv_x, recv_scales)
     return recv_x, (recv_scales if not _is_copy(f) else None)
 
 
@@ -358,7 +387,9 @@ def ep_dispatch(h: EPHandle, x: torch.Tensor, fmt: Optional[str] = None,
     f = _fmt_code(fmt, x.dtype)
     if _is_copy(f) and f != _COPY_FMT[x.dtype]:
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch: a row copy keeps x's type")
-    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
+    _same_device(h, "ep_dispatch", x)
+    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows,
+                                        "ep_dispatch")
     lib = load_library()
     with _on(h):
         if x.dtype == torch.bfloat16:
@@ -380,8 +411,8 @@ def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor,
     or fp16 copied as rows)."""
     if topk_idx.dtype != torch.int64 or topk_idx.dim() != 2 or topk_idx.shape[1] != h.k:
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be int64 [T, %d]" % h.k)
-    if not topk_idx.is_cuda or not topk_idx.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be contiguous CUDA")
+    if not topk_idx.is_contiguous():
+        raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: topk_idx must be contiguous")
     T = topk_idx.shape[0]
     if x.dtype not in _DTYPES or x.dim() != 2 or x.shape[0] != T or not x.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: x must be contiguous [T, H]")
@@ -390,7 +421,9 @@ def ep_layout_dispatch(h: EPHandle, topk_idx: torch.Tensor, x: torch.Tensor,
     if x.dtype == torch.float16 and f != EP_FMT_FP16:
         raise EPError(EP_ERR_INVALID_ARG, "ep_layout_dispatch: fp16 x takes the fp16 copy only; "
                       "for FP8 of fp16 rows call ep_layout then ep_dispatch")
-    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows)
+    _same_device(h, "ep_layout_dispatch", topk_idx, x)
+    recv_x, recv_scales = _recv_buffers(h, T, H, f, x.device, recv_x, recv_scales, capacity_rows,
+                                        "ep_layout_dispatch")
     with _on(h):
         _check(load_library().ep_layout_dispatch(
             h.handle, _ptr(topk_idx), T, _ptr(x), H, f, _ptr(recv_x), _ptr(recv_scales),
@@ -415,6 +448,7 @@ def ep_combine(h: EPHandle, y: torch.Tensor, topk_weights: torch.Tensor,
         out = torch.empty((h.T, H), dtype=y.dtype, device=y.device)
     if out.dtype != y.dtype or tuple(out.shape) != (h.T, H) or not out.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine: out must be contiguous [T, H], y's type")
+    _same_device(h, "ep_combine", y, topk_weights, out)
     lib = load_library()
     with _on(h):
         if y.dtype == torch.bfloat16:
@@ -441,8 +475,9 @@ def ep_dispatch_range(h: EPHandle, t_begin: int, x_rows: torch.Tensor, fmt: str,
             x_rows.dtype != torch.bfloat16:
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: x_rows type and format disagree")
     n, H = x_rows.shape
-    if recv_x.shape[1] != H or not recv_x.is_contiguous():
-        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_range: recv_x must be contiguous [*, H]")
+    _check_recv("ep_dispatch_range", H, f, recv_x, recv_scales)
+    _same_device(h, "ep_dispatch_range", x_rows, recv_x,
+                 recv_scales if not _is_copy(f) else None)
     with _on(h):
         _check(load_library().ep_dispatch_range(
             h.handle, t_begin, n, _ptr(x_rows), H, f, _ptr(recv_x),
@@ -457,12 +492,15 @@ def ep_combine_range(h: EPHandle, t_begin: int, y: torch.Tensor, topk_weights_ro
     (topk_weights_rows: f32 [n, k]; out_rows: bf16 [n, H], contiguous)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_combine_range")
+    if out_rows.dim() != 2 or y.dim() != 2:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_range: y and out_rows must be 2-D")
     n, H = out_rows.shape
     if (y.dtype != torch.bfloat16 or y.shape[1] != H or not y.is_contiguous()
             or out_rows.dtype != torch.bfloat16 or not out_rows.is_contiguous()
             or topk_weights_rows.dtype != torch.float32
             or tuple(topk_weights_rows.shape) != (n, h.k) or not topk_weights_rows.is_contiguous()):
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine_range: bad tensor")
+    _same_device(h, "ep_combine_range", y, topk_weights_rows, out_rows)
     with _on(h):
         _check(load_library().ep_combine_range(
             h.handle, t_begin, n, _ptr(y), y.shape[0], _ptr(topk_weights_rows), H, _ptr(out_rows),
@@ -491,9 +529,10 @@ def ep_dispatch_ranks(h: EPHandle, t_begin: int, x_rows: torch.Tensor, fmt: Opti
     n, H = x_rows.shape
     if len(recv_x) != h.R or (not _is_copy(f) and (recv_scales is None or len(recv_scales) != h.R)):
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: one buffer per rank")
-    for r in recv_x:
-        if r.shape[1] != H or not r.is_contiguous() or r.dtype != _recv_dtype(f):
-            raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks: recv_x[p] must be [*, H]")
+    _same_device(h, "ep_dispatch_ranks", x_rows)
+    _rank_list(h, "ep_dispatch_ranks", recv_x if _is_copy(f) else list(recv_x) + list(recv_scales))
+    for p, r in enumerate(recv_x):
+        _check_recv("ep_dispatch_ranks", H, f, r, None if _is_copy(f) else recv_scales[p])
     ptrs = _table([_ptr(r) for r in recv_x], ctypes.c_void_p)
     rows = _table([r.shape[0] for r in recv_x], ctypes.c_int64)
     sptrs = _table([_ptr(sc) for sc in recv_scales], ctypes.c_void_p) if not _is_copy(f) else None
@@ -510,12 +549,16 @@ def ep_combine_ranks(h: EPHandle, t_begin: int, y: list, topk_weights_rows: torc
     rank's buffer y[p] (bf16 or fp16, the type of out_rows)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_combine_ranks")
+    if out_rows.dim() != 2:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_ranks: out_rows must be 2-D")
+    _rank_list(h, "ep_combine_ranks", y)
     n, H = out_rows.shape
     if (out_rows.dtype not in _DTYPES or not out_rows.is_contiguous() or len(y) != h.R
             or topk_weights_rows.dtype != torch.float32
             or tuple(topk_weights_rows.shape) != (n, h.k) or not topk_weights_rows.is_contiguous()
             or any(t.dtype != out_rows.dtype or t.shape[1] != H or not t.is_contiguous() for t in y)):
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine_ranks: bad tensor")
+    _same_device(h, "ep_combine_ranks", topk_weights_rows, out_rows)
     ptrs = _table([_ptr(t) for t in y], ctypes.c_void_p)
     rows = _table([t.shape[0] for t in y], ctypes.c_int64)
     with _on(h):
@@ -531,6 +574,10 @@ def ep_dispatch_ranks_backward(h: EPHandle, t_begin: int, grad_recv: list,
     buffers grad_recv[p], rounded to grad_x_rows' type (bf16 or fp16)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_dispatch_ranks_backward")
+    if grad_x_rows.dim() != 2:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_ranks_backward: grad_x_rows must be 2-D")
+    _rank_list(h, "ep_dispatch_ranks_backward", grad_recv)
+    _same_device(h, "ep_dispatch_ranks_backward", grad_x_rows)
     n, H = grad_x_rows.shape
     if (grad_x_rows.dtype not in _DTYPES or not grad_x_rows.is_contiguous() or
             len(grad_recv) != h.R or any(t.dtype != grad_x_rows.dtype or t.shape[1] != H or
@@ -551,6 +598,10 @@ def ep_combine_ranks_backward(h: EPHandle, t_begin: int, grad_out_rows: torch.Te
     grad_weights f32 [n, k] (dot products of grad_out with the slots' y rows)."""
     if h.T is None:
         raise EPError(EP_ERR_STATE, "ep_combine_ranks_backward")
+    if grad_out_rows.dim() != 2:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_ranks_backward: grad_out_rows must be 2-D")
+    _rank_list(h, "ep_combine_ranks_backward", list(y) + list(grad_y))
+    _same_device(h, "ep_combine_ranks_backward", grad_out_rows, topk_weights_rows)
     n, H = grad_out_rows.shape
     dt = grad_out_rows.dtype
     if (dt not in _DTYPES or not grad_out_rows.is_contiguous() or len(y) != h.R
@@ -608,6 +659,7 @@ def ep_dispatch_backward(h: EPHandle, grad_recv: torch.Tensor,
     if grad_x.dtype != grad_recv.dtype or tuple(grad_x.shape) != (h.T, H) or \
             not grad_x.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_backward: grad_x must be [T, H]")
+    _same_device(h, "ep_dispatch_backward", grad_recv, grad_x)
     with _on(h):
         _check(load_library().ep_dispatch_backward_ex(
             h.handle, _ptr(grad_recv), grad_recv.shape[0], H, _DTYPES[grad_recv.dtype],
@@ -629,11 +681,14 @@ def ep_combine_backward(h: EPHandle, grad_out: torch.Tensor, y: torch.Tensor,
             or not topk_weights.is_contiguous()):
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: topk_weights must be f32 [T, k]")
     H = y.shape[1]
+    if tuple(grad_out.shape) != (h.T, H):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: grad_out must be [T, H]")
     if grad_y is None:
         grad_y = torch.empty_like(y)
     if grad_y.dtype != y.dtype or grad_y.dim() != 2 or grad_y.shape[1] != H or \
             not grad_y.is_contiguous():
         raise EPError(EP_ERR_INVALID_ARG, "ep_combine_backward: grad_y must be [*, H], y's type")
+    _same_device(h, "ep_combine_backward", grad_out, y, topk_weights, grad_y)
     grad_w = torch.empty((h.T, h.k), dtype=torch.float32, device=y.device)
     with _on(h):
         _check(load_library().ep_combine_backward_ex(
@@ -656,6 +711,10 @@ def ep_dispatch_weights(h: EPHandle, topk_weights: torch.Tensor,
         cap = capacity_rows if capacity_rows is not None else \
             ep_recv_rows_upper_bound(h.T, h.k, h.E, h.block_m)
         recv_weights = torch.zeros(cap, dtype=torch.float32, device=topk_weights.device)
+    if (recv_weights.dtype != torch.float32 or recv_weights.dim() != 1
+            or not recv_weights.is_contiguous()):
+        raise EPError(EP_ERR_INVALID_ARG, "ep_dispatch_weights: recv_weights must be f32 [cap]")
+    _same_device(h, "ep_dispatch_weights", topk_weights, recv_weights)
     with _on(h):
         _check(load_library().ep_dispatch_weights(h.handle, _ptr(topk_weights), _ptr(recv_weights),
                                                   recv_weights.shape[0], _stream(h.device)),
@@ -669,6 +728,7 @@ def ep_zero_pad_rows(h: EPHandle, rows: torch.Tensor) -> torch.Tensor:
         raise EPError(EP_ERR_STATE, "ep_zero_pad_rows")
     if not rows.is_contiguous() or rows.dim() < 1:
         raise EPError(EP_ERR_INVALID_ARG, "ep_zero_pad_rows: rows must be contiguous")
+    _same_device(h, "ep_zero_pad_rows", rows)
     row_bytes = rows[0].numel() * rows.element_size() if rows.shape[0] else 1
     with _on(h):
         _check(load_library().ep_zero_pad_rows(h.handle, _ptr(rows), row_bytes, rows.shape[0],

@@ -49,6 +49,15 @@
  * The library never allocates device memory; the handle itself is a small
  * host allocation made by ep_handle_create.
  *
+ * Buffer sizes.  The library sees a buffer's pointer and the row count
+ * (capacity) passed with it, never the allocation: every write is bounded by
+ * the capacities given, so each buffer must hold at least the rows and the
+ * row width its documented shape implies for that capacity (an FP8 row is H
+ * bytes, a BF16/FP16 row 2H; row-major scales [capacity][H/128] fp32; MN-major
+ * [H/128][capacity]).  A smaller buffer, or a host pointer where a device one
+ * is asked for, is outside this contract and the GPU faults.  The Python
+ * binding checks type, shape and device of every tensor before the call.
+ *
  * Errors.  Argument problems that the host can see are returned at once and
  * nothing is enqueued.  Problems only the GPU can see (an index outside
  * [-1, E), a receive row beyond the capacity given) set bits in a sticky
