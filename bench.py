@@ -583,9 +583,10 @@ def time_backward(dev, flush, seed, steps):
 
 # ----------------------------------------------------------------- CPU arm
 
-def cpu_oracle_step(w, tokens, y_full=None):
-    """One oracle step (layout + dispatch + combine) on the first `tokens`
-    tokens; y for combine is made by the oracle's stand-in expert (untimed)."""
+def oracle_sample(w, tokens):
+    """Inputs of an oracle step on the first `tokens` tokens, and the expert
+    output y that its combine reads (made by the oracle's stand-in expert;
+    not part of any timed step)."""
     import oracle
 
     idx = np.ascontiguousarray(w.topk_idx[:tokens])
@@ -598,14 +599,30 @@ def cpu_oracle_step(w, tokens, y_full=None):
     else:
         q0, s0 = oracle.dispatch_fp8(xb, lay0.dst_row, lay0.total_rows)
         y = oracle.expert_scale_fp8(q0, s0, lay0, w.expert_c)
+    return {"tokens": tokens, "idx": idx, "xb": xb, "wt": wt, "y": y}
+
+
+def oracle_timed_step(w, smp):
+    """One oracle step (layout + dispatch + combine) on a prepared sample; seconds."""
+    import oracle
+
     t0 = time.perf_counter()
-    lay = oracle.layout(idx, w.E, w.R, w.block_m)
+    lay = oracle.layout(smp["idx"], w.E, w.R, w.block_m)
     if w.fmt == "bf16":
-        oracle.dispatch_bf16(xb, lay.dst_row, lay.total_rows)
+        oracle.dispatch_bf16(smp["xb"], lay.dst_row, lay.total_rows)
     else:
-        oracle.dispatch_fp8(xb, lay.dst_row, lay.total_rows)
-    oracle.combine(y, wt, lay.dst_row)
+        oracle.dispatch_fp8(smp["xb"], lay.dst_row, lay.total_rows)
+    oracle.combine(smp["y"], smp["wt"], lay.dst_row)
     return time.perf_counter() - t0
+
+
+def oracle_seconds_per_token(w, probe=512):
+    """Per-token time of one oracle step, from the second of two steps on the
+    first `probe` tokens: the first also pays for first touches of freshly
+    mapped output pages and would overstate the cost of a larger sample."""
+    smp = oracle_sample(w, min(w.T, probe))
+    oracle_timed_step(w, smp)
+    return oracle_timed_step(w, smp) / smp["tokens"]
 
 
 def cpu_baseline(w, budget_s=15.0):
@@ -613,19 +630,18 @@ def cpu_baseline(w, budget_s=15.0):
     import oracle
 
     oracle.build()
-    probe = min(w.T, 64)
-    t = cpu_oracle_step(w, probe)
-    per_tok = t / probe
-    tokens = int(max(probe, min(w.T, budget_s / 2.0 / max(per_tok, 1e-9))))
-    reps = max(1, int(budget_s / max(per_tok * tokens, 1e-9)))
-    reps = min(reps, 5)
-    times = [cpu_oracle_step(w, tokens) for _ in range(reps)]
+    per_tok = oracle_seconds_per_token(w)
+    tokens = int(min(w.T, max(min(w.T, 512), budget_s / 2.0 / max(per_tok, 1e-9))))
+    smp = oracle_sample(w, tokens)
+    warm = oracle_timed_step(w, smp)                # warm-up; its time bounds the repetitions
+    reps = min(5, max(1, int(budget_s / max(warm, 1e-9))))
+    times = [oracle_timed_step(w, smp) for _ in range(reps)]
     d, c = algo_bytes(tokens, w.H, w.k, w.fmt)
     gbs = (d + c) / statistics.mean(times) / 1e9
     return {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "first %d of %d tokens of the same workload, %d repetitions, "
-                      "single-threaded C oracle (gcc -O2), layout+dispatch+combine" % (
-                          tokens, w.T, reps),
+            "sample": "first %d of %d tokens of the same workload, 1 warm-up + %d timed "
+                      "repetitions, single-threaded C oracle (gcc -O2), "
+                      "layout+dispatch+combine" % (tokens, w.T, reps),
             "host": host_cpu()}
 
 
@@ -653,13 +669,21 @@ def run_reference(args, rank, world):
 
     oracle.build()
     w = make_workload(MAIN_WORKLOAD, 0)
-    probe = 64
-    per_tok = cpu_oracle_step(w, probe) / probe
-    budget = 90.0
-    tokens = int(max(8, min(w.T, budget / max(1, args.steps + args.warmup) / per_tok)))
+    per_tok = oracle_seconds_per_token(w)
+    budget = 120.0                                  # seconds of timed and warm-up steps
+    per_step = budget / max(1, args.steps + args.warmup)
+    floor = min(w.T, 256)
+    tokens = int(max(floor, min(w.T, per_step / per_tok)))
+    smp = oracle_sample(w, tokens)
+    for _ in range(2):                              # the probe can misjudge a larger sample
+        t = oracle_timed_step(w, smp)
+        if t <= 1.5 * per_step or tokens == floor:
+            break
+        tokens = int(max(floor, tokens * per_step / t))
+        smp = oracle_sample(w, tokens)
     for _ in range(args.warmup):
-        cpu_oracle_step(w, tokens)
-    ts = [cpu_oracle_step(w, tokens) for _ in range(args.steps)]
+        oracle_timed_step(w, smp)
+    ts = [oracle_timed_step(w, smp) for _ in range(args.steps)]
     d, c = algo_bytes(tokens, w.H, w.k, w.fmt)
     ms = statistics.mean(ts) * 1e3
     val = (d + c) / (ms / 1e3) / 1e9

@@ -30,7 +30,7 @@ def test_package_sources_do_not_use_the_oracle():
 
 def test_bench_imports_the_oracle_only_in_its_cpu_legs():
     tree = ast.parse(open(os.path.join(ROOT, "bench.py"), encoding="utf-8").read())
-    allowed = {"cpu_oracle_step", "cpu_baseline", "run_reference"}
+    allowed = {"oracle_sample", "oracle_timed_step", "cpu_baseline", "run_reference"}
     for fn in ast.walk(tree):
         if not isinstance(fn, ast.FunctionDef):
             continue
