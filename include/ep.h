@@ -99,8 +99,9 @@ typedef enum {
 } ep_status_t;
 
 /* Element type of 16-bit hidden rows (x, y, out).  The yololab page lists
- * BF16, FP16 and FP8 as dispatch data types ("DeepEP是什麼？…", section
- * FP8與低精度通訊). */
+ * BF16, FP16 and FP8 as the precisions a deployment should test
+ * ("DeepEP是什麼？…", section Benchmark矩陣); its FP8與低精度通訊 section
+ * covers the FP8 form. */
 typedef enum {
     EP_DTYPE_BF16 = 0,            /* bfloat16 */
     EP_DTYPE_FP16 = 1             /* IEEE-754 binary16 */
@@ -146,21 +147,30 @@ typedef enum {
  * (host; pure arithmetic).  Returns 0 if the arguments are invalid:
  * max_tokens >= 0, 1 <= num_topk <= EP_MAX_TOPK,
  * 1 <= num_experts <= EP_MAX_EXPERTS, 1 <= num_ranks, num_experts % num_ranks
- * == 0, 1 <= block_m <= EP_MAX_BLOCK_M, and every row count below 2^31. */
+ * == 0, 1 <= block_m <= EP_MAX_BLOCK_M, and every row count below 2^31.
+ * The pages size the buffer from max tokens, top-k, hidden size and EP degree
+ * ("DeepEP是什麼？…", section ElasticBuffer); here the hidden rows live in the
+ * caller's buffers, so the workspace holds only the layout and is sized from
+ * the same quantities less the hidden size. */
 size_t ep_workspace_bytes(int max_tokens, int num_topk, int num_experts, int num_ranks,
                           int block_m);
 
 /* Upper bound on the padded receive rows P for T tokens (host, no sync):
  * T*k + min(E, T*k)*(block_m - 1), rounded down to a multiple of block_m.
  * Sizing recv buffers with it lets a whole step run without reading P back,
- * e.g. inside a CUDA graph.  Returns -1 for invalid arguments. */
+ * e.g. inside a CUDA graph.  Returns -1 for invalid arguments.  This is the
+ * capacity headroom for uneven routing that the same ElasticBuffer section
+ * asks for, taken at its worst case (every used expert one row short of a
+ * full block). */
 int64_t ep_recv_rows_upper_bound(int T, int num_topk, int num_experts, int block_m);
 
 /* Create a handle over a caller-owned device workspace (host; makes no CUDA
  * call).  workspace: device pointer, 256-byte aligned, at least
  * ep_workspace_bytes(...) bytes, owned by the caller and kept alive, and not
  * used for anything else, until ep_handle_destroy.  On success *out receives
- * the handle; on failure *out is set to NULL. */
+ * the handle; on failure *out is set to NULL.  The handle plays the part of
+ * the pages' EPHandle, which carries dispatch state into combine (DeepEP v2
+ * release notes, section Có gì mới trong v2). */
 ep_status_t ep_handle_create(void* workspace, size_t workspace_bytes, int max_tokens,
                              int num_topk, int num_experts, int num_ranks, int block_m,
                              ep_handle_t* out);
@@ -174,7 +184,15 @@ void ep_handle_destroy(ep_handle_t h);
  * [0, E) or -1 for an unused slot.  0 <= T <= max_tokens.  Fills every view
  * of ep_view_t.  The layout stays valid, and is what ep_dispatch and
  * ep_combine use, until the next ep_layout on this handle.  An index outside
- * [-1, E) sets EP_ERR_BAD_INDEX in the sticky error word and is treated as -1. */
+ * [-1, E) sets EP_ERR_BAD_INDEX in the sticky error word and is treated as -1.
+ * Source: the pages' ElasticBuffer manages a "dispatch layout" ("DeepEP是什麼？
+ * …", section ElasticBuffer); the same page's stage table (section
+ * MoE為什麼需要All-to-all) has dispatch turn tokens and top-k indices into
+ * hidden states arranged by expert, with sorting and imbalance as its cost,
+ * and its Load Imbalance section lists per-expert token counts and per-rank
+ * traffic as the figures to watch.  The exact layout rules (expert-major,
+ * block_m padding, (token, slot) order) are the reading stated at the top of
+ * this header. */
 ep_status_t ep_layout(ep_handle_t h, const int64_t* topk_idx, int T, void* stream);
 
 /* Layout followed by dispatch, the low-latency path for decode-sized batches
@@ -204,7 +222,9 @@ const void* ep_handle_view(ep_handle_t h, ep_view_t what, int64_t* count);
 /* Copy the counts of the last layout to host memory and wait for the stream
  * (SYNCHRONISING).  Any output pointer may be NULL.  num_tokens_per_expert:
  * int32 [E]; num_tokens_per_rank: int32 [R]; num_rows_per_rank: int32 [R];
- * total_recv_rows: int32 [1] (P). */
+ * total_recv_rows: int32 [1] (P).  These are the per-expert token counts and
+ * per-rank volumes that "DeepEP是什麼？…", section Load Imbalance, names as the
+ * signs of a hot expert or a straggling rank. */
 ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
                                   int32_t* num_tokens_per_rank, int32_t* num_rows_per_rank,
                                   int32_t* total_recv_rows, void* stream);
@@ -226,7 +246,11 @@ ep_status_t ep_handle_read_counts(ep_handle_t h, int32_t* num_tokens_per_expert,
  *   MN-major, fp32 [H/128][recv_capacity_rows] (scale of row r, block b at
  *   b * recv_capacity_rows + r), recv_capacity_rows % 4 == 0.
  * Only the rows listed in dst_row are written; pad rows keep their contents.
- * A row >= recv_capacity_rows is skipped and sets EP_ERR_CAPACITY. */
+ * A row >= recv_capacity_rows is skipped and sets EP_ERR_CAPACITY.
+ * Source of the operation: the Dispatch row of the stage table in
+ * "DeepEP是什麼？…", section MoE為什麼需要All-to-all (tokens and top-k indices
+ * in, hidden states arranged by expert out); its bytes, T k H sizeof(dtype),
+ * are those of "DeepEP 编址服务深度对抗分析", section 五.2. */
 ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void* recv_x,
                         float* recv_scales, int64_t recv_capacity_rows, void* stream);
 
@@ -237,7 +261,8 @@ ep_status_t ep_dispatch(ep_handle_t h, const void* x, int H, ep_fmt_t fmt, void*
  * the same amax, scale and rounding as above.  A copy format must match
  * x_dtype (EP_FMT_BF16 with bf16, EP_FMT_FP16 with fp16), else
  * EP_ERR_INVALID_ARG.  ep_dispatch itself takes fp16 rows only with
- * EP_FMT_FP16. */
+ * EP_FMT_FP16.  FP16 is one of the precisions (BF16, FP16, FP8) the yololab
+ * page's Benchmark矩陣 section asks a deployment to cover. */
 ep_status_t ep_dispatch_ex(ep_handle_t h, const void* x, ep_dtype_t x_dtype, int H, ep_fmt_t fmt,
                            void* recv_x, float* recv_scales, int64_t recv_capacity_rows,
                            void* stream);
@@ -249,14 +274,20 @@ ep_status_t ep_dispatch_ex(ep_handle_t h, const void* x, ep_dtype_t x_dtype, int
  * out[t][h] = bf16_rn(acc), acc = 0 then, for j = 0..k-1 over the used
  * slots, acc = fma(w[t][j], y[dst_row[t][j]][h], acc) in fp32.  Weights are
  * used as given (no renormalisation); unused slots (-1) are skipped.
- * A row >= y_rows is skipped and sets EP_ERR_CAPACITY. */
+ * A row >= y_rows is skipped and sets EP_ERR_CAPACITY.
+ * Source: the Combine row of the stage table in "DeepEP是什麼？…", section
+ * MoE為什麼需要All-to-all (expert outputs and routing weights in, results in
+ * the original token order out, by a reverse exchange and a reduction).  The
+ * pages leave the reduction's arithmetic open; the fp32 chain in slot order
+ * above is the reading taken. */
 ep_status_t ep_combine(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
                        int H, void* out, void* stream);
 
 /* ep_combine with the type of y and out named: EP_DTYPE_BF16 is ep_combine;
  * EP_DTYPE_FP16 reads binary16 expert outputs (widened exactly), accumulates
  * in fp32 in the same order and rounds the result to nearest even binary16
- * (sums beyond the binary16 range become infinities). */
+ * (sums beyond the binary16 range become infinities).  Precisions: the yololab
+ * page's Benchmark矩陣 section (BF16, FP16, FP8). */
 ep_status_t ep_combine_ex(ep_handle_t h, const void* y, int64_t y_rows, const float* topk_weights,
                           int H, ep_dtype_t dtype, void* out, void* stream);
 
@@ -269,7 +300,10 @@ ep_status_t ep_combine_ex(ep_handle_t h, const void* y, int64_t y_rows, const fl
  * the whole receive-layout buffers.  The ranges of one layout may run in any
  * order and on different streams: they write disjoint rows.  This lets a
  * caller overlap the transfer of token chunks (host copies, or an upstream
- * producer) with dispatch and combine of the chunks already present. */
+ * producer) with dispatch and combine of the chunks already present, the
+ * pipelining of communication with computation that "DeepEP：让大模型「专家们」
+ * 高效协作的通信高速公路" (section 技术架构：从NVSHMEM到NCCL Gin的演进) gives as
+ * the aim of the V2 buffer interface. */
 ep_status_t ep_dispatch_range(ep_handle_t h, int t_begin, int t_count, const void* x_rows, int H,
                               ep_fmt_t fmt, void* recv_x, float* recv_scales,
                               int64_t recv_capacity_rows, void* stream);

@@ -29,8 +29,8 @@
  *     and q = +0.
  *   - Combine: fp32 accumulation in slot order j = 0..k-1 with one fused
  *     multiply-add per term, then round-to-nearest-even to bf16.
- *   - FP16 rows: the yololab page lists BF16, FP16 and FP8 as data types
- *     (section FP8與低精度通訊); binary16 values are widened exactly and
+ *   - FP16 rows: the yololab page lists BF16, FP16 and FP8 as the precisions
+ *     to test (section Benchmark矩陣); binary16 values are widened exactly and
  *     results rounded to nearest even binary16 (formats written below from
  *     IEEE 754).
  *   - Backward (training use: the pomoai page, section 核心使用场景): the
