@@ -1,6 +1,11 @@
 // ep_api.cu -- the C ABI declared in include/ep.h: argument checks, the
 // workspace carve, the handle, and the kernel launches.  No device memory is
-// allocated here; the handle is one small host allocation.
+// allocated here; the handle is one small host allocation.  The split between
+// a caller-sized workspace holding the dispatch layout and a handle carrying it
+// from dispatch to combine follows the pages' ElasticBuffer ("DeepEP是什麼？
+// …", section ElasticBuffer: sized from max tokens, top-k, hidden size and EP
+// degree) and EPHandle (DeepEP v2 release notes, section Có gì mới trong v2);
+// each operation's own source is stated with its declaration in ep.h.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>

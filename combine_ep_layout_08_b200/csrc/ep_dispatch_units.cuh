@@ -1,5 +1,8 @@
 // ep_dispatch_units.cuh -- the per-unit bodies of the 256-bit dispatch
 // kernels, shared by ep_dispatch.cu and the fused layout + dispatch kernel.
+// The operation is dispatch as the stage table of "DeepEP是什麼？…" (section
+// MoE為什麼需要All-to-all) defines it, with the FP8 form read from that page's
+// FP8與低精度通訊 section (one fp32 scale per 128 channels, s = amax / 448).
 // A unit is one warp's share of one token row: BF16 512 channels (32 lanes x
 // one 32-byte vector), FP8 512 kU channels (32 lanes x kU 32-byte vectors =
 // 4 kU blocks of 128; kU = 2 in the dispatch kernels, 1 in the fused

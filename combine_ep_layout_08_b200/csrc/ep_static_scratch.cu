@@ -1,5 +1,7 @@
 // ep_static_scratch.cu -- ep_layout_static_scratch: the dispatch layout for
-// callers that cannot allocate device memory.
+// callers that cannot allocate device memory.  The pages ask for a stated
+// policy when a buffer cannot be allocated ("DeepEP是什麼？…", section
+// ElasticBuffer); this entry point takes allocation out of the call.
 //
 // Some callers have no way to hand the library a workspace: code that runs
 // while a CUDA graph is being captured (allocation is not a capturable
