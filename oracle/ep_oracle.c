@@ -255,7 +255,8 @@ static int64_t pad_up(int64_t c, int64_t block_m)
 
 /* Upper bound on the padded receive rows for T tokens: every non-empty
  * expert adds at most block_m - 1 pad rows, and at most min(E, T*k)
- * experts are non-empty. */
+ * experts are non-empty.  (Capacity headroom for uneven routing, which
+ * "DeepEP是什麼？…", section ElasticBuffer, asks a buffer to keep.) */
 int64_t oracle_recv_rows_bound(int64_t T, int k, int E, int block_m)
 {
     int64_t n = T * (int64_t)k;
@@ -280,6 +281,12 @@ int64_t oracle_recv_rows_bound(int64_t T, int k, int E, int block_m)
  *   total_rows[1]              P = expert_off[E]
  * Returns OR_ERR_BAD_INDEX for an index outside [-1, E) (outputs then
  * undefined), OR_ERR_CAPACITY if recv_cap < P.
+ * Source: the "dispatch layout" the pages' ElasticBuffer manages
+ * ("DeepEP是什麼？…", section ElasticBuffer), the per-expert token counts and
+ * per-rank traffic of its Load Imbalance section, and hidden states arranged
+ * by expert as dispatch's output (stage table, section MoE為什麼需要All-to-all).
+ * Expert-major order, block_m padding and (token, slot) order inside a block
+ * are the reading taken where the pages leave the "GEMM layout" undefined.
  */
 int oracle_layout(const int64_t* topk_idx, int64_t T, int k, int E, int R, int block_m,
                   int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
@@ -375,7 +382,9 @@ int oracle_layout(const int64_t* topk_idx, int64_t T, int k, int E, int R, int b
 /* Dispatch.                                                            */
 /* ------------------------------------------------------------------ */
 
-/* BF16 dispatch: every used slot (t, j) receives a byte copy of x[t]. */
+/* BF16 dispatch: every used slot (t, j) receives a byte copy of x[t]
+ * (dispatch as the stage table of "DeepEP是什麼？…", section
+ * MoE為什麼需要All-to-all, defines it: tokens in, rows arranged by expert out). */
 int oracle_dispatch_bf16(const uint16_t* x, int64_t T, int k, int64_t H,
                          const int32_t* dst_row, uint16_t* recv_x, int64_t recv_cap)
 {
@@ -395,7 +404,9 @@ int oracle_dispatch_bf16(const uint16_t* x, int64_t T, int k, int64_t H,
  * amax = max |x|, s = amax / 448 (fp32 division), q = e4m3(x / s) (fp32
  * division, then round-to-nearest-even with saturation); amax == 0 gives
  * s = 0 and q = +0 for the whole block.  x holds bfloat16 (dtype 0) or
- * binary16 (dtype 1) values, widened exactly to binary32. */
+ * binary16 (dtype 1) values, widened exactly to binary32.  "DeepEP是什麼？…",
+ * section FP8與低精度通訊, asks to confirm the scale granularity and format
+ * without fixing them; this is the reading taken. */
 void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, int dtype, uint8_t* q,
                                float* scales)
 {
@@ -422,7 +433,9 @@ void oracle_quantize_token_fp8(const uint16_t* x, int64_t H, int dtype, uint8_t*
 }
 
 /* FP8 dispatch: every used slot (t, j) receives the e4m3 row of x[t] and
- * its H/128 fp32 scales (row-major [rows][H/128]). */
+ * its H/128 fp32 scales (row-major [rows][H/128]).  FP8 dispatch with BF16
+ * combine is the pages' configuration (DeepEP v2 release notes, section Số
+ * liệu kỹ thuật). */
 int oracle_dispatch_fp8(const uint16_t* x, int64_t T, int k, int64_t H, int dtype,
                         const int32_t* dst_row, uint8_t* recv_q, float* recv_scales,
                         int64_t recv_cap)
@@ -504,7 +517,10 @@ void oracle_expert_scale_fp8(const uint8_t* recv_q, const float* recv_scales,
  * bfloat16 (dtype 0) or binary16 (dtype 1), rn16 the round-to-nearest-even
  * into that type.  The slot loop is
  * the outer loop over a row of accumulators; each element still sees its
- * terms in slot order. */
+ * terms in slot order.  Source: the Combine row of the stage table in
+ * "DeepEP是什麼？…", section MoE為什麼需要All-to-all (expert outputs and routing
+ * weights in, the original token order out, by a reduction); the fp32 fma
+ * chain in slot order is the reading taken of the reduction's arithmetic. */
 int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* dst_row,
                    int64_t T, int k, int64_t H, int dtype, uint16_t* out)
 {
