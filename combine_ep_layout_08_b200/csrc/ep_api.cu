@@ -89,6 +89,7 @@ bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c)
     c->rows_per_rank = take(sizeof(int32_t) * (size_t)R);
     c->total_rows = take(sizeof(int32_t));
     c->err = take(3 * sizeof(int32_t));
+    c->tile_acc = take(sizeof(int32_t) * tile_acc_words(E, R));
     c->is_token_in_rank = take((size_t)max_tokens * R);
     c->dst_row = take(sizeof(int32_t) * (size_t)max_tokens * k);
     c->recv_src = take(sizeof(int32_t) * (size_t)rows);
@@ -229,6 +230,8 @@ ep_status_t clear_error_words_once(Handle* h, cudaStream_t s)
     if (h->err_cleared)
         return EP_OK;
     cudaError_t rc = cudaMemsetAsync(h->err, 0, 3 * sizeof(int32_t), s);
+    if (rc == cudaSuccess)
+        rc = cudaMemsetAsync(h->tile_acc, 0, sizeof(int32_t) * ep::tile_acc_words(h->E, h->R), s);
     if (rc != cudaSuccess)
         return ep::cuda_fail(rc, "clearing the error words");
     h->err_cleared = 1;
@@ -317,6 +320,7 @@ ep_status_t ep_handle_create(void* workspace, size_t workspace_bytes, int max_to
     h->rows_per_rank = reinterpret_cast<int32_t*>(base + c.rows_per_rank);
     h->total_rows = reinterpret_cast<int32_t*>(base + c.total_rows);
     h->err = reinterpret_cast<int32_t*>(base + c.err);
+    h->tile_acc = reinterpret_cast<int32_t*>(base + c.tile_acc);
     h->is_token_in_rank = reinterpret_cast<uint8_t*>(base + c.is_token_in_rank);
     h->dst_row = reinterpret_cast<int32_t*>(base + c.dst_row);
     h->recv_src = reinterpret_cast<int32_t*>(base + c.recv_src);
@@ -762,9 +766,11 @@ ep_status_t ep_handle_check(ep_handle_t hh, void* stream)
     if (rc == cudaSuccess)
         rc = cudaStreamSynchronize(s);
     // Clear the error word; after a barrier time-out also reset the barrier
-    // (its count is left mid-way).
+    // (its count is left mid-way) and the single-launch layout's sums.
     if (rc == cudaSuccess)
         rc = cudaMemsetAsync(h->err, 0, ((word & ep::kErrTimeout) ? 3 : 1) * sizeof(int32_t), s);
+    if (rc == cudaSuccess && (word & ep::kErrTimeout) && h->tile_acc)
+        rc = cudaMemsetAsync(h->tile_acc, 0, sizeof(int32_t) * ep::tile_acc_words(h->E, h->R), s);
     if (rc == cudaSuccess)
         rc = cudaStreamSynchronize(s);
     if (rc != cudaSuccess)

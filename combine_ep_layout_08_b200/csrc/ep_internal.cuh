@@ -25,6 +25,13 @@ constexpr int kErrTimeout = 8;       // a grid barrier gave up waiting
 // per chunk: the (token, slot) entries of a chunk are contiguous in topk_idx.
 constexpr int kChunkTokens = 32;
 
+// The single-launch layout groups its tiles; at most kTileMaxGroups groups of
+// at most kTileMaxGroups tiles.
+constexpr int kTileMaxGroups = 32;
+// Words of the single-launch layout's sums (an epoch word and two buffers of
+// group rows and per-rank sums); zero when the handle is first used.
+size_t tile_acc_words(int E, int R);
+
 struct Handle {
     uint32_t magic;
     int max_tokens, k, E, R, block_m;
@@ -40,6 +47,7 @@ struct Handle {
     int32_t* rows_per_rank;  // [R]
     int32_t* total_rows;     // [1]
     int32_t* err;            // [3] sticky error bits, then the grid barrier's count and generation
+    int32_t* tile_acc;       // [tile_acc_words] the single-launch layout's sums (may be null)
     uint8_t* is_token_in_rank;  // [max_tokens][R]
     int32_t* dst_row;        // [max_tokens][k]
     int32_t* recv_src;       // [max_rows]
@@ -53,7 +61,7 @@ struct Handle {
 // total size, or 0 if the sizes overflow.
 struct Carve {
     size_t chunk_counts, chunk_rank, cnt, expert_off, rank_off, tokens_per_rank,
-        rows_per_rank, total_rows, err, is_token_in_rank, dst_row, recv_src, total;
+        rows_per_rank, total_rows, err, tile_acc, is_token_in_rank, dst_row, recv_src, total;
 };
 
 int64_t recv_rows_bound(int64_t T, int64_t k, int64_t E, int64_t block_m);

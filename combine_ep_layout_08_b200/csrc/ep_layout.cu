@@ -23,9 +23,10 @@
 //              each group of 32 entries by lane (a ballot per key bit), to give
 //              dst_row and recv_src; pad rows of recv_src are set to -1.
 // Large batches, one launch (the default): layout_tile_kernel runs the three
-// phases in one cooperative launch over 64-token tiles, its CTAs separated by
-// two grid barriers; the three kernels remain for shapes whose tile counts do
-// not fit in shared memory and for the static-scratch entry point.
+// phases in one cooperative launch, one tile of tokens per CTA, its CTAs
+// separated by a single grid barrier (every CTA then sums all tiles' counts
+// itself); the three kernels remain for shapes whose tiles do not fit in
+// shared memory and for the static-scratch entry point.
 // Small batches (T k <= 4096, E <= 1024, shared memory permitting) run with
 // one entry per thread in CTAs of 1024 threads that each compute the whole
 // layout (layout_small_kernel).
@@ -36,6 +37,7 @@
 // its predecessor drains, and waits (griddepcontrol.wait) before it touches
 // memory.
 #include <algorithm>
+#include <atomic>
 
 #include "ep_dispatch_units.cuh"
 #include "ep_internal.cuh"
@@ -128,8 +130,9 @@ __device__ void scan_padded(const int32_t* cnt, int E, int block_m, int32_t* off
 // (erank[t * k + j], -1 for unused); byte p = t * R + r goes to lane p % 32,
 // so consecutive lanes write consecutive bytes.  Tokens-per-rank counts are
 // added to rhist.  With R <= 32 each token's ranks are first folded into a
-// bitmask held by lane t, the counts come from ballots, and each byte is one
-// shuffle; larger R tests the k entries per byte.
+// bitmask held by lane t, lane r counts the masks holding rank r (one shuffle
+// per token), and each byte is one shuffle; larger R tests the k entries per
+// byte.
 __device__ __forceinline__ void chunk_rank_bytes(const int32_t* erank, int ntok, int k, int R,
                                                  int64_t t0, uint8_t* is_token_in_rank,
                                                  int32_t* rhist)
@@ -146,11 +149,11 @@ __device__ __forceinline__ void chunk_rank_bytes(const int32_t* erank, int ntok,
                 if (q >= 0)
                     mask |= 1u << q;
             }
-        for (int q = 0; q < R; ++q) {
-            const int c = __popc(__ballot_sync(kFull, (mask >> q) & 1u));
-            if (lane == 0 && c)
-                atomicAdd(&rhist[q], c);
-        }
+        // lane q counts the tokens whose mask holds rank q
+        int c = 0;
+        for (int u = 0; u < ntok; ++u) c += (int)((__shfl_sync(kFull, mask, u) >> lane) & 1u);
+        if (lane < R && c)
+            atomicAdd(&rhist[lane], c);
         for (int p0 = 0; p0 < total; p0 += 32) {
             const uint32_t m = __shfl_sync(kFull, mask, t & 31);
             if (p0 + lane < total)
@@ -854,14 +857,15 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
 // Grid barrier over the CTAs of a cooperative launch (all co-resident).
 // bar[0] is an arrival counter that only grows (32-bit wrap-around, compared
 // by signed difference); bar[1] is its value when the current launch began.
-// Each CTA reads the base at its start; barrier b of the launch waits until
-// the counter reaches base + b G; the last arrival of the last barrier
-// stores the next launch's base (every CTA read the old one before
-// arriving).  Waiters watch the counter itself: the last arrival's add is the
-// release, one L2 round trip earlier than a separate release flag.  Graph
-// replays need no host state, and G may differ between launches.  The poll
-// is bounded: past kSpinLimit polls the CTA sets kErrTimeout and the caller
-// abandons the launch (ep_handle_check then resets both words).
+// Each CTA reads the base at its start; the barrier waits until the counter
+// reaches base + G; the last arrival stores the next launch's base (every
+// CTA read the old one before arriving).  Waiters watch the counter itself:
+// the last arrival's add is the release, one L2 round trip earlier than a
+// separate release flag.  Graph replays need no host state, and G may
+// differ between launches.  The same last arrival advances an epoch word
+// that every CTA read at its start.  The poll is bounded: past kSpinLimit
+// polls the CTA sets kErrTimeout and the caller abandons the launch
+// (ep_handle_check then resets the words).
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls of one L2 read each
 
 __device__ __forceinline__ int32_t ld_acquire(const int32_t* p)
@@ -886,24 +890,33 @@ __device__ __forceinline__ int32_t signed_gap(int32_t a, int32_t b)
     return (int32_t)((uint32_t)a - (uint32_t)b);
 }
 
-__device__ bool grid_barrier(int32_t* bar, int32_t target, bool last_of_launch, int32_t* err)
+// The barrier comes in two halves, so that a CTA can work between its
+// arrival and its wait.  barrier_arrive: one thread, after a block barrier,
+// so that its release covers the CTA's writes; the last arrival stores the
+// next launch's base and advances the epoch word.  barrier_wait: every
+// thread; the same thread polls (bounded), the others wait at a block
+// barrier.
+__device__ __forceinline__ void barrier_arrive(int32_t* bar, int32_t target, int32_t* epoch_word,
+                                               int32_t next_epoch)
+{
+    const int32_t old = atom_add_acq_rel(bar, 1);
+    if (signed_gap(old, target) == -1) {
+        asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(bar + 1), "r"(target) : "memory");
+        asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(epoch_word), "r"(next_epoch)
+                     : "memory");
+    }
+}
+
+__device__ bool barrier_wait(int32_t* bar, int32_t target, int32_t* err, bool poller)
 {
     __shared__ int ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    if (poller) {
         int good = 1;
-        const int32_t old = atom_add_acq_rel(bar, 1);
-        if (signed_gap(old, target) == -1) {
-            if (last_of_launch)
-                asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(bar + 1), "r"(target)
-                             : "memory");
-        } else {
-            uint32_t polls = 0;
-            while (signed_gap(ld_acquire(bar), target) < 0) {
-                if (++polls > kSpinLimit) {
-                    good = 0;
-                    break;
-                }
+        uint32_t polls = 0;
+        while (signed_gap(ld_acquire(bar), target) < 0) {
+            if (++polls > kSpinLimit) {
+                good = 0;
+                break;
             }
         }
         if (!good)
@@ -914,231 +927,326 @@ __device__ bool grid_barrier(int32_t* bar, int32_t target, bool last_of_launch, 
     return ok != 0;
 }
 
-// One warp scans column col of an [nrows][ncol] count matrix: exclusive
-// prefix over rows written in place (if write_prefix); the column total is
-// returned to every lane.  Each batch covers 32 x kBatch consecutive rows,
-// lane l owning rows l*kBatch .. l*kBatch + kBatch - 1 of it, so a row's
-// prefix = earlier batches' total + lower lanes' sums + its lane's earlier
-// rows.  All loads of a batch are issued before any is used.
-__device__ int32_t column_scan(int32_t* M, int64_t nrows, int ncol, int col, bool write_prefix)
+// Large batches in one cooperative launch with a single grid barrier.  One
+// tile per CTA: kTileWarps warps of wt consecutive tokens each, wt chosen on
+// the host so that the tiles cover the SMs once.  Tiles form groups of gs
+// consecutive tiles.  Counts travel as uint16 pairs packed in 32-bit words
+// (a row of ldw = ceil(E / 8) * 4 words), which the host bounds: a group
+// holds fewer than 2^16 entries.
+//   phase 1  each warp loads its tokens' entries into shared memory and
+//            counts them into its own histogram row (shared atomics); the
+//            tile's expert counts go to its row of tile_rows and are added
+//            (red.add of the packed pairs: no carry crosses a half) to its
+//            group's row, its tokens-per-rank counts to per-rank sums;
+//            is_token_in_rank bytes;
+//   barrier  the only grid-wide wait;
+//   phase 2  every CTA reads all group rows (their sum is the expert totals;
+//            the rows of the groups before its own are most of its prefix)
+//            and the rows of the tiles before it in its group, with 16-byte
+//            loads all requested before any is used: about 2 sqrt(tiles) rows
+//            instead of one per tile.  One pass over the experts then sums the
+//            partial rows and scans the padded totals into expert_off (in
+//            every CTA, so no second grid-wide wait is needed); CTA 0 writes
+//            the totals, the offsets and the tokens per rank;
+//   phase 3  position = the tile's first row of the expert + the entry's
+//            place inside the tile's block of it, which each warp computed
+//            while it waited at the barrier (its warp prefix plus its rank
+//            among the equal experts before it, entries replayed in order);
+//            the pad rows of recv_src are set to -1.
+// The sums are double-buffered by launch: the epoch word's parity picks the
+// buffer a launch adds into, and the launch clears the other one for the
+// next launch (which starts after this one has finished); the last arrival
+// at the barrier advances the epoch, after every CTA has read it.
+// Shared memory (words, 16-byte aligned part first): part[nrg][nc][16]
+// (phase-2 partial sums, nc = ldw / 4), ents[W][wt k], erank[W][wt k] (entry
+// ranks, then their places in the tile), run[W][E] (warp histograms, then
+// warp prefixes), off[E+1], pre[E], tot[E], wsum[32], rhist[R], rtot[R].
+constexpr int kTileWarps = 8;                    // warps that own tokens
+constexpr int kTileThreads = 32 * kTileWarps;
+constexpr int kTileBlock = kTileThreads + 32;    // + one warp that holds the grid barrier
+constexpr int kRowBatch = 4;   // rows per thread requested together in phase 2
+constexpr int kMaxGroups = kTileMaxGroups;
+
+__host__ __device__ inline int tile_ldw(int E) { return ((E + 7) / 8) * 4; }
+
+__host__ __device__ inline size_t tile_smem_words(int wt, int k, int E, int R)
 {
-    const int lane = threadIdx.x & 31;
-    int32_t base = 0;
-    for (int64_t b0 = 0; b0 < nrows; b0 += 32 * kBatch) {
-        const int64_t r0 = b0 + (int64_t)lane * kBatch;
-        int32_t v[kBatch];
-#pragma unroll
-        for (int m = 0; m < kBatch; ++m) v[m] = (r0 + m < nrows) ? M[(r0 + m) * ncol + col] : 0;
-        int32_t sum = 0;
-#pragma unroll
-        for (int m = 0; m < kBatch; ++m) sum += v[m];
-        int32_t incl = sum;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t u = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o)
-                incl += u;
-        }
-        if (write_prefix) {
-            int32_t run = base + incl - sum;
-#pragma unroll
-            for (int m = 0; m < kBatch; ++m)
-                if (r0 + m < nrows) {
-                    M[(r0 + m) * ncol + col] = run;
-                    run += v[m];
-                }
-        }
-        base += __shfl_sync(kFull, incl, 31);
-    }
-    return base;
+    const int nc = tile_ldw(E) / 4, nrg = kTileThreads / nc;
+    return (size_t)nrg * nc * 16 + 2 * (size_t)kTileWarps * wt * k + (size_t)kTileWarps * E +
+           (size_t)(E + 1) + 2 * (size_t)E + 32 + 2 * (size_t)R;
 }
 
-// Large batches in one cooperative launch.  A tile is kTileWarps warps x
-// kWarpTokens tokens; the grid (all co-resident) strides over tiles.
-//   phase 1  per tile: each warp loads its tokens' entries into shared memory
-//            and counts them into its own histogram row; the tile's counts
-//            (sum of the rows), is_token_in_rank bytes and rank counts ->
-//            tile_counts / tile_rank rows in global memory;
-//   phase 2  one warp per column: exclusive prefix of tile_counts over tiles
-//            (in place) and the expert totals; the rank totals;
-//   phase 3  every CTA scans the padded expert sizes into expert_off; per
-//            tile, a per-expert scan over the warp rows (on top of the tile
-//            prefix) gives each warp its first free row per expert, and each
-//            warp replays its entries in order.
-// When every CTA owns one tile, the entries and warp rows stay in shared
-// memory from phase 1 to phase 3; otherwise phase 3 rebuilds them per tile.
-// Shared memory (words): ents[W][kWarpTokens k], run[W][E] (kept), then
-// phase 1: rank_hist[R], erank[W][kWarpTokens k]; phase 3: off[E+1],
-// wsum[32], cnt[E], tpre[E].
-constexpr int kTileWarps = 8;
-constexpr int kWarpTokens = 8;
-constexpr int kTileTokens = kTileWarps * kWarpTokens;
-
-__host__ __device__ inline size_t tile_smem_words(int k, int E, int R)
+__device__ __forceinline__ void red_add(int32_t* p, int32_t v)
 {
-    const size_t ent = (size_t)kTileWarps * kWarpTokens * k;
-    const size_t kept = ent + (size_t)kTileWarps * E;
-    const size_t p1 = (size_t)R + ent;
-    const size_t p3 = (size_t)E + 1 + 32 + E + E;
-    return kept + (p1 > p3 ? p1 : p3);
+    asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32)
+__global__ void __launch_bounds__(kTileBlock, 1)
 layout_tile_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R, int epr,
-                   uint64_t rank_magic, int block_m, int64_t ntiles,
-                   int32_t* __restrict__ tile_counts, int32_t* __restrict__ tile_rank,
+                   uint64_t rank_magic, int block_m, int bm_log, int k_log, int wt, int ntiles, int gs,
+                   int ngroups, uint32_t* __restrict__ tile_rows, int32_t* __restrict__ acc,
                    int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
                    int32_t* __restrict__ rank_off_g, int32_t* __restrict__ tokens_per_rank_g,
                    int32_t* __restrict__ rows_per_rank_g, int32_t* __restrict__ total_rows_g,
                    uint8_t* __restrict__ is_token_in_rank, int32_t* __restrict__ dst_row,
                    int32_t* __restrict__ recv_src, int32_t* err)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     pdl_wait();
     pdl_trigger();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nthr = blockDim.x;
-    const int64_t gwarp = (int64_t)blockIdx.x * kTileWarps + warp;
-    const int64_t nwarps_all = (int64_t)gridDim.x * kTileWarps;
-    const int went = kWarpTokens * k;
-    const bool resident = ntiles <= (int64_t)gridDim.x;  // one tile per CTA
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool worker = warp < kTileWarps;  // else the barrier warp
+    const int went = wt * k;
+    const int ldw = tile_ldw(E), nc = ldw >> 2, nrg = kTileThreads / nc;
+    const int tile = blockIdx.x, grp = tile / gs;
     int32_t* bar = err + 1;
-
-    int32_t* ents_all = smem;
-    int32_t* run_all = ents_all + (size_t)kTileWarps * went;
-    int32_t* scratch = run_all + (size_t)kTileWarps * E;
-    int32_t* ents = ents_all + (size_t)warp * went;
-    int32_t* run = run_all + (size_t)warp * E;
-
-    // A barrier that timed out earlier leaves its words inconsistent until
-    // ep_handle_check resets them: refuse to take part in the barriers (every
-    // CTA reads the same word).  Every CTA reads the launch's barrier base
-    // before it arrives at the first barrier, so before any CTA can finish
-    // the last barrier and store the next one.  Both words are requested
-    // here and used after phase 1, so their latency hides behind its loads.
-    __shared__ int stale;
-    __shared__ int32_t bar_base;
-    int32_t err_word = 0, base_word = 0;
-    if (threadIdx.x == 0) {
-        err_word = *(volatile int32_t*)err;
-        base_word = *(volatile int32_t*)(bar + 1);
-    }
-    const int32_t G = (int32_t)gridDim.x;
-
-    // a tile's entries into ents and each warp's histogram into its run row
-    auto load_tile = [&](int64_t tile, int32_t* erank) {
-        for (int e = lane; e < E; e += 32) run[e] = 0;
-        __syncwarp();
-        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
-        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
-        int bad = 0;
-        if (ntok > 0)
-            bad = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, ents, erank, run);
-        __syncwarp();
-        return bad;
+    int32_t* epoch_word = acc;
+    // acc: epoch word (padded to 16 bytes), then per buffer kMaxGroups group
+    // rows of ldw words and R tokens-per-rank sums
+    const size_t buf_words = (size_t)kMaxGroups * ldw + (size_t)((R + 3) & ~3);
+    int32_t* bufs = acc + 4;
+    auto padded = [&](int32_t c) {
+        return bm_log >= 0 ? ((c + block_m - 1) >> bm_log) << bm_log : pad_up(c, block_m);
     };
 
-    // ---- phase 1
-    {
-        int32_t* rhist = scratch;
-        int32_t* erank = rhist + R + (size_t)warp * went;
-        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            for (int r = threadIdx.x; r < R; r += nthr) rhist[r] = 0;
-            __syncthreads();
-            const int bad = load_tile(tile, erank);
-            if (bad && lane == 0)
-                atomicOr(err, kErrBadIndex);
-            const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
-            const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
-            if (ntok > 0)
-                chunk_rank_bytes(erank, ntok, k, R, t0, is_token_in_rank, rhist);
-            __syncthreads();
-            for (int e = threadIdx.x; e < E; e += nthr) {
-                int32_t h = 0;
-                for (int w = 0; w < kTileWarps; ++w) h += run_all[(size_t)w * E + e];
-                tile_counts[tile * E + e] = h;
-            }
-            for (int r = threadIdx.x; r < R; r += nthr) tile_rank[tile * R + r] = rhist[r];
-            __syncthreads();
-        }
+    int32_t* part = smem;
+    int32_t* ents_all = part + nrg * nc * 16;
+    int32_t* erank_all = ents_all + kTileWarps * went;
+    int32_t* run_all = erank_all + kTileWarps * went;
+    int32_t* off = run_all + kTileWarps * E;
+    int32_t* pre = off + E + 1;
+    int32_t* tot = pre + E;
+    int32_t* wsum = tot + E;
+    int32_t* rhist = wsum + 32;
+    int32_t* rtot = rhist + R;
+    int32_t* ents = ents_all + warp * went;
+    int32_t* run = run_all + warp * E;
+
+    // A barrier that timed out earlier leaves its words inconsistent until
+    // ep_handle_check resets them: refuse to take part (every CTA reads the
+    // same word).  Every CTA reads the barrier base and the epoch before it
+    // arrives, so before the last arrival stores the next ones.  The words
+    // are requested here and used after the loads of phase 1.
+    __shared__ int stale;
+    __shared__ int32_t bar_base, epoch;
+    int32_t err_word = 0, base_word = 0, epoch_w = 0;
+    if (tid == 0) {
+        err_word = *(volatile int32_t*)err;
+        base_word = *(volatile int32_t*)(bar + 1);
+        epoch_w = *(volatile int32_t*)epoch_word;
     }
-    if (threadIdx.x == 0) {
+
+    // ---- phase 1
+    if (worker) {
+        for (int e = lane; e < E; e += 32) run[e] = 0;
+        for (int r = tid; r < R; r += kTileThreads) rhist[r] = 0;
+    }
+    __syncthreads();
+    const int64_t t0 = ((int64_t)tile * kTileWarps + warp) * wt;
+    const int ntok = worker ? (int)max((int64_t)0, min((int64_t)wt, (int64_t)T - t0)) : 0;
+    if (ntok > 0) {
+        int32_t* erank = erank_all + warp * went;
+        const int bad = load_chunk(topk_idx + t0 * k, ntok * k, E, rank_magic, ents, erank, run);
+        if (bad && lane == 0)
+            atomicOr(err, kErrBadIndex);
+        __syncwarp();
+        for (int tb = 0; tb < ntok; tb += 32)
+            chunk_rank_bytes(erank + tb * k, min(32, ntok - tb), k, R, t0 + tb, is_token_in_rank,
+                             rhist);
+    }
+    if (tid == 0) {
         stale = (err_word & kErrTimeout) != 0;
         bar_base = base_word;
+        epoch = epoch_w;
     }
     __syncthreads();
+    int32_t* cur = bufs + (size_t)(epoch & 1) * buf_words;  // this launch's sums
+    int32_t* nxt = bufs + (size_t)((epoch & 1) ^ 1) * buf_words;
+    if (worker) {
+        uint32_t* grow = reinterpret_cast<uint32_t*>(cur) + (size_t)grp * ldw;
+        for (int i = tid; i < ldw; i += kTileThreads) {
+            uint32_t c[2] = {0u, 0u};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = 2 * i + h;
+                if (e < E)
+                    for (int w = 0; w < kTileWarps; ++w) {  // exclusive prefix over the warps
+                        const int32_t n = run_all[w * E + e];
+                        run_all[w * E + e] = (int32_t)c[h];
+                        c[h] += (uint32_t)n;
+                    }
+            }
+            const uint32_t pk = c[0] | (c[1] << 16);
+            tile_rows[(size_t)tile * ldw + i] = pk;
+            if (pk)
+                red_add(reinterpret_cast<int32_t*>(grow + i), (int32_t)pk);
+        }
+        int32_t* rsum = cur + (size_t)kMaxGroups * ldw;
+        for (int r = tid; r < R; r += kTileThreads)
+            if (rhist[r])
+                red_add(rsum + r, rhist[r]);
+    }
     if (stale)
         return;
-    if (!grid_barrier(bar, bar_base + G, false, err))
-        return;
-
-    // ---- phase 2
-    for (int64_t col = gwarp; col < E + R; col += nwarps_all) {
-        if (col < E) {
-            const int32_t tot = column_scan(tile_counts, ntiles, E, (int)col, true);
-            if (lane == 0)
-                cnt_g[col] = tot;
-        } else {
-            const int32_t tot = column_scan(tile_rank, ntiles, R, (int)(col - E), false);
-            if (lane == 0)
-                tokens_per_rank_g[col - E] = tot;
-        }
-    }
-    if (!grid_barrier(bar, bar_base + 2 * G, true, err))
-        return;
-
-    // ---- phase 3
-    int32_t* off = scratch;
-    int32_t* wsum = off + E + 1;
-    int32_t* cnt = wsum + 32;
-    int32_t* tpre = cnt + E;
-    int64_t tile = blockIdx.x;
-    {
-        for (int e = threadIdx.x; e < E; e += nthr) {
-            cnt[e] = cnt_g[e];
-            tpre[e] = tile_counts[tile * E + e];  // tile < ntiles: G <= ntiles
-        }
-    }
-    if (!resident)
-        (void)load_tile(tile, nullptr);
     __syncthreads();
-    scan_padded(cnt, E, block_m, off, wsum);
-    if (blockIdx.x == 0) {
-        for (int e = threadIdx.x; e <= E; e += nthr) expert_off_g[e] = off[e];
-        for (int r = threadIdx.x; r <= R; r += nthr) rank_off_g[r] = off[r * epr];
-        for (int r = threadIdx.x; r < R; r += nthr) {
-            int32_t s = 0;
-            for (int e = r * epr; e < (r + 1) * epr; ++e) s += cnt[e];
-            rows_per_rank_g[r] = s;
+    if (tid == kTileThreads)  // the barrier warp: its wait for the atomic stalls no token work
+        barrier_arrive(bar, bar_base + (int32_t)gridDim.x, epoch_word, epoch + 1);
+    // While the other tiles arrive: each warp replays its entries in order and
+    // gives each its position inside the tile's block of its expert (the warp
+    // prefix plus its rank among the equal experts before it), into lpos.
+    int32_t* lpos = erank_all + warp * went;
+    if (ntok > 0) {
+        const int nent = ntok * k;
+        const int ebits = 32 - __clz((unsigned)E);  // keys e + 1 in [0, E]
+        const unsigned lt = lanemask_lt();
+        for (int g = 0; g < nent; g += 32) {
+            const int f = g + lane;
+            const int e = f < nent ? ents[f] : -1;
+            const unsigned peers = match_key(e, ebits);
+            int32_t pos = -1;
+            if (e >= 0)
+                pos = run[e] + __popc(peers & lt);
+            __syncwarp();
+            if (e >= 0 && (peers & lt) == 0)
+                run[e] += __popc(peers);
+            __syncwarp();
+            if (f < nent)
+                lpos[f] = pos;
         }
-        if (threadIdx.x == 0)
+    }
+    if (!barrier_wait(bar, bar_base + (int32_t)gridDim.x, err, tid == kTileThreads))
+        return;
+
+    // ---- phase 2: totals and this tile's prefix
+    {
+        const int c = tid % nc, g = tid / nc;
+        const int gfirst = grp * gs;
+        const int nr = ngroups + (tile - gfirst);  // group rows, then tiles before this one
+        int32_t apre[8], atot[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) apre[i] = atot[i] = 0;
+        if (g < nrg) {
+            const uint32_t* grows = reinterpret_cast<const uint32_t*>(cur);
+            for (int j0 = g; j0 < nr; j0 += nrg * kRowBatch) {
+                int4 v[kRowBatch];
+#pragma unroll
+                for (int m = 0; m < kRowBatch; ++m) {
+                    const int j = j0 + m * nrg;
+                    const uint32_t* row = j < ngroups ? grows + (size_t)j * ldw
+                                                      : tile_rows + (size_t)(gfirst + j - ngroups) * ldw;
+                    v[m] = j < nr ? __ldcg(reinterpret_cast<const int4*>(row) + c)
+                                  : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int m = 0; m < kRowBatch; ++m) {
+                    const int j = j0 + m * nrg;
+                    const int32_t in_tot = j < ngroups ? -1 : 0;
+                    const int32_t in_pre = (j < grp || j >= ngroups) ? -1 : 0;
+                    const uint32_t wv[4] = {(uint32_t)v[m].x, (uint32_t)v[m].y, (uint32_t)v[m].z,
+                                            (uint32_t)v[m].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int32_t lo = (int32_t)(wv[i] & 0xffffu), hi = (int32_t)(wv[i] >> 16);
+                        atot[2 * i] += lo & in_tot;
+                        atot[2 * i + 1] += hi & in_tot;
+                        apre[2 * i] += lo & in_pre;
+                        apre[2 * i + 1] += hi & in_pre;
+                    }
+                }
+            }
+            int4* pp = reinterpret_cast<int4*>(part + (g * nc + c) * 16);
+            pp[0] = make_int4(apre[0], apre[1], apre[2], apre[3]);
+            pp[1] = make_int4(apre[4], apre[5], apre[6], apre[7]);
+            pp[2] = make_int4(atot[0], atot[1], atot[2], atot[3]);
+            pp[3] = make_int4(atot[4], atot[5], atot[6], atot[7]);
+        }
+        if (blockIdx.x == 0 && worker) {
+            const int32_t* rsum = cur + (size_t)kMaxGroups * ldw;
+            for (int r = tid; r < R; r += kTileThreads) rtot[r] = __ldcg(rsum + r);
+        }
+        // clear the other buffer for the next launch (no one reads it now)
+        if (worker)
+            for (int64_t i = (int64_t)blockIdx.x * kTileThreads + tid; i < (int64_t)buf_words;
+                 i += (int64_t)gridDim.x * kTileThreads)
+                nxt[i] = 0;
+    }
+    __syncthreads();
+    // One pass over the experts, thread tid owning [e0, e1) (empty for the
+    // barrier warp): the partial rows summed, the padded totals scanned across
+    // the block (each warp scans the warp sums itself), and the tile's first
+    // row per expert.
+    {
+        const int seg = (E + kTileThreads - 1) / kTileThreads;
+        const int e0 = min(E, tid * seg), e1 = min(E, e0 + seg);
+        int32_t local = 0;
+        for (int e = e0; e < e1; ++e) {
+            const int cc = e >> 3, j = e & 7;
+            int32_t p = 0, s = 0;
+            for (int g = 0; g < nrg; ++g) {
+                const int32_t* q = part + (g * nc + cc) * 16;
+                p += q[j];
+                s += q[8 + j];
+            }
+            pre[e] = p;
+            tot[e] = s;
+            local += padded(s);
+        }
+        int32_t incl = local;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o)
+                incl += u;
+        }
+        if (lane == 31)
+            wsum[warp] = incl;
+        __syncthreads();
+        const int32_t wv = lane < kTileWarps ? wsum[lane] : 0;
+        int32_t winc = wv;
+        for (int o = 1; o < kTileWarps; o <<= 1) {
+            const int32_t u = __shfl_up_sync(kFull, winc, o);
+            if (lane >= o)
+                winc += u;
+        }
+        int32_t at = __shfl_sync(kFull, winc - wv, warp) + incl - local;
+        for (int e = e0; e < e1; ++e) {
+            off[e] = at;
+            pre[e] += at;  // the tile's first row of expert e
+            at += padded(tot[e]);
+        }
+        if (tid == kTileThreads - 1)
+            off[E] = at;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && worker) {
+        for (int e = tid; e < E; e += kTileThreads) cnt_g[e] = tot[e];
+        for (int e = tid; e <= E; e += kTileThreads) expert_off_g[e] = off[e];
+        for (int r = tid; r <= R; r += kTileThreads) rank_off_g[r] = off[r * epr];
+        for (int r = tid; r < R; r += kTileThreads) {
+            int32_t s = 0;
+            for (int e = r * epr; e < (r + 1) * epr; ++e) s += tot[e];
+            rows_per_rank_g[r] = s;
+            tokens_per_rank_g[r] = rtot[r];
+        }
+        if (tid == 0)
             *total_rows_g = off[E];
     }
-    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
-    for (int64_t e = gwarp; e < E; e += nwarps_all)
-        fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
 
-    for (; tile < ntiles; tile += gridDim.x) {
-        if (tile != blockIdx.x) {
-            __syncthreads();  // the previous tile is done with run / ents / tpre
-            (void)load_tile(tile, nullptr);
-            for (int e = threadIdx.x; e < E; e += nthr) tpre[e] = tile_counts[tile * E + e];
-            __syncthreads();
+    // ---- phase 3
+    if (ntok > 0) {
+        const int nent = ntok * k;
+        for (int f = lane; f < nent; f += 32) {
+            const int e = ents[f];
+            const int32_t pos = e >= 0 ? pre[e] + lpos[f] : -1;
+            dst_row[t0 * k + f] = pos;
+            if (pos >= 0)
+                recv_src[pos] = (int32_t)(t0 + (k_log >= 0 ? f >> k_log : f / k));
         }
-        // run[w][e] = off[e] + tile prefix + the counts of earlier warps
-        for (int e = threadIdx.x; e < E; e += nthr) {
-            int32_t acc = off[e] + tpre[e];
-            for (int w = 0; w < kTileWarps; ++w) {
-                const int32_t h = run_all[(size_t)w * E + e];
-                run_all[(size_t)w * E + e] = acc;
-                acc += h;
-            }
-        }
-        __syncthreads();
-        const int64_t t0 = tile * kTileTokens + (int64_t)warp * kWarpTokens;
-        const int ntok = (int)max((int64_t)0, min((int64_t)kWarpTokens, (int64_t)T - t0));
-        if (ntok > 0)
-            chunk_assign(ents, ntok * k, k, E, t0, run, dst_row, recv_src);
     }
+    const bool vec = ((uintptr_t)recv_src & 15u) == 0;
+    if (worker)
+        for (int64_t e = (int64_t)blockIdx.x * kTileWarps + warp; e < E;
+             e += (int64_t)gridDim.x * kTileWarps)
+            fill_pad(recv_src, off[e] + tot[e], off[e + 1], vec);
 }
 
 uint64_t rank_magic_for(int epr) { return ((uint64_t(1) << 32) + (uint64_t)epr - 1) / (uint64_t)epr; }
@@ -1157,44 +1265,87 @@ cudaError_t set_smem(const void* fn, size_t bytes)
     return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// 0: not yet tried; 1: cooperative launches also take programmatic dependent
+// launch; -1: they refused it (cooperative alone).
+std::atomic<int> g_coop_pdl{0};
+
 }  // namespace
 
-// The single-launch layout: kTileWarps warps per CTA, G CTAs = min(tiles,
-// CTAs that fit on the GPU at once), cooperative so that all are resident.
+size_t tile_acc_words(int E, int R)
+{
+    return 4 + 2 * ((size_t)kMaxGroups * tile_ldw(E) + (size_t)((R + 3) & ~3));
+}
+
+// The single-launch layout: tiles of kTileWarps x wt tokens, one per CTA,
+// at most one CTA per SM, cooperative so that all CTAs are resident.
+// Returns cudaErrorCooperativeLaunchTooLarge when the shape does not suit it
+// (the caller then runs the three kernels).
 cudaError_t launch_fused(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
-    const size_t smem = sizeof(int32_t) * tile_smem_words(k, E, R);
-    if (smem > kSmemBudget)
-        return cudaErrorCooperativeLaunchTooLarge;  // the caller uses three kernels
-    const int64_t ntiles = ((int64_t)T + kTileTokens - 1) / kTileTokens;
+    const int ldw = tile_ldw(E);
+    if (ldw / 4 > kTileThreads || !h.tile_acc)
+        return cudaErrorCooperativeLaunchTooLarge;
     cudaError_t rc;
+    int dev = 0, sms = 0;
+    if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+        (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return rc;
+    // tokens per warp: the tiles cover the SMs once, and a tile holds at least
+    // kChunkTokens tokens (so the tile rows fit in the chunk count matrix)
+    int64_t wt = ((int64_t)T + (int64_t)kTileWarps * sms - 1) / ((int64_t)kTileWarps * sms);
+    wt = std::max<int64_t>(wt, kChunkTokens / kTileWarps);
+    const int64_t ntiles = ((int64_t)T + kTileWarps * wt - 1) / (kTileWarps * wt);
+    if (ntiles > (int64_t)kMaxGroups * kMaxGroups || ntiles * ldw > h.max_chunks * (int64_t)E)
+        return cudaErrorCooperativeLaunchTooLarge;
+    int gs = 1;  // group size: about sqrt(tiles), so that groups and tiles per group balance
+    while ((int64_t)gs * gs < ntiles) ++gs;
+    const int ngroups = (int)((ntiles + gs - 1) / gs);
+    if ((int64_t)gs * kTileWarps * wt * k > 65535)  // a group's count of one expert in 16 bits
+        return cudaErrorCooperativeLaunchTooLarge;
+    const size_t smem = sizeof(int32_t) * tile_smem_words((int)wt, k, E, R);
+    if (smem > kSmemBudget)
+        return cudaErrorCooperativeLaunchTooLarge;
     if ((rc = set_smem((const void*)layout_tile_kernel, smem)) != cudaSuccess)
         return rc;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
-        (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-        (rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_tile_kernel,
-                                                            32 * kTileWarps, smem)) != cudaSuccess)
+    int per_sm = 0;
+    if ((rc = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_tile_kernel,
+                                                            kTileBlock, smem)) != cudaSuccess)
         return rc;
-    if (per_sm < 1)
+    if (per_sm < 1 || ntiles > (int64_t)sms * per_sm)
         return cudaErrorCooperativeLaunchTooLarge;
-    const unsigned grid = (unsigned)std::min<int64_t>(ntiles, (int64_t)sms * per_sm);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(32 * kTileWarps);
+    cfg.gridDim = dim3((unsigned)ntiles);
+    cfg.blockDim = dim3(kTileBlock);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layout_tile_kernel, topk_idx, T, k, E, R, epr,
-                              rank_magic_for(epr), h.block_m, ntiles, h.chunk_counts,
-                              h.chunk_rank, h.cnt, h.expert_off, h.rank_off, h.tokens_per_rank,
-                              h.rows_per_rank, h.total_rows, h.is_token_in_rank, h.dst_row,
-                              h.recv_src, h.err);
+    auto launch = [&](int nattrs) {
+        cfg.numAttrs = nattrs;
+        return cudaLaunchKernelEx(&cfg, layout_tile_kernel, topk_idx, T, k, E, R, epr,
+                                  rank_magic_for(epr), h.block_m, log2_if_pow2(h.block_m),
+                                  log2_if_pow2(k), (int)wt, (int)ntiles, gs, ngroups,
+                                  reinterpret_cast<uint32_t*>(h.chunk_counts), h.tile_acc, h.cnt,
+                                  h.expert_off, h.rank_off, h.tokens_per_rank, h.rows_per_rank,
+                                  h.total_rows, h.is_token_in_rank, h.dst_row, h.recv_src, h.err);
+    };
+    if (g_coop_pdl.load() >= 0) {
+        rc = launch(2);
+        if (rc == cudaSuccess) {
+            g_coop_pdl = 1;
+            return rc;
+        }
+        if (g_coop_pdl.load() == 1 || (rc != cudaErrorInvalidValue && rc != cudaErrorNotSupported))
+            return rc;
+        (void)cudaGetLastError();  // refused: cooperative launches without PDL from now on
+        g_coop_pdl = -1;
+    }
+    return launch(1);
 }
 
 cudaError_t launch_layout(const Handle& h, const int64_t* topk_idx, int T, cudaStream_t s,
