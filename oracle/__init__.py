@@ -16,6 +16,7 @@ Every function cites the passage of the pages it follows in ``ep_oracle.c``.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -27,8 +28,11 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ep_oracle.c")
 _LIB = os.path.join(_HERE, "libep_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libep_oracle_omp.so")  # the same source with -fopenmp
 _lock = threading.Lock()
 _lib = None
+_lib_omp = None
+_active = None  # the OpenMP build while `threads` is in effect
 
 OK = 0
 ERR_ARG = 1
@@ -36,58 +40,94 @@ ERR_CAPACITY = 4
 ERR_BAD_INDEX = 5
 
 
-def build(force: bool = False) -> str:
-    """Compile ``ep_oracle.c`` into ``libep_oracle.so`` (gcc, -O2, strict fp)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp.%d" % os.getpid()
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile ``ep_oracle.c`` into ``libep_oracle.so`` (gcc, -O2, strict fp),
+    or with ``openmp`` into ``libep_oracle_omp.so``: the same source with its
+    token loops parallel over tokens, used only to time the oracle on all
+    host cores (its outputs are byte-identical, which a test pins)."""
+    out = _LIB_OMP if openmp else _LIB
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + ".tmp.%d" % os.getpid()
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-               "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+               "-fno-fast-math", "-Wall", "-Wextra",
+               "-fopenmp" if openmp else "-Wno-unknown-pragmas", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, out)
+    return out
 
 
 def _load():
     global _lib
+    if _active is not None:
+        return _active
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
-            P = ctypes.c_void_p
-            i64, i32 = ctypes.c_int64, ctypes.c_int
-            lib.oracle_layout.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i64, P]
-            lib.oracle_layout.restype = i32
-            lib.oracle_recv_rows_bound.argtypes = [i64, i32, i32, i32]
-            lib.oracle_recv_rows_bound.restype = i64
-            lib.oracle_dispatch_bf16.argtypes = [P, i64, i32, i64, P, P, i64]
-            lib.oracle_dispatch_bf16.restype = i32
-            lib.oracle_dispatch_fp8.argtypes = [P, i64, i32, i64, i32, P, P, P, i64]
-            lib.oracle_dispatch_fp8.restype = i32
-            lib.oracle_quantize_token_fp8.argtypes = [P, i64, i32, P, P]
-            lib.oracle_quantize_token_fp8.restype = None
-            lib.oracle_expert_scale_bf16.argtypes = [P, P, P, i32, i64, P, P]
-            lib.oracle_expert_scale_bf16.restype = None
-            lib.oracle_expert_scale_fp8.argtypes = [P, P, P, P, i32, i64, P, P]
-            lib.oracle_expert_scale_fp8.restype = None
-            lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, i32, P]
-            lib.oracle_combine.restype = i32
-            lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, i32, P]
-            lib.oracle_dispatch_backward.restype = i32
-            lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, i32, P, P]
-            lib.oracle_combine_backward.restype = i32
-            lib.oracle_dispatch_weights.argtypes = [P, P, i64, i32, P, i64]
-            lib.oracle_dispatch_weights.restype = i32
-            lib.oracle_zero_pad_rows.argtypes = [P, i64, P, i64]
-            lib.oracle_zero_pad_rows.restype = None
-            lib.oracle_dispatch_fp8_mn.argtypes = [P, i64, i32, i64, i32, P, P, P, i64, i64]
-            lib.oracle_dispatch_fp8_mn.restype = i32
-            for name in ("oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
-                         "oracle_f32_to_bf16_array", "oracle_fp16_to_f32_array",
-                         "oracle_f32_to_fp16_array"):
-                getattr(lib, name).argtypes = [P, P, i64]
-                getattr(lib, name).restype = None
-            _lib = lib
+            _lib = _configure(ctypes.CDLL(build()))
     return _lib
+
+
+def _load_omp():
+    global _lib_omp
+    with _lock:
+        if _lib_omp is None:
+            _lib_omp = _configure(ctypes.CDLL(build(openmp=True)))
+    return _lib_omp
+
+
+@contextlib.contextmanager
+def threads(n: int = 0):
+    """Inside the block, oracle calls run on the OpenMP build with n threads
+    (0: the OpenMP default, all host cores); yields the thread count.  For
+    timing the oracle on the host's cores; the results are the same bytes."""
+    global _active
+    lib = _load_omp()
+    got = int(lib.oracle_set_threads(n))
+    prev = _active
+    _active = lib
+    try:
+        yield got
+    finally:
+        _active = prev
+
+
+def _configure(lib):
+    """Argument and result types of the oracle's C functions."""
+    P = ctypes.c_void_p
+    i64, i32 = ctypes.c_int64, ctypes.c_int
+    lib.oracle_layout.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i64, P]
+    lib.oracle_layout.restype = i32
+    lib.oracle_recv_rows_bound.argtypes = [i64, i32, i32, i32]
+    lib.oracle_recv_rows_bound.restype = i64
+    lib.oracle_dispatch_bf16.argtypes = [P, i64, i32, i64, P, P, i64]
+    lib.oracle_dispatch_bf16.restype = i32
+    lib.oracle_dispatch_fp8.argtypes = [P, i64, i32, i64, i32, P, P, P, i64]
+    lib.oracle_dispatch_fp8.restype = i32
+    lib.oracle_quantize_token_fp8.argtypes = [P, i64, i32, P, P]
+    lib.oracle_quantize_token_fp8.restype = None
+    lib.oracle_expert_scale_bf16.argtypes = [P, P, P, i32, i64, P, P]
+    lib.oracle_expert_scale_bf16.restype = None
+    lib.oracle_expert_scale_fp8.argtypes = [P, P, P, P, i32, i64, P, P]
+    lib.oracle_expert_scale_fp8.restype = None
+    lib.oracle_combine.argtypes = [P, i64, P, P, i64, i32, i64, i32, P]
+    lib.oracle_combine.restype = i32
+    lib.oracle_dispatch_backward.argtypes = [P, i64, P, i64, i32, i64, i32, P]
+    lib.oracle_dispatch_backward.restype = i32
+    lib.oracle_combine_backward.argtypes = [P, P, i64, P, P, i64, i32, i64, i32, P, P]
+    lib.oracle_combine_backward.restype = i32
+    lib.oracle_dispatch_weights.argtypes = [P, P, i64, i32, P, i64]
+    lib.oracle_dispatch_weights.restype = i32
+    lib.oracle_zero_pad_rows.argtypes = [P, i64, P, i64]
+    lib.oracle_zero_pad_rows.restype = None
+    lib.oracle_dispatch_fp8_mn.argtypes = [P, i64, i32, i64, i32, P, P, P, i64, i64]
+    lib.oracle_dispatch_fp8_mn.restype = i32
+    for name in ("oracle_f32_to_e4m3_array", "oracle_e4m3_to_f32_array",
+                 "oracle_f32_to_bf16_array", "oracle_fp16_to_f32_array",
+                 "oracle_f32_to_fp16_array"):
+        getattr(lib, name).argtypes = [P, P, i64]
+        getattr(lib, name).restype = None
+    lib.oracle_set_threads.argtypes = [i32]
+    lib.oracle_set_threads.restype = i32
+    return lib
 
 
 def _p(a: np.ndarray):

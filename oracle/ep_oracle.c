@@ -43,11 +43,20 @@
  * see the test files named test_oracle_*.py.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math).
+ * The same source also builds with -fopenmp, only to time the oracle on all
+ * host cores: the token loops of dispatch, combine and the backward then run
+ * in parallel over tokens.  Every token's arithmetic is the same sequence of
+ * operations either way (a token is computed by one thread), so both builds
+ * give identical bytes; the layout stays serial.  Without -fopenmp the
+ * pragmas are ignored.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define OR_OK 0
 #define OR_ERR_ARG 1
@@ -378,6 +387,29 @@ int oracle_layout(const int64_t* topk_idx, int64_t T, int k, int E, int R, int b
     return OR_OK;
 }
 
+/* Threads of the parallel build (a no-op returning 1 in the serial one). */
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/* 1 if every row named in dst_row[0..n) is below cap (checked before the
+ * token loops, which then have no early exit). */
+static int rows_below(const int32_t* dst_row, int64_t n, int64_t cap)
+{
+    for (int64_t i = 0; i < n; ++i)
+        if (dst_row[i] >= cap)
+            return 0;
+    return 1;
+}
+
 /* ------------------------------------------------------------------ */
 /* Dispatch.                                                            */
 /* ------------------------------------------------------------------ */
@@ -388,14 +420,14 @@ int oracle_layout(const int64_t* topk_idx, int64_t T, int k, int E, int R, int b
 int oracle_dispatch_bf16(const uint16_t* x, int64_t T, int k, int64_t H,
                          const int32_t* dst_row, uint16_t* recv_x, int64_t recv_cap)
 {
+    if (!rows_below(dst_row, T * k, recv_cap))
+        return OR_ERR_CAPACITY;
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {
             int64_t d = dst_row[t * k + j];
-            if (d < 0)
-                continue;
-            if (d >= recv_cap)
-                return OR_ERR_CAPACITY;
-            memcpy(recv_x + d * H, x + t * H, sizeof(uint16_t) * (size_t)H);
+            if (d >= 0)
+                memcpy(recv_x + d * H, x + t * H, sizeof(uint16_t) * (size_t)H);
         }
     return OR_OK;
 }
@@ -442,31 +474,34 @@ int oracle_dispatch_fp8(const uint16_t* x, int64_t T, int k, int64_t H, int dtyp
 {
     if (H % 128 != 0)
         return OR_ERR_ARG;
+    if (!rows_below(dst_row, T * k, recv_cap))
+        return OR_ERR_CAPACITY;
     const int64_t nb = H / 128;
-    uint8_t* q = (uint8_t*)malloc((size_t)H);
-    float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
-    if (!q || !s) {
+    int rc = OR_OK;
+#pragma omp parallel
+    {
+        uint8_t* q = (uint8_t*)malloc((size_t)(H > 0 ? H : 1));
+        float* s = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+        if (!q || !s) {
+#pragma omp atomic write
+            rc = OR_ERR_ARG;
+        }
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            if (!q || !s)
+                continue;
+            oracle_quantize_token_fp8(x + t * H, H, dtype, q, s);
+            for (int j = 0; j < k; ++j) {
+                int64_t d = dst_row[t * k + j];
+                if (d < 0)
+                    continue;
+                memcpy(recv_q + d * H, q, (size_t)H);
+                memcpy(recv_scales + d * nb, s, sizeof(float) * (size_t)nb);
+            }
+        }
         free(q);
         free(s);
-        return OR_ERR_ARG;
     }
-    int rc = OR_OK;
-    for (int64_t t = 0; t < T && rc == OR_OK; ++t) {
-        oracle_quantize_token_fp8(x + t * H, H, dtype, q, s);
-        for (int j = 0; j < k; ++j) {
-            int64_t d = dst_row[t * k + j];
-            if (d < 0)
-                continue;
-            if (d >= recv_cap) {
-                rc = OR_ERR_CAPACITY;
-                break;
-            }
-            memcpy(recv_q + d * H, q, (size_t)H);
-            memcpy(recv_scales + d * nb, s, sizeof(float) * (size_t)nb);
-        }
-    }
-    free(q);
-    free(s);
     return rc;
 }
 
@@ -524,29 +559,36 @@ void oracle_expert_scale_fp8(const uint8_t* recv_q, const float* recv_scales,
 int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int32_t* dst_row,
                    int64_t T, int k, int64_t H, int dtype, uint16_t* out)
 {
-    float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
-    if (!acc)
-        return OR_ERR_ARG;
-    for (int64_t t = 0; t < T; ++t) {
-        for (int64_t h = 0; h < H; ++h)
-            acc[h] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            int64_t d = dst_row[t * k + j];
-            if (d < 0)
-                continue;
-            if (d >= y_rows) {
-                free(acc);
-                return OR_ERR_CAPACITY;
-            }
-            const float wj = w[t * k + j];
-            for (int64_t h = 0; h < H; ++h)
-                acc[h] = fmaf(wj, in16_to_f32(y[d * H + h], dtype), acc[h]);
+    if (!rows_below(dst_row, T * k, y_rows))
+        return OR_ERR_CAPACITY;
+    int rc = OR_OK;
+#pragma omp parallel
+    {
+        float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
+        if (!acc) {
+#pragma omp atomic write
+            rc = OR_ERR_ARG;
         }
-        for (int64_t h = 0; h < H; ++h)
-            out[t * H + h] = f32_to_out16(acc[h], dtype);
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            if (!acc)
+                continue;
+            for (int64_t h = 0; h < H; ++h)
+                acc[h] = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int64_t d = dst_row[t * k + j];
+                if (d < 0)
+                    continue;
+                const float wj = w[t * k + j];
+                for (int64_t h = 0; h < H; ++h)
+                    acc[h] = fmaf(wj, in16_to_f32(y[d * H + h], dtype), acc[h]);
+            }
+            for (int64_t h = 0; h < H; ++h)
+                out[t * H + h] = f32_to_out16(acc[h], dtype);
+        }
+        free(acc);
     }
-    free(acc);
-    return OR_OK;
+    return rc;
 }
 
 /* ------------------------------------------------------------------ */
@@ -563,28 +605,35 @@ int oracle_combine(const uint16_t* y, int64_t y_rows, const float* w, const int3
 int oracle_dispatch_backward(const uint16_t* grad_recv, int64_t rows, const int32_t* dst_row,
                              int64_t T, int k, int64_t H, int dtype, uint16_t* grad_x)
 {
-    float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
-    if (!acc)
-        return OR_ERR_ARG;
-    for (int64_t t = 0; t < T; ++t) {
-        for (int64_t h = 0; h < H; ++h)
-            acc[h] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            int64_t d = dst_row[t * k + j];
-            if (d < 0)
+    if (!rows_below(dst_row, T * k, rows))
+        return OR_ERR_CAPACITY;
+    int rc = OR_OK;
+#pragma omp parallel
+    {
+        float* acc = (float*)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
+        if (!acc) {
+#pragma omp atomic write
+            rc = OR_ERR_ARG;
+        }
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            if (!acc)
                 continue;
-            if (d >= rows) {
-                free(acc);
-                return OR_ERR_CAPACITY;
+            for (int64_t h = 0; h < H; ++h)
+                acc[h] = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int64_t d = dst_row[t * k + j];
+                if (d < 0)
+                    continue;
+                for (int64_t h = 0; h < H; ++h)
+                    acc[h] = acc[h] + in16_to_f32(grad_recv[d * H + h], dtype);
             }
             for (int64_t h = 0; h < H; ++h)
-                acc[h] = acc[h] + in16_to_f32(grad_recv[d * H + h], dtype);
+                grad_x[t * H + h] = f32_to_out16(acc[h], dtype);
         }
-        for (int64_t h = 0; h < H; ++h)
-            grad_x[t * H + h] = f32_to_out16(acc[h], dtype);
+        free(acc);
     }
-    free(acc);
-    return OR_OK;
+    return rc;
 }
 
 /* Backward of combine, out[t] = sum_j w[t][j] y[dst_row[t][j]]:
@@ -596,6 +645,9 @@ int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t
                             const float* w, const int32_t* dst_row, int64_t T, int k, int64_t H,
                             int dtype, uint16_t* grad_y, float* grad_w)
 {
+    if (!rows_below(dst_row, T * k, y_rows))
+        return OR_ERR_CAPACITY;
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t)
         for (int j = 0; j < k; ++j) {
             int64_t d = dst_row[t * k + j];
@@ -603,8 +655,6 @@ int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t
                 grad_w[t * k + j] = 0.0f;
                 continue;
             }
-            if (d >= y_rows)
-                return OR_ERR_CAPACITY;
             double dot = 0.0;
             for (int64_t h = 0; h < H; ++h) {
                 const float g = in16_to_f32(grad_out[t * H + h], dtype);
