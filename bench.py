@@ -625,11 +625,8 @@ def oracle_seconds_per_token(w, probe=512):
     return oracle_timed_step(w, smp) / smp["tokens"]
 
 
-def cpu_baseline(w, budget_s=15.0):
-    """The oracle as it stands, single-threaded, on a bounded token sample."""
-    import oracle
-
-    oracle.build()
+def _oracle_rate(w, budget_s):
+    """GB/s of oracle steps on a bounded token sample; (GB/s, tokens, reps)."""
     per_tok = oracle_seconds_per_token(w)
     tokens = int(min(w.T, max(min(w.T, 512), budget_s / 2.0 / max(per_tok, 1e-9))))
     smp = oracle_sample(w, tokens)
@@ -637,11 +634,26 @@ def cpu_baseline(w, budget_s=15.0):
     reps = min(5, max(1, int(budget_s / max(warm, 1e-9))))
     times = [oracle_timed_step(w, smp) for _ in range(reps)]
     d, c = algo_bytes(tokens, w.H, w.k, w.fmt)
-    gbs = (d + c) / statistics.mean(times) / 1e9
-    return {"value": round(gbs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "first %d of %d tokens of the same workload, 1 warm-up + %d timed "
-                      "repetitions, single-threaded C oracle (gcc -O2), "
-                      "layout+dispatch+combine" % (tokens, w.T, reps),
+    return (d + c) / statistics.mean(times) / 1e9, tokens, reps
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle as it stands, timed twice on bounded token samples: the
+    OpenMP build on all host cores (the reported value) and the
+    single-threaded build (the parity tests' ground truth)."""
+    import oracle
+
+    oracle.build()
+    oracle.build(openmp=True)
+    one, t1, r1 = _oracle_rate(w, budget_s)
+    with oracle.threads(0) as n:
+        alln, tn, rn = _oracle_rate(w, budget_s)
+    what = ("first %d of %d tokens of the same workload, 1 warm-up + %d timed repetitions, "
+            "C oracle (gcc -O2%s), layout (serial) + dispatch + combine")
+    return {"value": round(alln, 3), "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": what % (tn, w.T, rn, ", -fopenmp: tokens in parallel"),
+            "single_core": {"value": round(one, 3), "unit": UNIT, "cores": 1,
+                            "sample": what % (t1, w.T, r1, "")},
             "host": host_cpu()}
 
 
@@ -667,8 +679,15 @@ def run_reference(args, rank, world):
 
     import oracle
 
-    oracle.build()
+    oracle.build(openmp=True)
     w = make_workload(MAIN_WORKLOAD, 0)
+    with oracle.threads(0) as cores:
+        line = _reference_line(args, world, w, cores)
+    print(json.dumps(line), flush=True)
+
+
+def _reference_line(args, world, w, cores):
+    """The reference arm's steps (the oracle on `cores` threads) and its JSON line."""
     per_tok = oracle_seconds_per_token(w)
     budget = 120.0                                  # seconds of timed and warm-up steps
     per_step = budget / max(1, args.steps + args.warmup)
@@ -691,16 +710,26 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens_per_step": tokens},
-            "cpu_baseline": {"value": round(val, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": "first %d of %d tokens per step" % (tokens, w.T),
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": round(val, 3), "unit": UNIT, "cores": cores,
+                             "kind": "oracle",
+                             "sample": "first %d of %d tokens per step, C oracle (gcc -O2, "
+                                       "-fopenmp: tokens in parallel)" % (tokens, w.T),
                              "host": host_cpu()},
             "e2e": {"value": round(val, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 # ----------------------------------------------------------------- main
+
+def workload_config(w, world):
+    """The `config` object of the JSON line, the same in both arms."""
+    return {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens": w.T, "hidden": w.H,
+            "experts": w.E, "virtual_ranks": w.R, "topk": w.k, "fmt": w.fmt,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "flushed between steps (write of 2x L2), outside the events"}
+
 
 def aggregate_max(value: float, group=None) -> float:
     """Max over ranks (a scalar all-reduce; no data-path collective)."""
@@ -864,12 +893,9 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT[MAIN_WORKLOAD], "tokens": w.T, "hidden": w.H,
-                       "experts": w.E, "virtual_ranks": w.R, "topk": w.k, "fmt": w.fmt,
-                       "parallelism": "replicas" if world > 1 else "single GPU",
-                       "l2": "flushed between steps (write of 2x L2), outside the events",
-                       "bytes_per_step": d_bytes + c_bytes,
-                       "routing": routing_main},
+            "config": workload_config(w, world),
+            "bytes_per_step": d_bytes + c_bytes,
+            "routing": routing_main,
             "pct_of_measured_hbm": round(value / world / peak, 4),
             "pct_of_hbm_spec_8TBps": round(value / world / 8000.0, 4),
             "kernels": {"layout_us": round(lay_ms * 1e3, 2), "dispatch_us": round(dis_ms * 1e3, 2),
