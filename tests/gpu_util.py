@@ -71,3 +71,29 @@ def bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
 
 def nonpad_rows(lay) -> np.ndarray:
     return lay.dst_row[lay.dst_row >= 0].astype(np.int64)
+
+
+def grad_w_roundings(H):
+    """Roundings on the longest path of the combine backward's grad_w
+    reduction.  Rows of H % 16 == 0 (32-byte aligned, as torch allocates
+    them) take the one-warp-per-token kernel, as the per-rank combine
+    backward always does: each lane chains 16 fused multiply-adds per 32-byte
+    vector over ceil(H/16/32) vectors, then 5 xor-shuffle levels.  Other H
+    take the one-CTA-per-token kernel: each thread chains 8 per 16-byte
+    vector over its vectors, 5 shuffle levels, then the sum over the CTA's
+    warps in order."""
+    if H % 16 == 0:
+        vpr = H // 16
+        return 16 * -(-vpr // 32) + 5
+    vpr = H // 8
+    threads = min(256, 32 * -(-vpr // 32))
+    return 8 * -(-vpr // threads) + 5 + (threads // 32 - 1)
+
+
+def grad_w_bound(H, abs_dot, ref):
+    """gamma_n * sum|grad_out * y| (the bound of any summation tree whose
+    longest path has n roundings) plus half an fp32 ulp of the oracle's own
+    rounding of its fp64 dot product."""
+    n = grad_w_roundings(H)
+    u = 2.0 ** -24
+    return n * u / (1.0 - n * u) * abs_dot + u * abs(ref)

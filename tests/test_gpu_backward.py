@@ -2,14 +2,20 @@
 
 ep_dispatch_backward: bit-exact (fp32 sum in slot order, like combine).
 ep_combine_backward: grad_y bit-exact on every used row (one fp32 product,
-then bf16); pad rows keep their sentinel; grad_weights within the fp32
-summation bound H * 2^-24 * sum|grad_out * y| (plus the oracle's one
-rounding) of the oracle's fp64 dot product, and bitwise repeatable.
+then bf16); pad rows keep their sentinel; grad_weights within the error bound
+of the kernel's own reduction tree -- gamma_n * sum|grad_out * y| with
+gamma_n = n u / (1 - n u), u = 2^-24 and n the roundings on the longest path
+from a product to the result (each lane's chain of fused multiply-adds, the
+xor-shuffle tree, and for the 16-byte kernel the sum over warps) -- plus the
+oracle's one rounding of its fp64 dot product, and bitwise repeatable.  At
+H = 7168 that is n = 229, tight enough that one dropped 16-channel vector
+(an error of about N(0, 16) against a bound near 0.06) fails the check.
 """
 import numpy as np
 import pytest
 import torch
 
+from gpu_util import grad_w_bound
 from workloads import make_workload, make_x, random_topk
 
 pytestmark = pytest.mark.gpu
@@ -78,7 +84,7 @@ def _combine_backward_case(oracle, idx, E, R, H, rng, w=None):
             if d < 0:
                 assert gw_got[t, j] == 0.0
                 continue
-            bound = H * 2.0 ** -24 * float(np.abs(gf[t] * yf[d]).sum()) + 2.0 ** -24 * abs(gw_ref[t, j])
+            bound = grad_w_bound(H, float(np.abs(gf[t] * yf[d]).sum()), float(gw_ref[t, j]))
             assert abs(float(gw_got[t, j]) - float(gw_ref[t, j])) <= bound + 1e-30, (t, j)
     # bitwise repeatable
     _, gw2 = ep.ep_combine_backward(h, bits_to_bf16(g), bits_to_bf16(y),
@@ -126,7 +132,7 @@ def _f16_bits(t):
 ])
 def test_backward_fp16(oracle, T, H, E, R, k, p_unused):
     """fp16 rows: dispatch backward bit-exact; combine backward grad_y
-    bit-exact, grad_w within the fp32 summation bound of the fp64 dot."""
+    bit-exact, grad_w within the reduction tree's bound of the fp64 dot."""
     import combine_ep_layout_08_b200 as ep
     from workloads import make_x_fp16
 
@@ -159,5 +165,5 @@ def test_backward_fp16(oracle, T, H, E, R, k, p_unused):
             if d < 0:
                 assert gwg[t, j] == 0.0
                 continue
-            bound = H * 2.0 ** -24 * float(np.abs(gf[t] * yf[d]).sum()) + 2.0 ** -24 * abs(gw_ref[t, j])
+            bound = grad_w_bound(H, float(np.abs(gf[t] * yf[d]).sum()), float(gw_ref[t, j]))
             assert abs(float(gwg[t, j]) - float(gw_ref[t, j])) <= bound + 1e-30, (t, j)
