@@ -20,8 +20,8 @@
 namespace ep {
 
 namespace {
-
 thread_local char g_last_error[256] = "";
+}  // namespace
 
 ep_status_t cuda_fail(cudaError_t e, const char* where)
 {
@@ -29,6 +29,14 @@ ep_status_t cuda_fail(cudaError_t e, const char* where)
              cudaGetErrorString(e));
     return EP_ERR_CUDA;
 }
+
+ep_status_t fail_message(ep_status_t st, const char* what)
+{
+    snprintf(g_last_error, sizeof g_last_error, "%s", what);
+    return st;
+}
+
+namespace {
 
 constexpr size_t kAlign = 256;
 

@@ -65,6 +65,11 @@ struct Carve {
 };
 
 int64_t recv_rows_bound(int64_t T, int64_t k, int64_t E, int64_t block_m);
+
+// Record a CUDA error for ep_last_error_message and return EP_ERR_CUDA.
+ep_status_t cuda_fail(cudaError_t e, const char* where);
+// Record a message for ep_last_error_message and return st.
+ep_status_t fail_message(ep_status_t st, const char* what);
 bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c);
 
 // Programmatic dependent launch (sm_90+): every kernel of the library is

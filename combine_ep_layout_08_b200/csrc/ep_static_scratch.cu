@@ -3,11 +3,10 @@
 // policy when a buffer cannot be allocated ("DeepEP是什麼？…", section
 // ElasticBuffer); this entry point takes allocation out of the call.
 //
-// Some callers have no way to hand the library a workspace: code that runs
-// while a CUDA graph is being captured (allocation is not a capturable
-// operation), processes whose memory is owned up front by a framework
-// allocator or a pre-reserved pool that forbids further cudaMalloc calls, and
-// embedded or plug-in contexts that only receive input and output pointers.
+// Some callers have no way to hand the library a workspace: processes whose
+// device memory is owned up front by a framework allocator or a pre-reserved
+// pool that forbids further cudaMalloc calls, and embedded or plug-in
+// contexts that only receive input and output pointers.
 // This entry point needs nothing from them beyond those pointers: the layout's
 // only scratch (the per-chunk expert and rank count matrices) lives in a
 // fixed-size array of this library's own device memory, declared below, which
@@ -34,25 +33,27 @@ std::mutex g_mu;
 int32_t* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_layout_scratch on the current device (set-up on the
-// first call per device).
-cudaError_t scratch_address(int32_t** out)
+// first call per device).  Returns EP_OK or the status to report, with its
+// message recorded for ep_last_error_message.
+ep_status_t scratch_address(int32_t** out)
 {
     int dev = 0;
     cudaError_t rc = cudaGetDevice(&dev);
     if (rc != cudaSuccess)
-        return rc;
+        return cuda_fail(rc, "ep_layout_static_scratch: cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
+        return fail_message(EP_ERR_INVALID_ARG,
+                            "ep_layout_static_scratch: device ordinals above 63 are not served");
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
         rc = cudaGetSymbolAddress(&p, g_layout_scratch);
         if (rc != cudaSuccess)
-            return rc;
+            return cuda_fail(rc, "ep_layout_static_scratch: cudaGetSymbolAddress");
         g_scratch_addr[dev] = static_cast<int32_t*>(p);
     }
     *out = g_scratch_addr[dev];
-    return cudaSuccess;
+    return EP_OK;
 }
 
 }  // namespace
@@ -85,12 +86,13 @@ extern "C" ep_status_t ep_layout_static_scratch(
         return EP_ERR_ALIGNMENT;
 
     int32_t* scratch = nullptr;
-    cudaError_t rc = ep::scratch_address(&scratch);
+    const ep_status_t st = ep::scratch_address(&scratch);
+    if (st != EP_OK)
+        return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (rc == cudaSuccess)
-        rc = cudaMemsetAsync(error_word, 0, sizeof(int32_t), s);
+    cudaError_t rc = cudaMemsetAsync(error_word, 0, sizeof(int32_t), s);
     if (rc != cudaSuccess)
-        return EP_ERR_CUDA;
+        return ep::cuda_fail(rc, "ep_layout_static_scratch: clearing the error word");
 
     // A handle on the stack: scratch from the static array, every output
     // from the caller.  Nothing in the scratch needs to start at zero: the
@@ -120,5 +122,5 @@ extern "C" ep_status_t ep_layout_static_scratch(
     h.has_layout = 1;
     h.err_cleared = 1;
     rc = ep::launch_layout(h, topk_idx, T, s, /*allow_fused=*/false);
-    return rc == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    return rc == cudaSuccess ? EP_OK : ep::cuda_fail(rc, "ep_layout_static_scratch");
 }

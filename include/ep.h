@@ -445,10 +445,10 @@ ep_status_t ep_handle_check(ep_handle_t h, void* stream);
  * Dispatch layout without any caller-provided workspace.
  *
  * The pages have no counterpart of this call; it exists for callers that
- * cannot allocate device memory: code running while a CUDA graph is being
- * captured, processes whose device memory is owned up front by a framework
- * allocator or a pre-reserved pool that forbids more cudaMalloc calls, and
- * plug-ins that are handed only input and output pointers.
+ * cannot allocate device memory: processes whose device memory is owned up
+ * front by a framework allocator or a pre-reserved pool that forbids more
+ * cudaMalloc calls, and plug-ins that are handed only input and output
+ * pointers.
  *
  * It computes exactly what ep_layout computes, into caller-provided output
  * arrays, with the same kernels.  Its only scratch (4 bytes x ceil(T/32) x
@@ -461,7 +461,9 @@ ep_status_t ep_handle_check(ep_handle_t h, void* stream);
  *     return EP_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture.
+ *     stream capture.  Devices with an ordinal above 63 are refused
+ *     (EP_ERR_INVALID_ARG); CUDA failures return EP_ERR_CUDA with the
+ *     message in ep_last_error_message.
  *   - Every call shares the one array per device and it keeps the last
  *     call's contents (nothing in it needs to start at zero).  Calls that
  *     overlap on the GPU -- on different streams without ordering, or from

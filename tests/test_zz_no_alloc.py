@@ -1,16 +1,19 @@
 """ep_layout_static_scratch: the dispatch layout for callers that cannot
-allocate device memory (graph capture, a pre-reserved memory pool, plug-ins
-that receive only input and output pointers).  It keeps its scratch in a
-fixed array inside the library, so the caller passes nothing but inputs and
-outputs.
+allocate device memory (a framework or pre-reserved memory pool that forbids
+more cudaMalloc calls, plug-ins that receive only input and output pointers).
+It keeps its scratch in a fixed array inside the library, so the caller passes
+nothing but inputs and outputs.
 
-Checked here through the C ABI: two calls in a row (the array keeps the first
-call's contents when the second runs) must give exactly what the workspace
-entry point ep_layout gives on the same input -- the layout is integer work,
-so the tolerance is bit-exact, as in the other layout tests.  Sizes beyond the
-fixed scratch are rejected before anything is enqueued.  This file runs last
-so that a failure here leaves every other test already run; it also passes
-when run alone in a fresh process (the first call does the per-device set-up).
+Checked here through the C ABI, bit-exact (the layout is integer work, as in
+the other layout tests): every output field against the oracle, and two calls
+in a row (the array keeps the first call's contents when the second runs)
+against the workspace entry point ep_layout on the same input.  The cases
+cover each kernel path the entry point can take: the three-kernel path (large
+batches, and E = 8192), the one-CTA small-batch kernel, and the empty batch.
+Sizes beyond the fixed scratch are rejected before anything is enqueued.  This
+file runs last so that a failure here leaves every other test already run; it
+also passes when run alone in a fresh process (the first call does the
+per-device set-up).
 """
 import ctypes
 
@@ -96,24 +99,66 @@ def _same(a, b):
         assert np.array_equal(a[key], b[key]), key
 
 
-def test_two_calls_in_a_row_match_the_workspace_entry_point():
+def _same_as_oracle(a, lay):
+    """Every output field against the oracle's layout of the same input."""
+    for key in ("num_tokens_per_expert", "num_tokens_per_rank", "num_rows_per_rank",
+                "expert_off", "rank_off", "is_token_in_rank", "dst_row", "recv_src"):
+        exp = getattr(lay, key)
+        assert a[key].shape == exp.shape, (key, a[key].shape, exp.shape)
+        assert np.array_equal(a[key], exp), key
+    assert int(a["total"][0]) == lay.total_rows
+
+
+def test_two_calls_in_a_row_match_the_workspace_entry_point(oracle):
     lib = _lib()
     w1 = make_workload("8k", 0, H=128)                      # 8192 tokens, 8 ranks
     w2 = make_workload("skewed", 0, T=3000, H=128)          # fewer tokens, 32 ranks
     a1 = static_layout(lib, w1.topk_idx, w1.E, w1.R)
     a2 = static_layout(lib, w2.topk_idx, w2.E, w2.R)        # reuses the array
     assert a1["err"][0] == 0 and a2["err"][0] == 0
+    _same_as_oracle(a1, oracle.layout(w1.topk_idx, w1.E, w1.R))
+    _same_as_oracle(a2, oracle.layout(w2.topk_idx, w2.E, w2.R))
     _same(a1, workspace_layout(w1.topk_idx, w1.E, w1.R))
     _same(a2, workspace_layout(w2.topk_idx, w2.E, w2.R))
 
 
-def test_bad_index_sets_the_error_word():
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_small_batches_match_the_oracle(oracle, name):
+    """T k <= 4096: the one-CTA small-batch kernel, no bad index."""
+    lib = _lib()
+    w = make_workload(name, 0, H=128)
+    a = static_layout(lib, w.topk_idx, w.E, w.R)
+    assert a["err"][0] == 0
+    _same_as_oracle(a, oracle.layout(w.topk_idx, w.E, w.R))
+    _same(a, workspace_layout(w.topk_idx, w.E, w.R))
+
+
+def test_largest_expert_count_matches_the_oracle(oracle):
+    """E = 8192: the three-kernel path with a wide count matrix that still fits
+    the static array (4 * ceil(2000/32) * (8192 + 8) bytes)."""
+    lib = _lib()
+    idx, _ = random_topk(2000, 8192, 8, np.random.default_rng(11), p_unused=0.05)
+    a = static_layout(lib, idx, 8192, 8)
+    assert a["err"][0] == 0
+    _same_as_oracle(a, oracle.layout(idx, 8192, 8))
+
+
+def test_empty_batch_matches_the_oracle(oracle):
+    lib = _lib()
+    idx = np.zeros((0, 8), np.int64)
+    a = static_layout(lib, idx, 256, 8)
+    assert a["err"][0] == 0 and int(a["total"][0]) == 0
+    _same_as_oracle(a, oracle.layout(idx, 256, 8))
+
+
+def test_bad_index_sets_the_error_word(oracle):
     lib = _lib()
     idx, _ = random_topk(100, 64, 4, np.random.default_rng(2))
     idx[7, 2] = 64
     a = static_layout(lib, idx, 64, 8)
     assert a["err"][0] == 1  # the bad-index bit
-    idx[7, 2] = -1
+    idx[7, 2] = -1                                          # a bad index counts as unused
+    _same_as_oracle(a, oracle.layout(idx, 64, 8))
     _same(a, workspace_layout(idx, 64, 8))
 
 
