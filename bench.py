@@ -581,6 +581,116 @@ def time_backward(dev, flush, seed, steps):
     return res
 
 
+# ----------------------------------------------------------------- expert parallel
+
+def run_ep(args, rank, world, dev, flush, barrier, peak, peak_src):
+    """--ep: expert parallelism over the N ranks.  Every rank owns the 8k
+    workload's tokens (weak scaling: N x 8192 tokens in all) and rank p holds
+    experts [p E/N, (p+1) E/N).  A step: all-gather of the top-k indices,
+    the global layout, ep_dispatch_ranks of this rank's tokens into every
+    rank's receive buffer (peer buffers mapped with CUDA IPC), stream
+    synchronise + barrier, ep_combine_ranks of this rank's tokens from every
+    rank's expert outputs, stream synchronise + barrier.  The expert outputs
+    come from the stand-in expert op once, before timing.  Device time per
+    step with events, the max over ranks; value = all ranks' dispatch +
+    combine bytes / that time."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from workloads import expert_scale_table, make_workload
+
+    w = make_workload(MAIN_WORKLOAD, args.seed + rank)
+    x = torch.from_numpy(w.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.from_numpy(w.topk_idx).to(dev)
+    wt = torch.from_numpy(w.topk_weights).to(dev)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+
+    def gather():
+        if world == 1:
+            return idx, 0
+        return ep.ep_allgather_topk(idx)
+
+    glob, t0 = gather()
+    h = ep.ep_handle_create(glob.shape[0], w.k, w.E, world, w.block_m, device=dev)
+    ep.ep_layout(h, glob)
+    roff = ep.ep_handle_view(h, "rank_off").cpu().tolist()
+    rows = roff[rank + 1] - roff[rank]
+    recv = torch.empty((max(rows, 1), w.H), dtype=torch.bfloat16, device=dev)
+    y = torch.zeros_like(recv)
+    shares = []
+
+    def table(t):
+        if world == 1:
+            return [t]
+        sh = ep.ep_ipc_share([t])
+        shares.append(sh)
+        return [sh.tensors[p][0] for p in range(world)]
+
+    recv_tab = table(recv)
+    ep.ep_dispatch_ranks(h, t0, x, "bf16", recv_tab)
+    torch.cuda.synchronize()
+    barrier()
+    if rows:  # stand-in expert op on this rank's rows, once
+        eoff = ep.ep_handle_view(h, "expert_off")
+        e = torch.searchsorted(eoff[1:].contiguous(), torch.arange(rows, device=dev) + roff[rank],
+                               right=True)
+        c = torch.from_numpy(expert_scale_table(w.E)).to(dev)[e].unsqueeze(1)
+        y[:rows] = (recv[:rows].float() * c).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    y_tab = table(y)
+    barrier()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        g, _ = gather()
+        ep.ep_layout(h, g)
+        ep.ep_dispatch_ranks(h, t0, x, "bf16", recv_tab)
+        if ev is not None:
+            ev[1].record()
+        torch.cuda.synchronize()
+        barrier()
+        ep.ep_combine_ranks(h, t0, y_tab, wt, out)
+        if ev is not None:
+            ev[2].record()
+        torch.cuda.synchronize()
+        barrier()
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush()
+        step(evs[i])
+    torch.cuda.synchronize()
+    step_ms = aggregate_max(statistics.mean(e[0].elapsed_time(e[2]) for e in evs))
+    dis_ms = aggregate_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+    com_ms = aggregate_max(statistics.mean(e[1].elapsed_time(e[2]) for e in evs))
+    ep.ep_handle_check(h)
+    for sh in shares:
+        sh.close()
+    d_bytes, c_bytes = algo_bytes(w.T, w.H, w.k, w.fmt)
+    value = world * (d_bytes + c_bytes) / (step_ms / 1e3) / 1e9
+    if rank == 0:
+        cfg = workload_config(w, world)
+        cfg["virtual_ranks"] = world
+        cfg["parallelism"] = ("expert parallel over %d rank%s (one per GPU): %d experts each, "
+                              "rows exchanged through CUDA IPC peer buffers"
+                              % (world, "" if world == 1 else "s", w.E // world))
+        line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "kernels": {"gather_layout_dispatch_us": round(dis_ms * 1e3, 2),
+                            "combine_us": round(com_ms * 1e3, 2),
+                            "note": "each phase ends with a stream synchronise and a barrier "
+                                    "across the ranks (host-side ordering)"},
+                "peak": {"hbm_GBps": peak, "source": peak_src},
+                "gpu_launches": 3 * args.steps}
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------- CPU arm
 
 def oracle_sample(w, tokens):
@@ -759,6 +869,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--nvtx", action="store_true",
                     help="NVTX ranges around the three calls (for a profiler's timeline)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the N ranks (rows exchanged through CUDA IPC "
+                         "peer buffers) instead of N independent replicas")
     args = ap.parse_args()
     global NVTX
     NVTX = args.nvtx
@@ -798,6 +911,12 @@ def main():
         flush_buf.zero_()
 
     peak, peak_src = load_peaks()
+    if args.ep:
+        run_ep(args, rank, world, dev, flush, barrier, peak, peak_src)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     s = gpu_setup(MAIN_WORKLOAD, args.seed + rank, dev)
     w = s["w"]
     routing_main = s["routing"]

@@ -38,6 +38,7 @@ __all__ = [
     "ep_dispatch_range", "ep_combine_range", "ep_dispatch_backward", "ep_combine_backward",
     "ep_dispatch_weights", "ep_zero_pad_rows", "ep_dispatch_ranks", "ep_combine_ranks",
     "ep_dispatch_ranks_backward", "ep_combine_ranks_backward", "ep_allgather_topk",
+    "ep_ipc_export", "ep_ipc_open", "ep_ipc_close", "ep_ipc_share", "IPCShare",
     "ep_handle_check", "ep_strerror", "library_path", "load_library",
     "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_ALIGNMENT", "EP_ERR_WORKSPACE_TOO_SMALL",
     "EP_ERR_CAPACITY", "EP_ERR_BAD_INDEX", "EP_ERR_CUDA", "EP_ERR_STATE", "EP_ERR_NO_MEMORY",
@@ -141,6 +142,9 @@ def load_library():
             "ep_combine_backward": ([P, P, P, I64, P, I, P, I64, P, P], I),
             "ep_combine_range": ([P, I, I, P, I64, P, I, P, P], I),
             "ep_handle_check": ([P, P], I),
+            "ep_ipc_export": ([P, P, ctypes.POINTER(ctypes.c_uint64)], I),
+            "ep_ipc_open": ([P, ctypes.c_uint64, ctypes.POINTER(P), ctypes.POINTER(P)], I),
+            "ep_ipc_close": ([P], I),
             "ep_strerror": ([I], ctypes.c_char_p),
             "ep_last_error_message": ([], ctypes.c_char_p),
         }
@@ -642,6 +646,102 @@ def ep_allgather_topk(topk_idx: torch.Tensor, group=None):
     dist.all_gather(parts, pad, group=group)
     glob = torch.cat([parts[r][:counts[r]] for r in range(world)], dim=0).contiguous()
     return glob, sum(counts[:me])
+
+
+EP_IPC_HANDLE_BYTES = 64
+
+
+def ep_ipc_export(t: torch.Tensor):
+    """(handle bytes, offset) of a CUDA tensor's memory, for another process's
+    ep_ipc_open (the tensor must come from a cudaMalloc allocation, as the
+    default caching allocator's are)."""
+    if t.device.type != "cuda" or t.numel() == 0:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_ipc_export: a non-empty CUDA tensor")
+    buf = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    with torch.cuda.device(t.device):
+        _check(load_library().ep_ipc_export(t.data_ptr(), buf, ctypes.byref(off)), "ep_ipc_export")
+    return bytes(buf.raw), int(off.value)
+
+
+def ep_ipc_open(handle: bytes, offset: int):
+    """Open another process's exported handle on the current device; returns
+    (base, ptr) as integers: base for ep_ipc_close, ptr = base + offset."""
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise EPError(EP_ERR_INVALID_ARG, "ep_ipc_open: handle of %d bytes" % EP_IPC_HANDLE_BYTES)
+    base, ptr = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(load_library().ep_ipc_open(handle, offset, ctypes.byref(base), ctypes.byref(ptr)),
+           "ep_ipc_open")
+    return int(base.value), int(ptr.value)
+
+
+def ep_ipc_close(base: int) -> None:
+    _check(load_library().ep_ipc_close(base), "ep_ipc_close")
+
+
+_CAI_TYPE = {torch.bfloat16: ("<i2", torch.bfloat16), torch.float16: ("<f2", torch.float16),
+             torch.float32: ("<f4", torch.float32), torch.int32: ("<i4", torch.int32),
+             torch.int64: ("<i8", torch.int64), torch.uint8: ("|u1", torch.uint8),
+             torch.float8_e4m3fn: ("|u1", torch.float8_e4m3fn)}
+
+
+class _DeviceArray:
+    """A raw device pointer seen by torch.as_tensor (no copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"data": (ptr, False), "shape": tuple(shape),
+                                         "typestr": typestr, "strides": None, "version": 3}
+
+
+class IPCShare:
+    """Every rank's buffers, opened in this process: tensors[r][i] is rank r's
+    i-th shared tensor (this rank's own tensors as given, the others' as views
+    of their IPC mappings).  close() unmaps the peers' allocations; the views
+    must not be used after it."""
+
+    def __init__(self, tensors, bases):
+        self.tensors = tensors
+        self._bases = bases
+
+    def close(self) -> None:
+        for base in self._bases:
+            ep_ipc_close(base)
+        self._bases = []
+
+
+def ep_ipc_share(local: list, group=None) -> IPCShare:
+    """Share this rank's CUDA tensors with the other ranks of a process group
+    and open theirs: an all-gather of (handle, offset, shape, dtype) over the
+    group, then ep_ipc_open of each peer allocation once (tensors that share
+    an allocation share its mapping).  Every rank passes the same number of
+    tensors.  The writes to and reads from the views need the caller's own
+    ordering across ranks (stream synchronise, then a barrier)."""
+    import torch.distributed as dist
+
+    for t in local:
+        if t.dtype not in _CAI_TYPE or not t.is_contiguous() or t.device.type != "cuda":
+            raise EPError(EP_ERR_INVALID_ARG, "ep_ipc_share: contiguous CUDA tensors")
+    mine = [ep_ipc_export(t) + (tuple(t.shape), str(t.dtype)) for t in local]
+    world = dist.get_world_size(group)
+    me = dist.get_rank(group)
+    every = [None] * world
+    dist.all_gather_object(every, mine, group=group)
+    names = {str(dt): dt for dt in _CAI_TYPE}
+    opened = {}
+    tensors = []
+    for r in range(world):
+        if r == me:
+            tensors.append(list(local))
+            continue
+        views = []
+        for handle, offset, shape, dname in every[r]:
+            if handle not in opened:
+                opened[handle] = ep_ipc_open(handle, 0)[0]
+            typestr, dt = _CAI_TYPE[names[dname]]
+            arr = _DeviceArray(opened[handle] + offset, shape, typestr)
+            views.append(torch.as_tensor(arr).view(dt))  # the device of the mapping: no copy
+        tensors.append(views)
+    return IPCShare(tensors, list(opened.values()))
 
 
 def ep_dispatch_backward(h: EPHandle, grad_recv: torch.Tensor,

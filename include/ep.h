@@ -349,6 +349,36 @@ ep_status_t ep_combine_ranks(ep_handle_t h, int t_begin, int t_count, const void
                              const int64_t* y_rows, const float* topk_weights_rows, int H,
                              ep_dtype_t dtype, void* out_rows, void* stream);
 
+/* Mapping another process's buffer into this one (CUDA IPC), to fill the
+ * rank tables above when the ranks are separate processes (one per GPU, or
+ * several on one GPU).  The owner calls ep_ipc_export on a buffer; the
+ * handle bytes and the offset travel to the other ranks by any means (the
+ * Python binding all-gathers them over the process group); each of them
+ * calls ep_ipc_open and puts *ptr into its table.  Host-side ordering is the
+ * caller's: the writes of every rank's ep_dispatch_ranks must be finished
+ * (stream synchronised, then a barrier across the ranks) before any rank
+ * reads its receive buffer, and likewise around the expert outputs that
+ * ep_combine_ranks reads.  The pages' dispatch and combine are this
+ * exchange between GPUs ("DeepEP是什麼？…", section MoE為什麼需要All-to-all).
+ *
+ * ep_ipc_export: ptr is a device pointer inside an allocation made with
+ *   cudaMalloc (not a pool or virtual-memory allocation); handle receives
+ *   EP_IPC_HANDLE_BYTES bytes (host), *offset (host) the distance of ptr
+ *   from the start of its allocation.  A pointer outside any device
+ *   allocation returns EP_ERR_INVALID_ARG.
+ * ep_ipc_open: opens a handle exported by another process (CUDA allows no
+ *   process to open its own); *base (host) receives the mapping of the
+ *   whole allocation, to be passed to ep_ipc_close, and *ptr (host) = base +
+ *   offset.  One handle is opened once per process; buffers that share an
+ *   allocation share its mapping.
+ * ep_ipc_close: unmaps a base returned by ep_ipc_open.
+ * CUDA failures return EP_ERR_CUDA with the message in
+ * ep_last_error_message.  These calls enqueue nothing. */
+#define EP_IPC_HANDLE_BYTES 64
+ep_status_t ep_ipc_export(const void* ptr, void* handle, uint64_t* offset);
+ep_status_t ep_ipc_open(const void* handle, uint64_t offset, void** base, void** ptr);
+ep_status_t ep_ipc_close(void* base);
+
 /* Backward of the two calls above, for the source's tokens [t_begin,
  * t_begin + t_count) of the global layout (rows bf16 or fp16 as dtype).
  * ep_dispatch_ranks_backward: grad_x_rows[t] = the fp32 sum, in slot order,
