@@ -235,3 +235,28 @@ def test_binding_constants_match_the_header():
     assert enums["EP_FMT_FP16"] == ep._FMTS["fp16"]
     assert defines["EP_MAX_RANK_TABLE"] >= 8
     assert set(ep._DTYPES.values()) == {enums["EP_DTYPE_BF16"], enums["EP_DTYPE_FP16"]}
+
+
+def test_ipc_calls_reject_bad_arguments_without_a_gpu(lib):
+    """The IPC mapping calls refuse null pointers before any CUDA call, and the
+    binding's constant and checks mirror the header."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from combine_ep_layout_08_b200 import EP_ERR_INVALID_ARG
+
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    m = re.search(r"#define\s+EP_IPC_HANDLE_BYTES\s+(\d+)", src)
+    assert m and int(m.group(1)) == ep.EP_IPC_HANDLE_BYTES == 64
+    P = ctypes.c_void_p
+    off = ctypes.c_uint64(0)
+    buf = ctypes.create_string_buffer(64)
+    assert lib.ep_ipc_export(None, buf, ctypes.byref(off)) == EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_export(P(0x7f0000000000), None, ctypes.byref(off)) == EP_ERR_INVALID_ARG
+    base, ptr = P(), P()
+    assert lib.ep_ipc_open(None, 0, ctypes.byref(base), ctypes.byref(ptr)) == EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_close(None) == EP_ERR_INVALID_ARG
+    with pytest.raises(ep.EPError):
+        ep.ep_ipc_export(torch.zeros(4))                  # host memory
+    with pytest.raises(ep.EPError):
+        ep.ep_ipc_open(b"too short", 0)
