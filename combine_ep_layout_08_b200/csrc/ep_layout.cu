@@ -853,6 +853,278 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
     }
 }
 
+// Decode batches (T <= SMs, E <= 512, within the small-batch limits): layout
+// and dispatch in one launch with one CTA per token.  A CTA needs the expert
+// totals of the whole batch (for the padded offsets) but the positions of its
+// own token's k slots only: slot (t, j) of expert e goes to row
+// off[e] + #{entries before t k + j with expert e}, counted with one
+// warp-wide sum per slot over the batch's entries, instead of the full
+// per-warp grouping the other small kernel does in every CTA.  The CTA's
+// 32 warps work in two groups that meet at block barriers 1 and 5 only:
+//   layout warps 0-15 (named barrier 1):
+//     1  entries loaded (up to kR per thread) and the token's experts
+//        published (after the counters were zeroed, before the
+//        dependent-launch wait);
+//     2  histogram (shared atomics: order-free sums) and, per slot, each
+//        warp's count of equal experts before it (four slots per warp-wide
+//        sum, in 8-bit fields);
+//     3  padded and plain exclusive scans over the experts (thread e = expert e);
+//     4  the token's positions (warp w sums the counts of slots w, w + 16),
+//        is_token_in_rank, the pad rows of the experts this CTA owns, and
+//        (the last CTA) the totals and offsets;
+//   dispatch warps 16-31 (named barrier 2): warp 16 + p loads 512-channel
+//     piece p of the token's row before the layout starts and quantises it
+//     (FP8) while the layout warps work; meanwhile CTA c counts the tokens on
+//     rank c (c + G, ...): the entries that are their token's first slot on
+//     that rank;
+//   5  (block) the rows stored to the k positions.
+// Dynamic shared memory: ent[T k] (the entries, for the first-slot test).
+constexpr int kDecLayoutWarps = 16;
+constexpr int kDecThreads = 32 * kDecLayoutWarps;  // threads of each group
+constexpr int kDecMaxE = kDecThreads;               // one expert per layout thread
+
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// The whole block at barrier 0 from code paths that differ between the warp
+// groups (the non-aligned form: the groups reach it at different instructions).
+__device__ __forceinline__ void block_sync_unaligned()
+{
+    asm volatile("barrier.sync 0;" ::: "memory");
+}
+
+// Number of threads of the named barrier's group whose predicate is true.
+__device__ __forceinline__ int named_count(int id, int nthreads, bool pred)
+{
+    int n;
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.popc.u32 %0, %2, %3, p;\n\t}"
+                 : "=r"(n)
+                 : "r"((unsigned)pred), "r"(id), "r"(nthreads)
+                 : "memory");
+    return n;
+}
+
+template <int kR>
+__global__ void __launch_bounds__(kSmallThreads)
+decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, int R,
+                              int epr, uint64_t rank_magic, int block_m, int bm_log, int k_log,
+                              int32_t* __restrict__ cnt_g, int32_t* __restrict__ expert_off_g,
+                              int32_t* __restrict__ rank_off_g,
+                              int32_t* __restrict__ tokens_per_rank_g,
+                              int32_t* __restrict__ rows_per_rank_g,
+                              int32_t* __restrict__ total_rows_g,
+                              uint8_t* __restrict__ is_token_in_rank,
+                              int32_t* __restrict__ dst_row, int32_t* __restrict__ recv_src,
+                              int32_t* err, FusedDispatch fd)
+{
+    extern __shared__ __align__(16) int32_t ent[];  // [T k]
+    __shared__ int32_t cnt[kDecMaxE];
+    __shared__ int32_t off[kDecMaxE + 1], uoff[kDecMaxE + 1];
+    __shared__ int32_t wsum[2][kDecLayoutWarps];
+    __shared__ int32_t part[32][EP_MAX_TOPK];  // rows 0..15 used
+    __shared__ int32_t tgt_e[EP_MAX_TOPK], tgt_pos[EP_MAX_TOPK];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool layout_group = warp < kDecLayoutWarps;
+    const int t = blockIdx.x;
+    const bool leader = blockIdx.x == gridDim.x - 1;  // writes the totals and offsets
+    const int nent = T * k;
+    auto padded = [&](int32_t c) {
+        return bm_log >= 0 ? ((c + block_m - 1) >> bm_log) << bm_log : pad_up(c, block_m);
+    };
+    const int64_t vpr = fd.H / 16;
+    const int64_t upr = (vpr + 31) / 32;  // 512-channel pieces of the row
+    const int piece = warp - kDecLayoutWarps;
+
+    // 1
+    if (layout_group)
+        for (int e = tid; e < E; e += kDecThreads) cnt[e] = 0;
+    pdl_wait();
+    pdl_trigger();
+    units::Vec32 cur[1];
+    int e_r[kR];
+    if (!layout_group) {
+        if (piece < upr)
+            units::fp8_load<1>(static_cast<const units::Vec32*>(fd.x) + (int64_t)t * vpr, vpr,
+                               piece, cur);
+    } else {
+        int bad = 0;
+#pragma unroll
+        for (int q = 0; q < kR; ++q) {
+            const int f = q * kDecThreads + tid;
+            e_r[q] = f < nent ? to_expert(topk_idx[f], E, bad) : -1;
+            if (f < nent) {
+                ent[f] = e_r[q];
+                if (f >= t * k && f < t * k + k)
+                    tgt_e[f - t * k] = e_r[q];
+            }
+        }
+        if (__any_sync(kFull, bad) && lane == 0 && leader)
+            atomicOr(err, kErrBadIndex);
+    }
+    __syncthreads();
+
+    if (layout_group) {
+        // 2
+#pragma unroll
+        for (int q = 0; q < kR; ++q)
+            if (e_r[q] >= 0)
+                atomicAdd(&cnt[e_r[q]], 1);
+        // four slots per warp-wide sum in 8-bit fields: a warp counts at most
+        // 32 kR <= 224 entries per slot (the host keeps kR <= 7)
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            uint32_t c = 0;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = j0 + jj;
+                if (j < k) {
+                    const int ej = tgt_e[j], fj = t * k + j;
+#pragma unroll
+                    for (int q = 0; q < kR; ++q)
+                        c += (e_r[q] == ej && q * kDecThreads + tid < fj) ? (1u << (8 * jj)) : 0u;
+                }
+            }
+            c = __reduce_add_sync(kFull, c);
+            if (lane < 4 && j0 + lane < k)
+                part[warp][j0 + lane] = (int32_t)((c >> (8 * lane)) & 0xffu);
+        }
+        named_sync(1, kDecThreads);
+
+        // 3: thread e owns expert e
+        const int32_t c_e = tid < E ? cnt[tid] : 0, p_e = padded(c_e);
+        int32_t pin = p_e, uin = c_e;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t a = __shfl_up_sync(kFull, pin, o), b = __shfl_up_sync(kFull, uin, o);
+            if (lane >= o) {
+                pin += a;
+                uin += b;
+            }
+        }
+        if (lane == 31) {
+            wsum[0][warp] = pin;
+            wsum[1][warp] = uin;
+        }
+        named_sync(1, kDecThreads);
+        {
+            const int32_t v = lane < kDecLayoutWarps ? wsum[0][lane] : 0;
+            const int32_t v2 = lane < kDecLayoutWarps ? wsum[1][lane] : 0;
+            int32_t inc = v, inc2 = v2;
+            for (int o = 1; o < kDecLayoutWarps; o <<= 1) {
+                const int32_t a = __shfl_up_sync(kFull, inc, o), b = __shfl_up_sync(kFull, inc2, o);
+                if (lane >= o) {
+                    inc += a;
+                    inc2 += b;
+                }
+            }
+            const int32_t base = __shfl_sync(kFull, inc - v, warp);
+            const int32_t base2 = __shfl_sync(kFull, inc2 - v2, warp);
+            if (tid < E) {
+                off[tid] = base + pin - p_e;
+                uoff[tid] = base2 + uin - c_e;
+                if (tid == E - 1) {
+                    off[E] = base + pin;
+                    uoff[E] = base2 + uin;
+                }
+            }
+        }
+        named_sync(1, kDecThreads);
+
+        // 4
+        for (int j = warp; j < k; j += kDecLayoutWarps) {  // warp w: slots w, w + 16
+            const int e = tgt_e[j];
+            const int32_t c = __reduce_add_sync(kFull, lane < kDecLayoutWarps ? part[lane][j] : 0);
+            if (lane == 0) {
+                const int32_t pos = e >= 0 ? off[e] + c : -1;
+                tgt_pos[j] = pos;
+                dst_row[(int64_t)t * k + j] = pos;
+                if (pos >= 0)
+                    recv_src[pos] = t;
+            }
+        }
+        for (int r = tid; r < R; r += kDecThreads) {
+            uint8_t hit = 0;
+            for (int j = 0; j < k; ++j)
+                hit |= (tgt_e[j] >= 0 && (int)(((uint64_t)tgt_e[j] * rank_magic) >> 32) == r);
+            is_token_in_rank[(int64_t)t * R + r] = hit;
+        }
+        const bool vec = ((uintptr_t)recv_src & 15u) == 0;
+        for (int e = blockIdx.x + warp * (int)gridDim.x; e < E; e += (int)gridDim.x * kDecLayoutWarps)
+            fill_pad(recv_src, off[e] + cnt[e], off[e + 1], vec);
+        if (leader) {
+            for (int e = tid; e < E; e += kDecThreads) cnt_g[e] = cnt[e];
+            for (int e = tid; e <= E; e += kDecThreads) expert_off_g[e] = off[e];
+            for (int r = tid; r <= R; r += kDecThreads) rank_off_g[r] = off[r * epr];
+            for (int r = tid; r < R; r += kDecThreads)
+                rows_per_rank_g[r] = uoff[(r + 1) * epr] - uoff[r * epr];
+            if (tid == 0)
+                *total_rows_g = off[E];
+        }
+    } else {
+        // the dispatch group: codes of its piece, then the tokens per rank
+        const int dt = tid - kDecThreads;
+        uint4 q8[1];
+        float my_scale = 0.0f;
+        if (fd.fp8 && piece < upr)
+            units::fp8_quantize<1>(cur, q8, my_scale);
+        for (int r = blockIdx.x; r < R; r += (int)gridDim.x) {  // uniform over the group
+            int32_t n = 0;
+            for (int f0 = 0; f0 < nent; f0 += kDecThreads) {
+                const int f = f0 + dt;
+                bool first = false;
+                if (f < nent) {
+                    const int e = ent[f];
+                    if (e >= 0 && (int)(((uint64_t)e * rank_magic) >> 32) == r) {
+                        const int tok = k_log >= 0 ? f >> k_log : f / k;
+                        first = true;
+                        for (int g = tok * k; g < f; ++g)
+                            first &= ent[g] < 0 || (int)(((uint64_t)ent[g] * rank_magic) >> 32) != r;
+                    }
+                }
+                n += named_count(2, kDecThreads, first);
+            }
+            if (dt == 0)
+                tokens_per_rank_g[r] = n;
+        }
+        block_sync_unaligned();  // 5: the positions are in shared memory
+
+        if (piece < upr) {
+            int d = lane < k ? tgt_pos[lane] : -1;
+            if (d >= fd.cap_rows) {
+                atomicOr(err, kErrDispatchCap);
+                d = -1;
+            }
+            const int64_t v = (int64_t)piece * 32 + lane;
+            if (fd.fp8) {
+                const int nblk = fd.H / 128;
+                const int64_t blk = (int64_t)piece * 4 + lane;
+                const bool sc_ok = lane < 4 && blk < nblk;
+                uint8_t* rq = static_cast<uint8_t*>(fd.recv_x);
+                for (int j0 = 0; j0 < k; j0 += 8) {  // the rows of 8 slots, then their stores
+                    int dj[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) dj[jj] = __shfl_sync(kFull, d, (j0 + jj) & 31);
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        if (j0 + jj >= k || dj[jj] < 0)
+                            continue;
+                        if (v < vpr)
+                            reinterpret_cast<uint4*>(rq + (int64_t)dj[jj] * fd.H)[v] = q8[0];
+                        if (sc_ok)
+                            fd.recv_scales[units::scale_index(dj[jj], blk, nblk, fd.scales_ld)] =
+                                my_scale;
+                    }
+                }
+            } else {
+                units::bf16_store(cur[0], v, vpr, d, k, static_cast<units::Vec32*>(fd.recv_x));
+            }
+        }
+        return;
+    }
+    block_sync_unaligned();  // 5 (layout group)
+}
+
 // ------------------------------------------------------------------ fused
 // Grid barrier over the CTAs of a cooperative launch (all co-resident).
 // bar[0] is an arrival counter that only grows (32-bit wrap-around, compared
@@ -1420,6 +1692,40 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
                                    int64_t scales_ld, int64_t cap_rows, cudaStream_t s)
 {
     const int k = h.k, E = h.E, R = h.R, epr = h.E / h.R;
+    {
+        // one CTA per token when the batch fits on the SMs once
+        int dev = 0, sms = 0;
+        cudaError_t rc;
+        if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+            (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return rc;
+        const int rounds = (int)(((int64_t)T * k + kDecThreads - 1) / kDecThreads);
+        const size_t dsmem = sizeof(int32_t) * (size_t)T * k;
+        if (T <= sms && E <= kDecMaxE && rounds <= 7 && dsmem <= 64 * 1024 &&
+            (H / 16 + 31) / 32 <= kSmallThreads / 32 - kDecLayoutWarps) {
+            FusedDispatch fd{x, H, fp8 ? 1 : 0, recv_x, recv_scales, scales_ld, cap_rows};
+            auto go = [&](auto kern) {
+                cudaError_t r2 = set_smem((const void*)kern, dsmem);
+                if (r2 != cudaSuccess)
+                    return r2;
+                return launch_pdl(kern, (unsigned)T, kSmallThreads, dsmem, s, topk_idx, T, k, E,
+                                  R, epr, rank_magic_for(epr), h.block_m,
+                                  log2_if_pow2(h.block_m), log2_if_pow2(k), h.cnt, h.expert_off,
+                                  h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
+                                  h.is_token_in_rank, h.dst_row, h.recv_src, h.err, fd);
+            };
+            switch (rounds) {
+            case 0:
+            case 1: return go(decode_layout_dispatch_kernel<1>);
+            case 2: return go(decode_layout_dispatch_kernel<2>);
+            case 3: return go(decode_layout_dispatch_kernel<3>);
+            case 4: return go(decode_layout_dispatch_kernel<4>);
+            case 5: return go(decode_layout_dispatch_kernel<5>);
+            case 6: return go(decode_layout_dispatch_kernel<6>);
+            default: return go(decode_layout_dispatch_kernel<7>);
+            }
+        }
+    }
     const size_t smem = small_smem_bytes(E, R, small_rounds((int64_t)T * k));
     cudaError_t rc;
     const bool one_round = small_rounds((int64_t)T * k) == 1;

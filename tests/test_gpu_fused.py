@@ -66,6 +66,9 @@ def test_fused_configs(oracle, name, seed):
     (130, 7168, 1024, 64, 8, "fp8", 0.0), # E = 1024
     (600, 256, 64, 8, 8, "bf16", 0.0),    # 4800 entries: two launches
     (40, 264, 16, 4, 2, "bf16", 0.0),     # H % 16 != 0: two launches
+    (148, 1024, 256, 16, 8, "fp8", 0.05), # one CTA per token on every SM
+    (60, 512, 64, 8, 32, "bf16", 0.1),    # k = 32 slots per token
+    (149, 1024, 256, 16, 8, "bf16", 0.0), # one token more than SMs: the replicated layout
 ])
 def test_fused_shapes(oracle, T, H, E, R, k, fmt, p_unused):
     rng = np.random.default_rng(T * 7 + H)
