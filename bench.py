@@ -210,13 +210,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm
 
-def gpu_setup(name, seed, dev):
+def gpu_setup(name, seed, dev, T=None):
     import torch
 
     import combine_ep_layout_08_b200 as ep
     from workloads import make_workload
 
-    w = make_workload(name, seed)
+    w = make_workload(name, seed, T=T)
     h = ep.ep_handle_create(w.T, w.k, w.E, w.R, w.block_m, device=dev)
     x = torch.from_numpy(w.x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
     idx = torch.from_numpy(w.topk_idx).to(dev)
@@ -581,6 +581,48 @@ def time_backward(dev, flush, seed, steps):
     return res
 
 
+# ----------------------------------------------------------------- profiler cases
+
+KERNEL_CASES = {
+    "layout_8k": "ep_layout alone on the 8k routing (8192 tokens, top-8 of 256, 8 ranks): "
+                 "only topk_idx and the workspace are allocated",
+    "decode_fused": "the decode step in its fused form: ep_layout_dispatch (FP8) + ep_combine",
+    "dispatch_2k": "layout + BF16 dispatch + combine on the first 2048 tokens of the 8k workload "
+                   "(a quarter of the 8k launch; inputs and outputs larger than L2)",
+}
+
+
+def run_kernel_case(name, steps, dev):
+    """One small case of a kernel, `steps` times, for a profiler capture."""
+    import torch
+
+    import combine_ep_layout_08_b200 as ep
+    from workloads import make_workload
+
+    if name == "layout_8k":
+        w = make_workload(MAIN_WORKLOAD, 0, H=16)
+        h = ep.ep_handle_create(w.T, w.k, w.E, w.R, w.block_m, device=dev)
+        idx = torch.from_numpy(w.topk_idx).to(dev)
+        for _ in range(steps):
+            ep.ep_layout(h, idx)
+        shape = "T=%d k=%d E=%d R=%d" % (w.T, w.k, w.E, w.R)
+    elif name == "decode_fused":
+        s = gpu_setup("decode", 0, dev)
+        for _ in range(steps):
+            fused_step(s)
+        h, shape = s["h"], "decode: T=%d H=%d E=%d R=%d k=%d fp8" % (s["w"].T, s["w"].H, s["w"].E,
+                                                                   s["w"].R, s["w"].k)
+    else:
+        s = gpu_setup(MAIN_WORKLOAD, 0, dev, T=2048)
+        for _ in range(steps):
+            gpu_step(s)
+        h, shape = s["h"], "T=%d H=%d E=%d R=%d k=%d bf16" % (s["w"].T, s["w"].H, s["w"].E,
+                                                              s["w"].R, s["w"].k)
+    torch.cuda.synchronize()
+    ep.ep_handle_check(h)
+    print("kernel case %s (%s), %d steps: %s" % (name, shape, steps, KERNEL_CASES[name]), flush=True)
+
+
 # ----------------------------------------------------------------- expert parallel
 
 def run_ep(args, rank, world, dev, flush, barrier, peak, peak_src):
@@ -869,6 +911,9 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--nvtx", action="store_true",
                     help="NVTX ranges around the three calls (for a profiler's timeline)")
+    ap.add_argument("--kernel-case", choices=sorted(KERNEL_CASES),
+                    help="run one small case of a kernel --steps times and print its shape (for a "
+                         "profiler; no timing line)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the N ranks (rows exchanged through CUDA IPC "
                          "peer buffers) instead of N independent replicas")
@@ -911,6 +956,9 @@ def main():
         flush_buf.zero_()
 
     peak, peak_src = load_peaks()
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case, args.steps, dev)
+        return
     if args.ep:
         run_ep(args, rank, world, dev, flush, barrier, peak, peak_src)
         if world > 1:
