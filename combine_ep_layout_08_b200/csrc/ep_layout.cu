@@ -860,24 +860,32 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
 // off[e] + #{entries before t k + j with expert e}, counted with one
 // warp-wide sum per slot over the batch's entries, instead of the full
 // per-warp grouping the other small kernel does in every CTA.  The CTA's
-// 32 warps work in two groups that meet at block barriers 1 and 5 only:
+// 32 warps work in two groups that meet at block barrier 1 and at barrier 3:
 //   layout warps 0-15 (named barrier 1):
 //     1  entries loaded (up to kR per thread) and the token's experts
 //        published (after the counters were zeroed, before the
 //        dependent-launch wait);
-//     2  histogram (shared atomics: order-free sums) and, per slot, each
-//        warp's count of equal experts before it (four slots per warp-wide
-//        sum, in 8-bit fields);
+//     2  per slot, each warp's count of equal experts before it (one ballot
+//        per slot and round), and the histogram (shared atomics: order-free
+//        sums);
 //     3  padded and plain exclusive scans over the experts (thread e = expert e);
 //     4  the token's positions (warp w sums the counts of slots w, w + 16),
-//        is_token_in_rank, the pad rows of the experts this CTA owns, and
-//        (the last CTA) the totals and offsets;
+//        released to the dispatch group at once; then is_token_in_rank, the
+//        pad rows of the experts this CTA owns, (the last CTA) the totals and
+//        offsets, and for R > 32 the tokens on rank c (c + G, ...) counted
+//        in CTA c, the entries that are their token's first slot on that
+//        rank;
 //   dispatch warps 16-31 (named barrier 2): warp 16 + p loads 512-channel
 //     piece p of the token's row before the layout starts and quantises it
-//     (FP8) while the layout warps work; meanwhile CTA c counts the tokens on
-//     rank c (c + G, ...): the entries that are their token's first slot on
-//     that rank;
-//   5  (block) the rows stored to the k positions.
+//     (FP8) while the layout warps work; for R <= 32 one CTA's dispatch
+//     group also counts the tokens per rank meanwhile (one rank mask per
+//     token, one ballot per rank);
+//   5  (barrier 3: the layout warps that wrote positions and the dispatch
+//      group) the rows stored to the k positions, while the layout group
+//      finishes the rest of step 4.
+// When T + 1 CTAs fit on the SMs, an extra CTA without a token of its own
+// takes the leader's and the counter's work, so that no token's stores wait
+// for them.
 // Dynamic shared memory: ent[T k] (the entries, for the first-slot test).
 constexpr int kDecLayoutWarps = 16;
 constexpr int kDecThreads = 32 * kDecLayoutWarps;  // threads of each group
@@ -888,12 +896,14 @@ __device__ __forceinline__ void named_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// The whole block at barrier 0 from code paths that differ between the warp
-// groups (the non-aligned form: the groups reach it at different instructions).
-__device__ __forceinline__ void block_sync_unaligned()
+// The same from code paths that differ between the warps taking part (the
+// non-aligned form: they reach it at different instructions).
+__device__ __forceinline__ void named_sync_unaligned(int id, int nthreads)
 {
-    asm volatile("barrier.sync 0;" ::: "memory");
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+
 
 // Number of threads of the named barrier's group whose predicate is true.
 __device__ __forceinline__ int named_count(int id, int nthreads, bool pred)
@@ -925,11 +935,17 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
     __shared__ int32_t off[kDecMaxE + 1], uoff[kDecMaxE + 1];
     __shared__ int32_t wsum[2][kDecLayoutWarps];
     __shared__ int32_t part[32][EP_MAX_TOPK];  // rows 0..15 used
+    __shared__ int32_t rpart[kDecLayoutWarps][32];  // per-warp tokens per rank (R <= 32)
     __shared__ int32_t tgt_e[EP_MAX_TOPK], tgt_pos[EP_MAX_TOPK];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool layout_group = warp < kDecLayoutWarps;
     const int t = blockIdx.x;
-    const bool leader = blockIdx.x == gridDim.x - 1;  // writes the totals and offsets
+    const bool has_token = t < T;  // else the extra CTA (grid T + 1): no token of its own
+    const bool extra = (int)gridDim.x > T;
+    // the leader writes the totals and offsets; the counter's dispatch group
+    // counts the tokens per rank when R <= 32 (both the extra CTA if there is one)
+    const bool leader = extra ? t == T : t == T - 1;
+    const bool counter = extra ? t == T : t == max(T - 2, 0);
     const int nent = T * k;
     auto padded = [&](int32_t c) {
         return bm_log >= 0 ? ((c + block_m - 1) >> bm_log) << bm_log : pad_up(c, block_m);
@@ -937,6 +953,9 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
     const int64_t vpr = fd.H / 16;
     const int64_t upr = (vpr + 31) / 32;  // 512-channel pieces of the row
     const int piece = warp - kDecLayoutWarps;
+    // barrier 3: the layout warps that write positions, then the dispatch group
+    const int pos_warps = min(k, kDecLayoutWarps);
+    const int release_threads = 32 * (pos_warps + kDecLayoutWarps);
 
     // 1
     if (layout_group)
@@ -946,7 +965,7 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
     units::Vec32 cur[1];
     int e_r[kR];
     if (!layout_group) {
-        if (piece < upr)
+        if (piece < upr && has_token)
             units::fp8_load<1>(static_cast<const units::Vec32*>(fd.x) + (int64_t)t * vpr, vpr,
                                piece, cur);
     } else {
@@ -968,28 +987,36 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
 
     if (layout_group) {
         // 2
+        // The entries are read back from shared memory from here on: the
+        // registers of the global loads would be reloaded from global memory
+        // when the compiler rematerialises them (read-only data), an L2 round
+        // trip per use.
+        int e_s[kR];
+#pragma unroll
+        for (int q = 0; q < kR; ++q) {
+            const int f = q * kDecThreads + tid;
+            e_s[q] = f < nent ? ent[f] : -1;
+        }
+        // per slot and round, one ballot of the warp's equal experts before it;
+        // lane j keeps slot j's count
+        if (has_token) {
+            int32_t mine = 0;
+            for (int j = 0; j < k; ++j) {
+                const int ej = tgt_e[j], fj = t * k + j;
+                int32_t c = 0;
+#pragma unroll
+                for (int q = 0; q < kR; ++q)
+                    c += __popc(__ballot_sync(kFull, e_s[q] == ej && q * kDecThreads + tid < fj));
+                if (lane == (j & 31))
+                    mine = c;
+            }
+            if (lane < k)
+                part[warp][lane] = mine;
+        }
 #pragma unroll
         for (int q = 0; q < kR; ++q)
-            if (e_r[q] >= 0)
-                atomicAdd(&cnt[e_r[q]], 1);
-        // four slots per warp-wide sum in 8-bit fields: a warp counts at most
-        // 32 kR <= 224 entries per slot (the host keeps kR <= 7)
-        for (int j0 = 0; j0 < k; j0 += 4) {
-            uint32_t c = 0;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = j0 + jj;
-                if (j < k) {
-                    const int ej = tgt_e[j], fj = t * k + j;
-#pragma unroll
-                    for (int q = 0; q < kR; ++q)
-                        c += (e_r[q] == ej && q * kDecThreads + tid < fj) ? (1u << (8 * jj)) : 0u;
-                }
-            }
-            c = __reduce_add_sync(kFull, c);
-            if (lane < 4 && j0 + lane < k)
-                part[warp][j0 + lane] = (int32_t)((c >> (8 * lane)) & 0xffu);
-        }
+            if (e_s[q] >= 0)
+                atomicAdd(&cnt[e_s[q]], 1);
         named_sync(1, kDecThreads);
 
         // 3: thread e owns expert e
@@ -1032,18 +1059,21 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
         named_sync(1, kDecThreads);
 
         // 4
-        for (int j = warp; j < k; j += kDecLayoutWarps) {  // warp w: slots w, w + 16
-            const int e = tgt_e[j];
-            const int32_t c = __reduce_add_sync(kFull, lane < kDecLayoutWarps ? part[lane][j] : 0);
-            if (lane == 0) {
-                const int32_t pos = e >= 0 ? off[e] + c : -1;
-                tgt_pos[j] = pos;
-                dst_row[(int64_t)t * k + j] = pos;
-                if (pos >= 0)
-                    recv_src[pos] = t;
+        if (warp < pos_warps && has_token) {
+            for (int j = warp; j < k; j += kDecLayoutWarps) {  // warp w: slots w, w + 16
+                const int e = tgt_e[j];
+                const int32_t c = __reduce_add_sync(kFull, lane < kDecLayoutWarps ? part[lane][j] : 0);
+                if (lane == 0) {
+                    const int32_t pos = e >= 0 ? off[e] + c : -1;
+                    tgt_pos[j] = pos;
+                    dst_row[(int64_t)t * k + j] = pos;
+                    if (pos >= 0)
+                        recv_src[pos] = t;
+                }
             }
+            named_sync_unaligned(3, release_threads);  // the positions are in shared memory
         }
-        for (int r = tid; r < R; r += kDecThreads) {
+        for (int r = tid; r < R && has_token; r += kDecThreads) {
             uint8_t hit = 0;
             for (int j = 0; j < k; ++j)
                 hit |= (tgt_e[j] >= 0 && (int)(((uint64_t)tgt_e[j] * rank_magic) >> 32) == r);
@@ -1061,33 +1091,70 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
             if (tid == 0)
                 *total_rows_g = off[E];
         }
+        // tokens per rank for R > 32: CTA c counts rank c (c + G, ...), the
+        // entries that are their token's first slot on that rank (R <= 32:
+        // the dispatch group of one CTA, below)
+        if (R > 32) {
+            for (int r = blockIdx.x; r < R; r += (int)gridDim.x) {  // uniform over the group
+                int32_t n = 0;
+#pragma unroll
+                for (int q = 0; q < kR; ++q) {
+                    const int f = q * kDecThreads + tid;
+                    bool first = false;
+                    if (f < nent && e_s[q] >= 0 &&
+                        (int)(((uint64_t)e_s[q] * rank_magic) >> 32) == r) {
+                        const int tok = k_log >= 0 ? f >> k_log : f / k;
+                        first = true;
+                        for (int g = tok * k; g < f; ++g)
+                            first &= ent[g] < 0 ||
+                                     (int)(((uint64_t)ent[g] * rank_magic) >> 32) != r;
+                    }
+                    n += named_count(1, kDecThreads, first);
+                }
+                if (tid == 0)
+                    tokens_per_rank_g[r] = n;
+            }
+        }
     } else {
-        // the dispatch group: codes of its piece, then the tokens per rank
-        const int dt = tid - kDecThreads;
+        // the dispatch group: the codes of its piece, then the stores
         uint4 q8[1];
         float my_scale = 0.0f;
         if (fd.fp8 && piece < upr)
             units::fp8_quantize<1>(cur, q8, my_scale);
-        for (int r = blockIdx.x; r < R; r += (int)gridDim.x) {  // uniform over the group
-            int32_t n = 0;
-            for (int f0 = 0; f0 < nent; f0 += kDecThreads) {
-                const int f = f0 + dt;
-                bool first = false;
-                if (f < nent) {
-                    const int e = ent[f];
-                    if (e >= 0 && (int)(((uint64_t)e * rank_magic) >> 32) == r) {
-                        const int tok = k_log >= 0 ? f >> k_log : f / k;
-                        first = true;
-                        for (int g = tok * k; g < f; ++g)
-                            first &= ent[g] < 0 || (int)(((uint64_t)ent[g] * rank_magic) >> 32) != r;
+        if (R <= 32 && counter) {
+            // tokens per rank while the positions are computed: thread t
+            // builds token t's rank mask, each warp counts the masks holding
+            // rank r with one ballot per rank
+            const int dw = warp - kDecLayoutWarps;
+            int32_t mine = 0;  // lane r: this warp's tokens on rank r
+            for (int t0 = dw * 32; t0 < T; t0 += kDecThreads) {
+                const int tt = t0 + lane;
+                uint32_t mask = 0;
+                if (tt < T)
+                    for (int j = 0; j < k; ++j) {
+                        const int e = ent[tt * k + j];
+                        if (e >= 0)
+                            mask |= 1u << (int)(((uint64_t)e * rank_magic) >> 32);
                     }
+                for (int r = 0; r < R; ++r) {
+                    const int c = __popc(__ballot_sync(kFull, (mask >> r) & 1u));
+                    if (lane == r)
+                        mine += c;
                 }
-                n += named_count(2, kDecThreads, first);
             }
-            if (dt == 0)
-                tokens_per_rank_g[r] = n;
+            if (lane < R)
+                rpart[dw][lane] = mine;
+            named_sync(2, kDecThreads);
+            const int dt = tid - kDecThreads;
+            if (dt < R) {
+                int32_t n = 0;
+                for (int w = 0; w * 32 < T && w < kDecLayoutWarps; ++w) n += rpart[w][dt];
+                tokens_per_rank_g[dt] = n;
+            }
         }
-        block_sync_unaligned();  // 5: the positions are in shared memory
+        if (!has_token)
+            return;
+        named_sync_unaligned(3, release_threads);  // 5: the positions are in shared memory
 
         if (piece < upr) {
             int d = lane < k ? tgt_pos[lane] : -1;
@@ -1120,9 +1187,7 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
                 units::bf16_store(cur[0], v, vpr, d, k, static_cast<units::Vec32*>(fd.recv_x));
             }
         }
-        return;
     }
-    block_sync_unaligned();  // 5 (layout group)
 }
 
 // ------------------------------------------------------------------ fused
@@ -1701,14 +1766,15 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
             return rc;
         const int rounds = (int)(((int64_t)T * k + kDecThreads - 1) / kDecThreads);
         const size_t dsmem = sizeof(int32_t) * (size_t)T * k;
-        if (T <= sms && E <= kDecMaxE && rounds <= 7 && dsmem <= 64 * 1024 &&
+        if (T <= sms && E <= kDecMaxE && dsmem <= 64 * 1024 &&
             (H / 16 + 31) / 32 <= kSmallThreads / 32 - kDecLayoutWarps) {
             FusedDispatch fd{x, H, fp8 ? 1 : 0, recv_x, recv_scales, scales_ld, cap_rows};
             auto go = [&](auto kern) {
                 cudaError_t r2 = set_smem((const void*)kern, dsmem);
                 if (r2 != cudaSuccess)
                     return r2;
-                return launch_pdl(kern, (unsigned)T, kSmallThreads, dsmem, s, topk_idx, T, k, E,
+                const unsigned grid = (unsigned)(T + 1 <= sms ? T + 1 : T);  // + the extra CTA
+                return launch_pdl(kern, grid, kSmallThreads, dsmem, s, topk_idx, T, k, E,
                                   R, epr, rank_magic_for(epr), h.block_m,
                                   log2_if_pow2(h.block_m), log2_if_pow2(k), h.cnt, h.expert_off,
                                   h.rank_off, h.tokens_per_rank, h.rows_per_rank, h.total_rows,
@@ -1722,7 +1788,8 @@ cudaError_t launch_layout_dispatch(const Handle& h, const int64_t* topk_idx, int
             case 4: return go(decode_layout_dispatch_kernel<4>);
             case 5: return go(decode_layout_dispatch_kernel<5>);
             case 6: return go(decode_layout_dispatch_kernel<6>);
-            default: return go(decode_layout_dispatch_kernel<7>);
+            case 7: return go(decode_layout_dispatch_kernel<7>);
+            default: return go(decode_layout_dispatch_kernel<8>);
             }
         }
     }

@@ -69,6 +69,8 @@ def test_fused_configs(oracle, name, seed):
     (148, 1024, 256, 16, 8, "fp8", 0.05), # one CTA per token on every SM
     (60, 512, 64, 8, 32, "bf16", 0.1),    # k = 32 slots per token
     (149, 1024, 256, 16, 8, "bf16", 0.0), # one token more than SMs: the replicated layout
+    (100, 512, 256, 64, 8, "fp8", 0.1),   # one CTA per token, R > 32 ranks
+    (90, 512, 32, 32, 5, "bf16", 0.0),    # one CTA per token, R = E = 32, k not dividing 32
 ])
 def test_fused_shapes(oracle, T, H, E, R, k, fmt, p_unused):
     rng = np.random.default_rng(T * 7 + H)
