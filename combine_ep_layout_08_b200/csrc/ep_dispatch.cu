@@ -20,7 +20,10 @@
 // batch size tried, 4096 and 8192 tokens.)
 // The main kernels move 32-byte vectors (sm_100's 256-bit ld/st.global.v8),
 // halving the store instructions of 16-byte vectors; 16-byte kernels remain
-// for rows that are not 32-byte multiples.  The grid gives every warp one
+// for rows that are not 32-byte multiples.  Before the dependent-launch wait
+// each warp of the main kernels prefetches its unit of x into L2 (x does not
+// depend on the layout; a prefetch returns no data), so the loads after the
+// wait find it there: measured 1.5 us less per launch at 8192 tokens.  The grid gives every warp one
 // unit (a grid-stride loop covers grids beyond kMaxGrid): measured on B200,
 // a persistent single wave, in which every warp loads and then stores in
 // lock step with all the others, reaches ~5.4 TB/s; two waves 5.8; one unit
@@ -49,12 +52,30 @@ using units::kUnitVec32;
 using units::kUnitVec32Fp8;
 constexpr int64_t kMaxGrid = 1 << 20;
 
+// A hint that brings a line into L2; it reads nothing, so it may be issued
+// before the dependent-launch wait (the data it fetches is never used
+// directly: the loads after the wait see the memory as it is then).
+__device__ __forceinline__ void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // BF16 dispatch with 32-byte vectors; vpr = H / 16.
 __global__ void __launch_bounds__(kThreads, 8)
 dispatch_bf16_v32_kernel(const Vec32* __restrict__ x, int T, int k, int64_t vpr,
                          const int32_t* __restrict__ dst_row, Vec32* __restrict__ recv,
                          int64_t cap_rows, int32_t* err)
 {
+    {   // this warp's first unit of x into L2 while the previous kernel finishes
+        const int64_t wg0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+        const int64_t upr0 = (vpr + kUnitVec32 - 1) / kUnitVec32;
+        if (wg0 < (int64_t)T * upr0) {
+            const int64_t t0 = wg0 / upr0;
+            const int64_t v = (wg0 - t0 * upr0) * kUnitVec32 + (threadIdx.x & 31);
+            if (v < vpr)
+                prefetch_l2(x + t0 * vpr + v);
+        }
+    }
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -217,6 +238,19 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                         float* __restrict__ recv_scales, int64_t scales_ld, int64_t cap_rows,
                         int32_t* err)
 {
+    {   // this warp's first unit of x into L2 while the previous kernel finishes
+        const int64_t wg0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+        const int64_t vpr0 = H / 16;
+        const int64_t upr0 = (vpr0 + kUnitVec32Fp8 - 1) / kUnitVec32Fp8;
+        if (wg0 < (int64_t)T * upr0) {
+            const int64_t t0 = wg0 / upr0;
+            const int64_t v = (wg0 - t0 * upr0) * kUnitVec32Fp8 + (threadIdx.x & 31);
+            if (v < vpr0)
+                prefetch_l2(x + t0 * vpr0 + v);
+            if (v + 32 < vpr0)
+                prefetch_l2(x + t0 * vpr0 + v + 32);
+        }
+    }
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
