@@ -273,7 +273,9 @@ def _range(name):
     return torch.cuda.nvtx.range(name)
 
 
-def gpu_step(s, ev=None):
+def gpu_step(s, ev=None, skip=None):
+    """One step: layout, dispatch, combine (skip: leave one of the last two
+    out, for the marginal timing)."""
     import combine_ep_layout_08_b200 as ep
 
     h, w = s["h"], s["w"]
@@ -283,12 +285,14 @@ def gpu_step(s, ev=None):
         ep.ep_layout(h, s["idx"])
     if ev is not None:
         ev[1].record()
-    with _range("ep_dispatch"):
-        ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
+    if skip != "dispatch":
+        with _range("ep_dispatch"):
+            ep.ep_dispatch(h, s["x"], w.fmt, recv_x=s["recv"], recv_scales=s["scales"])
     if ev is not None:
         ev[2].record()
-    with _range("ep_combine"):
-        ep.ep_combine(h, s["y"], s["wt"], out=s["out"])
+    if skip != "combine":
+        with _range("ep_combine"):
+            ep.ep_combine(h, s["y"], s["wt"], out=s["out"])
     if ev is not None:
         ev[3].record()
 
@@ -318,6 +322,17 @@ def time_gpu(s, steps, warmup, flush, barrier):
     for i in range(steps):
         flush()
         gpu_step(s, evs[i])
+    # the step without one of the two kernels, events at its ends only: what
+    # each kernel adds to the step when its launch overlaps its neighbours'
+    part = {}
+    for name, skip in (("no_dispatch", "dispatch"), ("no_combine", "combine")):
+        pe = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            flush()
+            pe[i][0].record()
+            gpu_step(s, skip=skip)
+            pe[i][1].record()
+        part[name] = pe
     torch.cuda.synchronize()
     t1 = time.time()
     barrier()
@@ -326,7 +341,22 @@ def time_gpu(s, steps, warmup, flush, barrier):
     dis = [e[1].elapsed_time(e[2]) for e in evs]
     com = [e[2].elapsed_time(e[3]) for e in evs]
     split = [e[0].elapsed_time(e[3]) for e in evs]
-    return dict(layout=lay, dispatch=dis, combine=com, step=tot, step_split=split, wall=(t0, t1))
+    nod = [e[0].elapsed_time(e[1]) for e in part["no_dispatch"]]
+    noc = [e[0].elapsed_time(e[1]) for e in part["no_combine"]]
+    return dict(layout=lay, dispatch=dis, combine=com, step=tot, step_split=split,
+                step_no_dispatch=nod, step_no_combine=noc, wall=(t0, t1))
+
+
+def marginal(tm, d_bytes, c_bytes, agg=lambda v: v):
+    """What dispatch and combine each add to the step: the step time minus
+    the step without that kernel, both with events at the ends only."""
+    step = agg(statistics.mean(tm["step"]))
+    d = step - agg(statistics.mean(tm["step_no_dispatch"]))
+    c = step - agg(statistics.mean(tm["step_no_combine"]))
+    return {"dispatch_marginal_us": round(d * 1e3, 2),
+            "dispatch_marginal_GBps": round(d_bytes / (d / 1e3) / 1e9, 1) if d > 0 else None,
+            "combine_marginal_us": round(c * 1e3, 2),
+            "combine_marginal_GBps": round(c_bytes / (c / 1e3) / 1e9, 1) if c > 0 else None}
 
 
 def time_gpu_e2e(s, steps, warmup):
@@ -982,6 +1012,7 @@ def main():
     lay_ms = aggregate_max(statistics.mean(tm["layout"]))
     dis_ms = aggregate_max(statistics.mean(tm["dispatch"]))
     com_ms = aggregate_max(statistics.mean(tm["combine"]))
+    marg_main = marginal(tm, d_bytes, c_bytes, aggregate_max)  # every rank: collectives inside
     value = world * (d_bytes + c_bytes) / (step_ms / 1e3) / 1e9
 
     e2e = None
@@ -1018,7 +1049,8 @@ def main():
                    "combine_us": round(statistics.mean(t2["combine"]) * 1e3, 2),
                    "dispatch_GBps": round(db / (statistics.mean(t2["dispatch"]) / 1e3) / 1e9, 1),
                    "combine_GBps": round(cb / (statistics.mean(t2["combine"]) / 1e3) / 1e9, 1),
-                   "value_GBps": round((db + cb) / (statistics.mean(t2["step"]) / 1e3) / 1e9, 1)}
+                   "value_GBps": round((db + cb) / (statistics.mean(t2["step"]) / 1e3) / 1e9, 1),
+                   **marginal(t2, db, cb)}
             if name == "decode":
                 # per step inside a graph of 20 steps; one-step graphs as well
                 ent["graph_step_us"] = round(graph_latency_us(s2, reps=50, inner=20), 2)
@@ -1074,9 +1106,12 @@ def main():
                         "combine_p50_p95_p99_us": [round(np.percentile(tm["combine"], q) * 1e3, 2)
                                                    for q in (50, 95, 99)],
                         "split_step_us": round(statistics.mean(tm["step_split"]) * 1e3, 2),
+                        **marg_main,
                         "note": "per-kernel times from a second pass of the same steps with "
                                 "events between the kernels (split_step_us is that pass's step); "
-                                "value and ms_per_step come from events at the step's ends only"},
+                                "value and ms_per_step come from events at the step's ends only; "
+                                "*_marginal_*: the step time minus the step without that kernel "
+                                "(events at the ends only), what the kernel adds to the step"},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,

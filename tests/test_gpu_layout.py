@@ -59,6 +59,10 @@ FUZZ = [
     (1000, 2048, 8, 8, 128, 0.0, True),    # E above the one-CTA limit
     (5000, 8192, 64, 4, 128, 0.0, True),   # tile counts too big for shared memory: 3 kernels
     (3000, 256, 8, 8, 3, 0.1, True),       # block_m = 3: pad ranges not 4-aligned
+    (40000, 256, 8, 8, 128, 0.02, True),   # tile layout, 34 tokens per warp (> 32)
+    (2000, 20, 4, 4, 16, 0.1, True),       # tile layout, E not a multiple of 8
+    (9000, 1024, 16, 6, 128, 0.0, True),   # tile layout at E = 1024, k = 6
+    (150000, 64, 8, 2, 128, 0.0, True),    # tile layout, 127 tokens per warp, 13 groups
 ]
 
 
