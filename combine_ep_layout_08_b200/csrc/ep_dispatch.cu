@@ -194,10 +194,10 @@ dispatch_fp8_kernel(const uint4* __restrict__ x, int T, int k, int H,
             } else {
                 const float s = __fdiv_rn(m, 448.0f);
                 sc[i] = s;
-                q[i].x = e4m3x4(__fdiv_rn(f[0], s), __fdiv_rn(f[1], s), __fdiv_rn(f[2], s),
-                                __fdiv_rn(f[3], s));
-                q[i].y = e4m3x4(__fdiv_rn(f[4], s), __fdiv_rn(f[5], s), __fdiv_rn(f[6], s),
-                                __fdiv_rn(f[7], s));
+                float v[8];
+                units::div_n_by_scale<8>(f, s, v);
+                q[i].x = e4m3x4(v[0], v[1], v[2], v[3]);
+                q[i].y = e4m3x4(v[4], v[5], v[6], v[7]);
             }
         }
         // lane L < 8 takes the scale of block 2 (L/2) + (L%2) of the unit

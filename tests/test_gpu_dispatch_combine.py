@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from workloads import make_workload, make_x, random_topk
+from workloads import make_workload, make_x, make_x_scale_sweep, random_topk
 
 pytestmark = pytest.mark.gpu
 
@@ -144,6 +144,15 @@ def test_dispatch_fp8_special_values(oracle):
     dispatch_case(oracle, x, idx, E, R, "fp8")
 
 
+@pytest.mark.parametrize("x_offset", [0, 8])  # the 32-byte and the 16-byte kernels
+def test_dispatch_fp8_scale_sweep(oracle, x_offset):
+    rng = np.random.default_rng(2024 + x_offset)
+    T, H, E, R, k = 512, 7168, 16, 4, 2
+    x = make_x_scale_sweep(T, H, rng)
+    idx, _ = random_topk(T, E, k, rng)
+    dispatch_case(oracle, x, idx, E, R, "fp8", x_offset=x_offset)
+
+
 def test_dispatch_capacity_overflow_is_reported_and_bounded(oracle):
     import combine_ep_layout_08_b200 as ep
     from gpu_util import DEV, bits_to_bf16
@@ -213,6 +222,37 @@ def test_combine_random_y(oracle, T, H, E, R, k, p_unused):
     P = oracle.layout(idx, E, R).total_rows
     y = make_x(max(P, 1), H, rng)
     combine_case(oracle, y, w, idx, E, R)
+
+
+def test_combine_right_after_a_new_layout(oracle):
+    """Layouts of two different routings alternate on one handle with no
+    synchronisation, each followed at once by a combine: a combine starts
+    while the layout ahead of it still writes dst_row, so the rows it
+    prefetches before its dependent-launch wait may be the previous
+    routing's.  Every result must be the one of its own routing (bit-exact)."""
+    import combine_ep_layout_08_b200 as ep
+    from gpu_util import DEV, bf16_to_bits, bits_to_bf16
+
+    rng = np.random.default_rng(5150)
+    T, H, E, R, k = 128, 7168, 256, 16, 8
+    idx_a, w_a = random_topk(T, E, k, rng)
+    idx_b, w_b = random_topk(T, E, k, rng)
+    idx_b[::7] = idx_a[::7]  # some tokens keep their rows, most move
+    lays = [oracle.layout(idx_a, E, R), oracle.layout(idx_b, E, R)]
+    P = max(l.total_rows for l in lays)
+    y_bits = make_x(P, H, rng)
+    y = bits_to_bf16(y_bits)
+    h = _handle(T, k, E, R)
+    idx_d = [torch.from_numpy(i).to(DEV) for i in (idx_a, idx_b)]
+    w_d = [torch.from_numpy(w).to(DEV) for w in (w_a, w_b)]
+    outs = [torch.empty((T, H), dtype=torch.bfloat16, device=DEV) for _ in range(20)]
+    for i in range(20):
+        ep.ep_layout(h, idx_d[i % 2])
+        ep.ep_combine(h, y, w_d[i % 2], out=outs[i])
+    ep.ep_handle_check(h)
+    exp = [oracle.combine(y_bits, w, l.dst_row) for w, l in zip((w_a, w_b), lays)]
+    for i in range(20):
+        assert np.array_equal(bf16_to_bits(outs[i]), exp[i % 2]), "combine %d" % i
 
 
 def test_combine_cancellation_and_fma_cases(oracle):

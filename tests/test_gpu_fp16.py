@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from workloads import make_x_fp16, random_topk
+from workloads import make_x_fp16, make_x_scale_sweep, random_topk
 
 pytestmark = pytest.mark.gpu
 
@@ -134,6 +134,33 @@ def test_fp8_of_fp16_rows(oracle, fmt, T, H, E, R, k, x_offset):
     got = recv.view(torch.uint8).cpu().numpy()
     assert np.array_equal(got[rows], q_ref[rows])
     assert _guards_ok(full)
+
+
+@pytest.mark.parametrize("x_offset", [0, 8])  # the 32-byte and the 16-byte kernels
+def test_fp8_of_fp16_scale_sweep(oracle, x_offset):
+    """Block maxima over every binade of binary16 (all of them take the
+    corrected-reciprocal division): codes and scales bit-exact."""
+    import combine_ep_layout_08_b200 as ep
+
+    T, H, E, R, k = 256, 7168, 16, 4, 2
+    x = make_x_scale_sweep(T, H, np.random.default_rng(99 + x_offset), fmt="fp16")
+    h, lay, x, idx, _, _ = _setup(oracle, T, H, E, R, k, 5, p_unused=0.0, x_bits=x)
+    P = lay.total_rows
+    if x_offset:
+        base = torch.empty(T * H + x_offset, dtype=torch.float16, device="cuda:0")
+        xd = base[x_offset:].view(T, H)
+        xd.copy_(_f16(x))
+    else:
+        xd = _f16(x)
+    rows = lay.dst_row[lay.dst_row >= 0]
+    full, recv = _guarded(P, H, torch.float8_e4m3fn)
+    sfull, sc = _guarded(P, H // 128, torch.float32)
+    ep.ep_dispatch(h, xd, "fp8", recv_x=recv, recv_scales=sc)
+    ep.ep_handle_check(h)
+    q_ref, s_ref = oracle.dispatch_fp8(x, lay.dst_row, P, dtype="fp16")
+    assert np.array_equal(sc.cpu().numpy()[rows].view(np.uint32), s_ref[rows].view(np.uint32))
+    assert np.array_equal(recv.view(torch.uint8).cpu().numpy()[rows], q_ref[rows])
+    assert _guards_ok(full) and _guards_ok(sfull)
 
 
 def test_fp8_of_fp16_special_values(oracle):

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from workloads import make_workload, make_x, random_topk
+from workloads import make_workload, make_x, make_x_scale_sweep, random_topk
 
 pytestmark = pytest.mark.gpu
 SENT = 0x5A
@@ -77,6 +77,15 @@ def test_fused_shapes(oracle, T, H, E, R, k, fmt, p_unused):
     x = make_x(T, H, rng)
     idx, _ = random_topk(T, E, k, rng, p_unused=p_unused)
     fused_case(oracle, x, idx, E, R, fmt)
+
+
+@pytest.mark.parametrize("T,H", [(128, 7168),   # one CTA per token (decode kernel)
+                                 (300, 2048)])  # the replicated-layout kernel
+def test_fused_fp8_scale_sweep(oracle, T, H):
+    rng = np.random.default_rng(T + H)
+    x = make_x_scale_sweep(T, H, rng)
+    idx, _ = random_topk(T, 256, 8, rng)
+    fused_case(oracle, x, idx, 256, 16, "fp8")
 
 
 def test_fused_errors(oracle):

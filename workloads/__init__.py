@@ -20,8 +20,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-__all__ = ["CONFIGS", "Workload", "make_workload", "make_x", "make_x_fp16", "route",
-           "expert_scale_table", "random_topk"]
+__all__ = ["CONFIGS", "Workload", "make_workload", "make_x", "make_x_fp16", "make_x_scale_sweep",
+           "route", "expert_scale_table", "random_topk"]
 
 # name -> shape and recipe.  fmt is the dispatch format; combine is BF16 always.
 CONFIGS = {
@@ -79,6 +79,24 @@ def make_x_fp16(T: int, H: int, rng: np.random.Generator) -> np.ndarray:
     """Hidden states for FP16 inputs: N(0,1) in fp32, cast to IEEE binary16 by NumPy;
     returned as bits."""
     return rng.standard_normal((T, H), dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def make_x_scale_sweep(T: int, H: int, rng: np.random.Generator, fmt: str = "bf16") -> np.ndarray:
+    """Hidden states (bits) whose 128-channel blocks have their largest
+    magnitude spread over every binade of the 16-bit format (encodings 1 to
+    the largest finite one, plus, for bf16, every encoding from 0x1180 to
+    0x1280, magnitudes near 448 * 2^-100); each block's other elements are
+    random encodings below its largest, every sign random.  H % 128 == 0."""
+    top = 0x7F7F if fmt == "bf16" else 0x7BFF
+    nb = T * H // 128
+    near = np.arange(0x1180, 0x1281) if fmt == "bf16" else np.zeros(0, np.int64)
+    spread = np.linspace(1, top, max(nb - near.size, 1)).astype(np.int64)
+    amax = np.concatenate([spread, near])[:nb]
+    rng.shuffle(amax)
+    blocks = (rng.random((nb, 128)) * (amax[:, None] + 1)).astype(np.int64)
+    blocks[np.arange(nb), rng.integers(0, 128, nb)] = amax
+    blocks |= rng.integers(0, 2, (nb, 128)) << 15
+    return blocks.astype(np.uint16).reshape(T, H)
 
 
 def expert_scale_table(E: int, identity: bool = False) -> np.ndarray:
