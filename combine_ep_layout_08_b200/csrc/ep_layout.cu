@@ -865,16 +865,17 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
 //     1  entries loaded (up to kR per thread) and the token's experts
 //        published (after the counters were zeroed, before the
 //        dependent-launch wait);
-//     2  per slot, each warp's count of equal experts before it (one ballot
-//        per slot and round), and the histogram (shared atomics: order-free
-//        sums);
-//     3  padded and plain exclusive scans over the experts (thread e = expert e);
-//     4  the token's positions (warp w sums the counts of slots w, w + 16),
-//        released to the dispatch group at once; then is_token_in_rank, the
-//        pad rows of the experts this CTA owns, (the last CTA) the totals and
-//        offsets, and for R > 32 the tokens on rank c (c + G, ...) counted
-//        in CTA c, the entries that are their token's first slot on that
-//        rank;
+//     2  the histogram of all entries and of those of the tokens before
+//        this CTA's token (shared atomics: order-free sums);
+//     3  the token's positions (warp w takes slots w, w + 16: the padded
+//        counts of the experts below the slot's, the slot's expert's
+//        entries before the token, its equal slots before it), released to
+//        the dispatch group at once;
+//     4  padded and plain exclusive scans over the experts (thread e =
+//        expert e); then is_token_in_rank, the pad rows of the experts this
+//        CTA owns, (the leader) the totals and offsets, and for R > 32 the
+//        tokens on rank c (c + G, ...) counted in CTA c, the entries that
+//        are their token's first slot on that rank;
 //   dispatch warps 16-31 (named barrier 2): warp 16 + p loads 512-channel
 //     piece p of the token's row before the layout starts and quantises it
 //     (FP8) while the layout warps work; for R <= 32 one CTA's dispatch
@@ -882,7 +883,7 @@ layout_small_kernel(const int64_t* __restrict__ topk_idx, int T, int k, int E, i
 //     token, one ballot per rank);
 //   5  (barrier 3: the layout warps that wrote positions and the dispatch
 //      group) the rows stored to the k positions, while the layout group
-//      finishes the rest of step 4.
+//      does step 4.
 // When T + 1 CTAs fit on the SMs, an extra CTA without a token of its own
 // takes the leader's and the counter's work, so that no token's stores wait
 // for them.
@@ -931,10 +932,9 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
                               int32_t* err, FusedDispatch fd)
 {
     extern __shared__ __align__(16) int32_t ent[];  // [T k]
-    __shared__ int32_t cnt[kDecMaxE];
+    __shared__ int32_t cnt[kDecMaxE], cnt_before[kDecMaxE];
     __shared__ int32_t off[kDecMaxE + 1], uoff[kDecMaxE + 1];
     __shared__ int32_t wsum[2][kDecLayoutWarps];
-    __shared__ int32_t part[32][EP_MAX_TOPK];  // rows 0..15 used
     __shared__ int32_t rpart[kDecLayoutWarps][32];  // per-warp tokens per rank (R <= 32)
     __shared__ int32_t tgt_e[EP_MAX_TOPK], tgt_pos[EP_MAX_TOPK];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -959,7 +959,10 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
 
     // 1
     if (layout_group)
-        for (int e = tid; e < E; e += kDecThreads) cnt[e] = 0;
+        for (int e = tid; e < E; e += kDecThreads) {
+            cnt[e] = 0;
+            cnt_before[e] = 0;
+        }
     pdl_wait();
     pdl_trigger();
     units::Vec32 cur[1];
@@ -997,29 +1000,44 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
             const int f = q * kDecThreads + tid;
             e_s[q] = f < nent ? ent[f] : -1;
         }
-        // per slot and round, one ballot of the warp's equal experts before it;
-        // lane j keeps slot j's count
-        if (has_token) {
-            int32_t mine = 0;
-            for (int j = 0; j < k; ++j) {
-                const int ej = tgt_e[j], fj = t * k + j;
-                int32_t c = 0;
-#pragma unroll
-                for (int q = 0; q < kR; ++q)
-                    c += __popc(__ballot_sync(kFull, e_s[q] == ej && q * kDecThreads + tid < fj));
-                if (lane == (j & 31))
-                    mine = c;
-            }
-            if (lane < k)
-                part[warp][lane] = mine;
-        }
+        // the histogram of all entries and of the entries of the tokens
+        // before t (shared atomics: order-free sums)
+        const int before = t * k;
 #pragma unroll
         for (int q = 0; q < kR; ++q)
-            if (e_s[q] >= 0)
+            if (e_s[q] >= 0) {
                 atomicAdd(&cnt[e_s[q]], 1);
+                if (q * kDecThreads + tid < before)
+                    atomicAdd(&cnt_before[e_s[q]], 1);
+            }
         named_sync(1, kDecThreads);
 
-        // 3: thread e owns expert e
+        // 3: the token's positions, released to the dispatch group at once.
+        // Warp w takes slots w, w + 16: slot j of expert e lands at the padded
+        // counts of the experts below e (summed here from the histogram; the
+        // full scans follow, off the stores' path), plus the entries of e in
+        // the tokens before t, plus the slots j' < j of token t with expert e.
+        if (warp < pos_warps && has_token) {
+            const int my_e = lane < k ? tgt_e[lane] : -1;
+            for (int j = warp; j < k; j += kDecLayoutWarps) {
+                const int e = tgt_e[j];
+                int32_t below = 0;
+#pragma unroll 4
+                for (int f = lane; f < e; f += 32) below += padded(cnt[f]);
+                below = __reduce_add_sync(kFull, below);
+                const int dup = __popc(__ballot_sync(kFull, lane < j && my_e == e));
+                if (lane == 0) {
+                    const int32_t p = e >= 0 ? below + cnt_before[e] + dup : -1;
+                    tgt_pos[j] = p;
+                    dst_row[(int64_t)t * k + j] = p;
+                    if (p >= 0)
+                        recv_src[p] = t;
+                }
+            }
+            named_sync_unaligned(3, release_threads);  // the positions are in shared memory
+        }
+
+        // 4: padded and plain exclusive scans, thread e owns expert e
         const int32_t c_e = tid < E ? cnt[tid] : 0, p_e = padded(c_e);
         int32_t pin = p_e, uin = c_e;
         for (int o = 1; o < 32; o <<= 1) {
@@ -1058,21 +1076,6 @@ decode_layout_dispatch_kernel(const int64_t* __restrict__ topk_idx, int T, int k
         }
         named_sync(1, kDecThreads);
 
-        // 4
-        if (warp < pos_warps && has_token) {
-            for (int j = warp; j < k; j += kDecLayoutWarps) {  // warp w: slots w, w + 16
-                const int e = tgt_e[j];
-                const int32_t c = __reduce_add_sync(kFull, lane < kDecLayoutWarps ? part[lane][j] : 0);
-                if (lane == 0) {
-                    const int32_t pos = e >= 0 ? off[e] + c : -1;
-                    tgt_pos[j] = pos;
-                    dst_row[(int64_t)t * k + j] = pos;
-                    if (pos >= 0)
-                        recv_src[pos] = t;
-                }
-            }
-            named_sync_unaligned(3, release_threads);  // the positions are in shared memory
-        }
         for (int r = tid; r < R && has_token; r += kDecThreads) {
             uint8_t hit = 0;
             for (int j = 0; j < k; ++j)
