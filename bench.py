@@ -274,15 +274,17 @@ def _range(name):
 
 
 def gpu_step(s, ev=None, skip=None):
-    """One step: layout, dispatch, combine (skip: leave one of the last two
-    out, for the marginal timing)."""
+    """One step: layout, dispatch, combine (skip: leave one of the three out,
+    for the marginal timing; without the layout, dispatch and combine use the
+    handle's layout of the same routing from the step before)."""
     import combine_ep_layout_08_b200 as ep
 
     h, w = s["h"], s["w"]
     if ev is not None:
         ev[0].record()
-    with _range("ep_layout"):
-        ep.ep_layout(h, s["idx"])
+    if skip != "layout":
+        with _range("ep_layout"):
+            ep.ep_layout(h, s["idx"])
     if ev is not None:
         ev[1].record()
     if skip != "dispatch":
@@ -322,10 +324,11 @@ def time_gpu(s, steps, warmup, flush, barrier):
     for i in range(steps):
         flush()
         gpu_step(s, evs[i])
-    # the step without one of the two kernels, events at its ends only: what
+    # the step without one of the three kernels, events at its ends only: what
     # each kernel adds to the step when its launch overlaps its neighbours'
     part = {}
-    for name, skip in (("no_dispatch", "dispatch"), ("no_combine", "combine")):
+    for name, skip in (("no_layout", "layout"), ("no_dispatch", "dispatch"),
+                       ("no_combine", "combine")):
         pe = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         for i in range(steps):
             flush()
@@ -341,19 +344,22 @@ def time_gpu(s, steps, warmup, flush, barrier):
     dis = [e[1].elapsed_time(e[2]) for e in evs]
     com = [e[2].elapsed_time(e[3]) for e in evs]
     split = [e[0].elapsed_time(e[3]) for e in evs]
+    nol = [e[0].elapsed_time(e[1]) for e in part["no_layout"]]
     nod = [e[0].elapsed_time(e[1]) for e in part["no_dispatch"]]
     noc = [e[0].elapsed_time(e[1]) for e in part["no_combine"]]
     return dict(layout=lay, dispatch=dis, combine=com, step=tot, step_split=split,
-                step_no_dispatch=nod, step_no_combine=noc, wall=(t0, t1))
+                step_no_layout=nol, step_no_dispatch=nod, step_no_combine=noc, wall=(t0, t1))
 
 
 def marginal(tm, d_bytes, c_bytes, agg=lambda v: v):
-    """What dispatch and combine each add to the step: the step time minus
-    the step without that kernel, both with events at the ends only."""
+    """What each kernel adds to the step: the step time minus the step
+    without that kernel, both with events at the ends only."""
     step = agg(statistics.mean(tm["step"]))
+    lay = step - agg(statistics.mean(tm["step_no_layout"]))
     d = step - agg(statistics.mean(tm["step_no_dispatch"]))
     c = step - agg(statistics.mean(tm["step_no_combine"]))
-    return {"dispatch_marginal_us": round(d * 1e3, 2),
+    return {"layout_marginal_us": round(lay * 1e3, 2),
+            "dispatch_marginal_us": round(d * 1e3, 2),
             "dispatch_marginal_GBps": round(d_bytes / (d / 1e3) / 1e9, 1) if d > 0 else None,
             "combine_marginal_us": round(c * 1e3, 2),
             "combine_marginal_GBps": round(c_bytes / (c / 1e3) / 1e9, 1) if c > 0 else None}
@@ -619,6 +625,8 @@ KERNEL_CASES = {
     "decode_fused": "the decode step in its fused form: ep_layout_dispatch (FP8) + ep_combine",
     "dispatch_2k": "layout + BF16 dispatch + combine on the first 2048 tokens of the 8k workload "
                    "(a quarter of the 8k launch; inputs and outputs larger than L2)",
+    "dispatch_fp8_dsv3": "layout + FP8 dispatch + combine on the DeepSeek-V3 shape (4096 tokens, "
+                         "group-limited top-8 of 256; inputs and outputs larger than L2)",
 }
 
 
@@ -643,11 +651,13 @@ def run_kernel_case(name, steps, dev):
         h, shape = s["h"], "decode: T=%d H=%d E=%d R=%d k=%d fp8" % (s["w"].T, s["w"].H, s["w"].E,
                                                                    s["w"].R, s["w"].k)
     else:
-        s = gpu_setup(MAIN_WORKLOAD, 0, dev, T=2048)
+        s = (gpu_setup(MAIN_WORKLOAD, 0, dev, T=2048) if name == "dispatch_2k"
+             else gpu_setup("dsv3", 0, dev))
+        torch.cuda.empty_cache()  # the set-up's temporaries: keep the device footprint small
         for _ in range(steps):
             gpu_step(s)
-        h, shape = s["h"], "T=%d H=%d E=%d R=%d k=%d bf16" % (s["w"].T, s["w"].H, s["w"].E,
-                                                              s["w"].R, s["w"].k)
+        h, shape = s["h"], "T=%d H=%d E=%d R=%d k=%d %s" % (s["w"].T, s["w"].H, s["w"].E,
+                                                            s["w"].R, s["w"].k, s["w"].fmt)
     torch.cuda.synchronize()
     ep.ep_handle_check(h)
     print("kernel case %s (%s), %d steps: %s" % (name, shape, steps, KERNEL_CASES[name]), flush=True)
