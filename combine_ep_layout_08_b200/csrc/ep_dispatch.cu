@@ -23,7 +23,12 @@
 // for rows that are not 32-byte multiples.  Before the dependent-launch wait
 // each warp of the main kernels prefetches its unit of x into L2 (x does not
 // depend on the layout; a prefetch returns no data), so the loads after the
-// wait find it there: measured 1.5 us less per launch at 8192 tokens.  The grid gives every warp one
+// wait find it there: measured 1.5 us less per launch at 8192 tokens.  The
+// first wave's warps also prefetch the x of the next few waves (about 36 MB,
+// evict_last) while the layout ahead still runs and HBM is otherwise idle:
+// 4-5 us less per step at 8192 tokens (BF16) and at the DeepSeek-V3 shape
+// (FP8); with the default L2 priority the row stores evicted those lines
+// before use and the step got slower.  The grid gives every warp one
 // unit (a grid-stride loop covers grids beyond kMaxGrid): measured on B200,
 // a persistent single wave, in which every warp loads and then stores in
 // lock step with all the others, reaches ~5.4 TB/s; two waves 5.8; one unit
@@ -60,22 +65,52 @@ __device__ __forceinline__ void prefetch_l2(const void* p)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// The same with the L2 eviction priority evict_last, so that the row stores
+// streaming through L2 meanwhile do not push the line out before it is read.
+__device__ __forceinline__ void prefetch_l2_last(const void* p)
+{
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
+// Before the dependent-launch wait: the x of this warp's first unit into L2,
+// and, for the warps of the first wave (warp index < stride), the units
+// stride, 2 stride, ..., waves x stride ahead of it, which the later waves
+// of the grid will read (evict_last).  A unit is kVecs 32-byte vectors per
+// lane of one token row (upr units per row).  Prefetches return no data:
+// the loads after the wait read the memory as it is then.
+template <int kVecs>
+__device__ __forceinline__ void prefetch_x(const Vec32* x, int64_t vpr, int64_t upr,
+                                           int64_t nunits, int64_t stride, int waves)
+{
+    const int64_t wg0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    for (int w = 0; w <= waves; ++w) {
+        if (w > 0 && wg0 >= stride)
+            break;
+        const int64_t u = wg0 + (int64_t)w * stride;
+        if (u >= nunits)
+            break;
+        const int64_t t = u / upr;
+        const int64_t v = (u - t * upr) * (32 * kVecs) + lane;
+#pragma unroll
+        for (int i = 0; i < kVecs; ++i)
+            if (v + 32 * i < vpr) {
+                if (w == 0)
+                    prefetch_l2(x + t * vpr + v + 32 * i);
+                else
+                    prefetch_l2_last(x + t * vpr + v + 32 * i);
+            }
+    }
+}
+
 // BF16 dispatch with 32-byte vectors; vpr = H / 16.
 __global__ void __launch_bounds__(kThreads, 8)
 dispatch_bf16_v32_kernel(const Vec32* __restrict__ x, int T, int k, int64_t vpr,
                          const int32_t* __restrict__ dst_row, Vec32* __restrict__ recv,
-                         int64_t cap_rows, int32_t* err)
+                         int64_t cap_rows, int32_t* err, int64_t pf_stride, int pf_waves)
 {
-    {   // this warp's first unit of x into L2 while the previous kernel finishes
-        const int64_t wg0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-        const int64_t upr0 = (vpr + kUnitVec32 - 1) / kUnitVec32;
-        if (wg0 < (int64_t)T * upr0) {
-            const int64_t t0 = wg0 / upr0;
-            const int64_t v = (wg0 - t0 * upr0) * kUnitVec32 + (threadIdx.x & 31);
-            if (v < vpr)
-                prefetch_l2(x + t0 * vpr + v);
-        }
-    }
+    const int64_t upr0 = (vpr + kUnitVec32 - 1) / kUnitVec32;
+    prefetch_x<1>(x, vpr, upr0, (int64_t)T * upr0, pf_stride, pf_waves);
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -236,20 +271,12 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
                         const int32_t* __restrict__ dst_row, uint8_t* __restrict__ recv_q,
                         float* __restrict__ recv_scales, int64_t scales_ld, int64_t cap_rows,
-                        int32_t* err)
+                        int32_t* err, int64_t pf_stride, int pf_waves)
 {
-    {   // this warp's first unit of x into L2 while the previous kernel finishes
-        const int64_t wg0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    {
         const int64_t vpr0 = H / 16;
         const int64_t upr0 = (vpr0 + kUnitVec32Fp8 - 1) / kUnitVec32Fp8;
-        if (wg0 < (int64_t)T * upr0) {
-            const int64_t t0 = wg0 / upr0;
-            const int64_t v = (wg0 - t0 * upr0) * kUnitVec32Fp8 + (threadIdx.x & 31);
-            if (v < vpr0)
-                prefetch_l2(x + t0 * vpr0 + v);
-            if (v + 32 < vpr0)
-                prefetch_l2(x + t0 * vpr0 + v + 32);
-        }
+        prefetch_x<units::kU32Fp8>(x, vpr0, upr0, (int64_t)T * upr0, pf_stride, pf_waves);
     }
     pdl_wait();
     pdl_trigger();
@@ -273,6 +300,29 @@ dispatch_fp8_v32_kernel(const Vec32* __restrict__ x, int T, int k, int H,
 
 bool aligned32(const void* p) { return ((uintptr_t)p & 31u) == 0; }
 
+// x bytes the first wave prefetches ahead (about what HBM delivers while the
+// layout kernel ahead of the dispatch runs; 29-39 MB measured best at the
+// 8k and DeepSeek-V3 shapes, 47 MB and more slower).
+constexpr int64_t kPrefetchBudget = 36ll << 20;
+
+// The first wave's size in warps (the CTAs resident per SM beside one CTA of
+// the kernel ahead, x the SMs) and how many waves ahead of it to prefetch.
+cudaError_t prefetch_plan(const void* kernel, int64_t unit_x_bytes, int64_t* stride, int* waves)
+{
+    int full = 0;
+    cudaError_t rc = persistent_grid(kernel, kThreads, 0, 1 << 16, &full);
+    if (rc != cudaSuccess)
+        return rc;
+    int dev = 0, sms = 1;
+    if ((rc = cudaGetDevice(&dev)) != cudaSuccess ||
+        (rc = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return rc;
+    const int64_t ctas = std::max<int64_t>(sms, full - sms);
+    *stride = ctas * (kThreads / 32);
+    *waves = (int)std::max<int64_t>(0, kPrefetchBudget / (*stride * unit_x_bytes) - 1);
+    return cudaSuccess;
+}
+
 // One unit per warp: ceil(units / warps per CTA) CTAs, capped at kMaxGrid.
 unsigned unit_grid(int64_t T, int64_t vec_per_row, int64_t unit_vec)
 {
@@ -288,10 +338,18 @@ cudaError_t launch_dispatch_bf16(const Handle& h, const void* x, int H, void* re
 {
     if (h.T == 0)
         return cudaSuccess;
-    if (H % 16 == 0 && aligned32(x) && aligned32(recv_x))
+    if (H % 16 == 0 && aligned32(x) && aligned32(recv_x)) {
+        int64_t pf_stride = 0;
+        int pf_waves = 0;
+        cudaError_t rc = prefetch_plan((const void*)dispatch_bf16_v32_kernel,
+                                       kUnitVec32 * (int64_t)sizeof(Vec32), &pf_stride, &pf_waves);
+        if (rc != cudaSuccess)
+            return rc;
         return launch_pdl(dispatch_bf16_v32_kernel, unit_grid(h.T, H / 16, kUnitVec32), kThreads,
                           0, s, static_cast<const Vec32*>(x), h.T, h.k, (int64_t)H / 16,
-                          h.dst_row, static_cast<Vec32*>(recv_x), cap_rows, h.err);
+                          h.dst_row, static_cast<Vec32*>(recv_x), cap_rows, h.err, pf_stride,
+                          pf_waves);
+    }
     return launch_pdl(dispatch_bf16_kernel, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
                       static_cast<const uint4*>(x), h.T, h.k, (int64_t)H / 8, h.dst_row,
                       static_cast<uint4*>(recv_x), cap_rows, h.err);
@@ -305,10 +363,16 @@ cudaError_t launch_dispatch_fp8(const Handle& h, const void* x, int H, void* rec
         return cudaSuccess;
     if (aligned32(x)) {
         auto kern = half ? dispatch_fp8_v32_kernel<true> : dispatch_fp8_v32_kernel<false>;
+        int64_t pf_stride = 0;
+        int pf_waves = 0;
+        cudaError_t rc = prefetch_plan((const void*)kern, kUnitVec32Fp8 * (int64_t)sizeof(Vec32),
+                                       &pf_stride, &pf_waves);
+        if (rc != cudaSuccess)
+            return rc;
         return launch_pdl(kern, unit_grid(h.T, H / 16, kUnitVec32Fp8), kThreads, 0, s,
                           static_cast<const Vec32*>(x), h.T, h.k, H, h.dst_row,
                           static_cast<uint8_t*>(recv_q), recv_scales, scales_ld, cap_rows,
-                          h.err);
+                          h.err, pf_stride, pf_waves);
     }
     auto kern = half ? dispatch_fp8_kernel<true> : dispatch_fp8_kernel<false>;
     return launch_pdl(kern, unit_grid(h.T, H / 8, kUnitVec), kThreads, 0, s,
