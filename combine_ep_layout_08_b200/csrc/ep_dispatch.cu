@@ -304,6 +304,7 @@ bool aligned32(const void* p) { return ((uintptr_t)p & 31u) == 0; }
 // layout kernel ahead of the dispatch runs; 29-39 MB measured best at the
 // 8k and DeepSeek-V3 shapes, 47 MB and more slower).
 constexpr int64_t kPrefetchBudget = 36ll << 20;
+constexpr int64_t kMaxPrefetchWaves = 8;  // bounds the loop where few CTAs fit per SM
 
 // The first wave's size in warps (the CTAs resident per SM beside one CTA of
 // the kernel ahead, x the SMs) and how many waves ahead of it to prefetch.
@@ -319,7 +320,8 @@ cudaError_t prefetch_plan(const void* kernel, int64_t unit_x_bytes, int64_t* str
         return rc;
     const int64_t ctas = std::max<int64_t>(sms, full - sms);
     *stride = ctas * (kThreads / 32);
-    *waves = (int)std::max<int64_t>(0, kPrefetchBudget / (*stride * unit_x_bytes) - 1);
+    *waves = (int)std::min<int64_t>(kMaxPrefetchWaves,
+                                    std::max<int64_t>(0, kPrefetchBudget / (*stride * unit_x_bytes) - 1));
     return cudaSuccess;
 }
 
