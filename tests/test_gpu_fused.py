@@ -88,6 +88,34 @@ def test_fused_fp8_scale_sweep(oracle, T, H):
     fused_case(oracle, x, idx, 256, 16, "fp8")
 
 
+def _decode_shapes(n, seed):
+    """Batches that take the one-CTA-per-token kernel (T <= 148, E <= 512):
+    duplicate experts in a token, unused slots, k up to 32, R above and
+    below 32, block_m not a power of two."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < n:
+        E = int(rng.choice([1, 2, 5, 16, 64, 100, 256, 320, 512]))
+        R = int(rng.choice([r for r in range(1, min(E, 64) + 1) if E % r == 0]))
+        k = int(rng.choice([1, 2, 3, 6, 8, 13, 32]))
+        T = int(rng.integers(1, 149))
+        B = int(rng.choice([1, 7, 64, 128]))
+        distinct = bool(rng.random() < 0.5) and k <= E
+        p_unused = float(rng.choice([0.0, 0.2]))
+        fmt = str(rng.choice(["bf16", "fp8"]))
+        H = int(rng.choice([128, 1024, 7168]))
+        out.append((T, H, E, R, k, B, distinct, p_unused, fmt))
+    return out
+
+
+@pytest.mark.parametrize("T,H,E,R,k,B,distinct,p_unused,fmt", _decode_shapes(24, 31337))
+def test_fused_decode_kernel_random_shapes(oracle, T, H, E, R, k, B, distinct, p_unused, fmt):
+    rng = np.random.default_rng(T * 13 + E * 3 + k)
+    x = make_x(T, H, rng)
+    idx, _ = random_topk(T, E, k, rng, distinct=distinct, p_unused=p_unused)
+    fused_case(oracle, x, idx, E, R, fmt, B=B)
+
+
 def test_fused_errors(oracle):
     import combine_ep_layout_08_b200 as ep
     from gpu_util import DEV, bits_to_bf16
