@@ -73,11 +73,13 @@ ep_status_t fail_message(ep_status_t st, const char* what);
 bool carve_workspace(int max_tokens, int k, int E, int R, int block_m, Carve* c);
 
 // Programmatic dependent launch (sm_90+): every kernel of the library is
-// launched with programmatic stream serialization allowed, starts with
+// launched with programmatic stream serialization allowed and calls
 // pdl_wait() -- it returns once the preceding kernel in the stream has
 // completed and its memory is visible -- and then pdl_trigger(), which lets
-// the next kernel's CTAs be scheduled while this one drains.  Nothing is
-// read or written before pdl_wait(), so a kernel may follow any other work.
+// the next kernel's CTAs be scheduled while this one drains.  Before
+// pdl_wait() a kernel writes nothing but its own shared memory and issues
+// nothing but L2 prefetch hints (whose addresses may come from a read whose
+// value is used for nothing else), so a kernel may follow any other work.
 // 16-bit input values packed two to a 32-bit word: bfloat16 (kHalf = false,
 // the upper half of a binary32, widened by a shift) or IEEE binary16
 // (kHalf = true, widened exactly by the conversion instruction); and binary32
