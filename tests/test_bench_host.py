@@ -62,6 +62,24 @@ def test_aggregate_max_single_process_is_identity():
     assert bench.aggregate_max(1.5) == 1.5
 
 
+def test_marginal_cost_is_the_step_minus_the_step_without_the_kernel():
+    # per-step times in ms, as time_gpu returns them
+    tm = {"step": [0.330, 0.334], "step_no_layout": [0.325, 0.325],
+          "step_no_dispatch": [0.172, 0.174], "step_no_combine": [0.170, 0.172]}
+    m = bench.marginal(tm, 1056964608, 1056964608)
+    assert m["layout_marginal_us"] == pytest.approx(7.0)
+    assert m["dispatch_marginal_us"] == pytest.approx(159.0)
+    assert m["combine_marginal_us"] == pytest.approx(161.0)
+    assert m["dispatch_marginal_GBps"] == pytest.approx(1056964608 / 159.0e-6 / 1e9, rel=1e-3)
+    # the aggregate (max over ranks) is applied to each mean before the difference
+    seen = []
+    bench.marginal(tm, 1, 1, agg=lambda v: seen.append(v) or v)
+    assert len(seen) == 4
+    # a kernel that adds nothing has no rate
+    tm["step_no_combine"] = tm["step"]
+    assert bench.marginal(tm, 1, 1)["combine_marginal_GBps"] is None
+
+
 def test_kernel_hash_is_stable():
     for k in ("dispatch_bf16_v32_kernel", "combine_kernel"):
         assert bench.kernel_source_hash(k) == bench.kernel_source_hash(k)
